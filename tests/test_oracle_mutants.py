@@ -1,0 +1,67 @@
+"""The oracle's pins are sensitive: plant one plausible mistake at a time in a copy of the
+oracle (on the CPU), rebuild it, and check that at least one pin in test_oracle_pins fails.
+
+Each mutation is a mistake someone writing the Sparse GQA definition could make: a reversed
+tie rule, the own block not counted in the budget, a lost causal limit, the wrong softmax
+scale, a flipped gate sign, an off-by-one in the candidate range, a dropped term in the block
+mean, an interleaved head->group mapping, or the wrong group's index query.
+"""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+import tests.test_oracle_pins as pins
+
+MUTANTS = {
+    "tie_to_higher_block": ("return a.s > b.s || (a.s == b.s && a.j < b.j);",
+                            "return a.s > b.s || (a.s == b.s && a.j > b.j);"),
+    "own_block_not_in_budget": ("const int m = std::min(Kb - 1, c);", "const int m = std::min(Kb, c);"),
+    "no_causal_limit": ("u < (j + 1) * dm->B && u <= t;", "u < (j + 1) * dm->B;"),
+    "scale_by_index_dim": ("1.0 / std::sqrt((double)d);", "1.0 / std::sqrt((double)dm->d_idx);"),
+    "gate_sign": ("std::exp(-gl)", "std::exp(gl)"),
+    "complete_own_block_is_candidate": ("const int c = t / dm->B;                  //",
+                                        "const int c = (t + 1) / dm->B;            //"),
+    "dropped_term_in_mean": ("for (int r = 0; r < dm->B; ++r)", "for (int r = 0; r < dm->B - 1 + (dm->B == 1); ++r)"),
+    "interleaved_heads": ("const int h = (int)(rh % dm->Hq), g = h / R;\n    const long b = rows_bt[2 * row];\n    const int t = rows_bt[2 * row + 1];\n    const int32_t* S",
+                          "const int h = (int)(rh % dm->Hq), g = h % dm->G;\n    const long b = rows_bt[2 * row];\n    const int t = rows_bt[2 * row + 1];\n    const int32_t* S"),
+    "wrong_group_query": ("q_idx + rg * dm->d_idx", "q_idx + row * dm->G * dm->d_idx"),
+}
+
+PIN_CALLS = [
+    lambda: pins.test_brute_force_small(None, 8, 40),
+    lambda: pins.test_brute_force_small(None, 1, 13),
+    lambda: pins.test_brute_force_batch2_uneven(None),
+    lambda: pins.test_dense_reduction_matches_sdpa(None, 96, 8, 8, 2, 16),
+    lambda: pins.test_hand_worked_example(None),
+    lambda: pins.test_compress_closed_forms(None),
+    lambda: pins.test_first_token_is_gated_v0(None),
+    lambda: pins.test_selection_invariants(None, 8, 24),
+    lambda: pins.test_exact_ties_go_to_lower_block(None),
+]
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(tmp_path, name):
+    old, new = MUTANTS[name]
+    src = open(oracle.SRC).read()
+    assert src.count(old) >= 1, f"mutation anchor not found: {name}"
+    mutated = src.replace(old, new)
+    cpp = tmp_path / "mut.cpp"
+    so = tmp_path / "libmut.so"
+    cpp.write_text(mutated)
+    subprocess.run(["g++", "-O2", "-fopenmp", "-ffp-contract=off", "-shared", "-fPIC", "-o", str(so), str(cpp)],
+                   check=True)
+    saved = oracle._lib
+    oracle._lib = oracle.load(str(so))
+    caught = []
+    try:
+        for call in PIN_CALLS:
+            try:
+                call()
+            except (AssertionError, ValueError) as e:
+                caught.append(type(e).__name__)
+    finally:
+        oracle._lib = saved
+    assert caught, f"no pin caught mutant {name}"
