@@ -1,0 +1,478 @@
+#!/usr/bin/env python
+"""Sparse GQA benchmark on B200: prefill tokens/s at 128K (B=8, k=4096), decode tok/s at 1M.
+
+One step is one pass of the whole layer (block-key compression, per-group block selection,
+gated attention over the selected tokens) over one 131072-token sequence per GPU, inputs
+resident in HBM (q, gate and out alone are 3.2 GB, far above the 126 MB L2, so no flush is
+needed between steps). Launch:
+
+    python bench.py [--gpus 1] [--steps 5] [--warmup 3]
+    python -m torch.distributed.run --nproc-per-node N ... bench.py --gpus N ...   (one sequence per rank)
+    python bench.py --impl reference ...   (the fp64 CPU oracle on a bounded sample, host cores)
+
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from sgqa_inputs import CONFIGS, DECODE_NEW, gen_rows  # noqa: E402
+
+METRIC = "Sparse GQA prefill tokens/s at 128K (B=8,k=4096); decode tok/s at 1M ctx"
+CLOCK_FIELDS = ["pci.bus_id", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+                "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+                "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "sm_max_mhz": d.get("sm_max_mhz", 1965.0),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0,
+            "source": "fallback"}
+
+
+# ---- analytic work counts (the definition's, not the kernels') -------------------------------
+
+def work_counts(cfg):
+    """Scored candidates, attended (query, group, token) visits and byte streams of one pass."""
+    T, B, Kb = cfg.T, cfg.B, cfg.Kb
+    t = np.arange(T, dtype=np.int64)
+    c = t // B
+    scored = int(c.sum()) * cfg.G * cfg.batch
+    nsel = np.minimum(Kb, c + 1)
+    visits_per_t = (nsel - 1) * B + (t % B) + 1
+    visits = int(visits_per_t.sum()) * cfg.G * cfg.batch
+    R = cfg.Hq // cfg.G
+    nblk = T // B
+    return {
+        "scored": scored,
+        "index_flops": 2 * cfg.d_idx * scored,
+        "visits": visits,
+        "attn_flops": 4 * cfg.d * R * visits,
+        "gather_bytes": visits * 2 * cfg.d * 2,
+        "qgo_bytes": 3 * cfg.batch * T * cfg.Hq * cfg.d * 2,
+        "sel_bytes": cfg.batch * T * cfg.G * Kb * 4,
+        "kv_bytes": 2 * cfg.batch * T * cfg.G * cfg.d * 2,
+        "compress_bytes": cfg.batch * T * cfg.d_idx * 2 + cfg.batch * nblk * cfg.d_idx * 4,
+    }
+
+
+# ---- clocks sampled during the timed region -------------------------------------------------
+
+class ClockSampler:
+    def __init__(self, bus_id: int | None):
+        self.bus_id = bus_id
+        self.f = tempfile.NamedTemporaryFile(mode="w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={','.join(CLOCK_FIELDS)}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                                      stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.flush()
+        lines = open(self.f.name).read().strip().splitlines()
+        os.unlink(self.f.name)
+        sm, mx, reasons = [], [], set()
+        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < len(CLOCK_FIELDS):
+                continue
+            try:
+                bus = int(f[0].split(":")[1], 16)
+            except (IndexError, ValueError):
+                bus = None
+            if self.bus_id is not None and bus is not None and bus != self.bus_id:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names[1:], f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ---- distributed plumbing --------------------------------------------------------------------
+
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---- the CPU oracle on a bounded sample (cpu_baseline and the reference arm) ------------------
+
+def oracle_inputs_host(cfg, rows):
+    """Host bf16 inputs for the oracle: whole k, v, k_idx of sequence 0, the sampled rows' q,
+    q_idx, gate (made by the shared seeded generator on the host)."""
+    b = 0
+    t_all = np.arange(cfg.T)
+    full = {}
+    for n in ("k", "v", "k_idx"):
+        parts = [gen_rows(cfg, n, b, t_all[i:i + 8192]) for i in range(0, cfg.T, 8192)]
+        full[n] = np.concatenate(parts).reshape((1, cfg.T, -1))
+    ts = rows[:, 1]
+    part = {n: gen_rows(cfg, n, b, ts) for n in ("q", "q_idx", "gate")}
+    return full, part
+
+
+def oracle_sample_time(cfg, stride, full, part, rows):
+    import oracle
+    dm = oracle.dims(1, cfg.T, cfg.Hq, cfg.G, cfg.d, cfg.d_idx, cfg.B, cfg.k)
+    t0 = time.perf_counter()
+    kbar = oracle.compress(dm, full["k_idx"])
+    sel, _, _ = oracle.select(dm, kbar, rows, part["q_idx"])
+    oracle.attend(dm, rows, part["q"], full["k"], full["v"], part["gate"], sel)
+    return time.perf_counter() - t0
+
+
+def to_host(t) -> np.ndarray:
+    import torch
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def sample_rows_strided(cfg, stride, offset=0):
+    ts = np.arange(offset % stride, cfg.T, stride, dtype=np.int32)
+    return np.stack([np.zeros_like(ts), ts], axis=1)
+
+
+# ---- our arm ---------------------------------------------------------------------------------
+
+def run_ours(args, world, rank):
+    import torch
+    import block_sparse_long_kbar_b200 as sg
+    from sgqa_inputs import gen_device
+    cfg = CONFIGS[args.config]
+    shape_of = lambda c, n, **kw: c.shape(n, **kw)
+    peaks = load_peaks()
+    dims = sg.sgqa_dims.of(cfg)
+    s = torch.cuda.Stream()
+    dev = {}
+    for n in ("q", "k", "v", "gate", "q_idx", "k_idx"):
+        dev[n] = torch.empty(shape_of(cfg, n), dtype=torch.bfloat16, device="cuda")
+        gen_device(cfg, n, dev[n])
+    out = torch.empty(shape_of(cfg, "q"), dtype=torch.bfloat16, device="cuda")
+    sel = torch.empty((cfg.batch, cfg.T, cfg.G, cfg.Kb), dtype=torch.int32, device="cuda")
+    kbar = torch.empty((cfg.batch, cfg.T // cfg.B, cfg.d_idx), dtype=torch.float32, device="cuda")
+    ws = sg.alloc_workspace(sg.sgqa_workspace_size(dims))
+    sg.sgqa_reset_device_status(ws)
+    torch.cuda.synchronize()
+
+    def step():
+        sg.sgqa_forward(dims, dev["q"], dev["k"], dev["v"], dev["q_idx"], dev["k_idx"], dev["gate"], out, ws,
+                        sel_out=sel, stream=s)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    bus = getattr(torch.cuda.get_device_properties(torch.cuda.current_device()), "pci_bus_id", None)
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(bus)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(args.steps):
+        step()
+    e1.record(s)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    status = sg.sgqa_get_device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+    tokens_step = world * cfg.batch * cfg.T
+    value = tokens_step / (ms / 1e3)
+
+    # per-stage times: the same kernels through the per-stage entry points, events on the launch stream
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    st = {"compress": [], "select": [], "attend": []}
+    for _ in range(args.steps):
+        ev[0].record(s)
+        sg.sgqa_compress_keys(dims, dev["k_idx"], kbar, ws, stream=s)
+        ev[1].record(s)
+        sg.sgqa_select(dims, dev["q_idx"], kbar, sel, ws, stream=s)
+        ev[2].record(s)
+        sg.sgqa_attend(dims, dev["q"], dev["k"], dev["v"], dev["gate"], sel, out, ws, stream=s)
+        ev[3].record(s)
+        torch.cuda.synchronize()
+        for i, k in enumerate(st):
+            st[k].append(ev[i].elapsed_time(ev[i + 1]))
+    stage_ms = {k: statistics.mean(v) for k, v in st.items()}
+    wc = work_counts(cfg)
+    sm_mhz = (clocks or {}).get("sm_mhz") or peaks["sm_max_mhz"]
+    fp32_peak_tflops = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+    stage_roof = {
+        "compress": {"bound": "hbm", "achieved": wc["compress_bytes"] / (stage_ms["compress"] / 1e3) / 1e9,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s"},
+        "select": {"bound": "alu", "achieved": wc["index_flops"] / (stage_ms["select"] / 1e3) / 1e12,
+                   "peak": fp32_peak_tflops, "unit": "TFLOP/s"},
+        "attend": {"bound": "tensor", "achieved": wc["attn_flops"] / (stage_ms["attend"] / 1e3) / 1e12,
+                   "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s"},
+    }
+    for k, r in stage_roof.items():
+        r["frac"] = r["achieved"] / r["peak"]
+        r["ms"] = stage_ms[k]
+    dominant = max(stage_ms, key=stage_ms.get)
+    roof = dict(stage_roof[dominant])
+    roof.pop("ms")
+    roof["kernel"] = dominant
+    roof["traffic"] = None
+    roof["peak_source"] = peaks["source"]
+
+    # end to end through the C ABI with host buffers: H2D of the step's inputs, D2H of its output
+    host = {n: torch.empty(dev[n].shape, dtype=torch.bfloat16, pin_memory=True) for n in dev}
+    for n in dev:
+        host[n].copy_(dev[n])
+    out_h = torch.empty(out.shape, dtype=torch.bfloat16, pin_memory=True)
+    h2d = sum(t.numel() * 2 for t in host.values())
+    d2h = out.numel() * 2
+    torch.cuda.synchronize()
+
+    def e2e_step():
+        with torch.cuda.stream(s):
+            for n in dev:
+                dev[n].copy_(host[n], non_blocking=True)
+        step()
+        with torch.cuda.stream(s):
+            out_h.copy_(out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0.record(s)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(s)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+
+    gather_gbs = wc["gather_bytes"] / (stage_ms["attend"] / 1e3) / 1e9
+    result = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded topic-structured generator)",
+        "config": {"workload": f"prefill {cfg.name}: batch {cfg.batch} per GPU, T={cfg.T}, Hq={cfg.Hq}, G={cfg.G}, "
+                               f"d={cfg.d}, d_idx={cfg.d_idx}, B={cfg.B}, k={cfg.k}, topic span {cfg.span}, "
+                               f"seed {cfg.seed}",
+                   "global_batch": world * cfg.batch, "seq_len": cfg.T, "parallelism": f"dp{world} (one sequence per GPU)",
+                   "l2": "inputs larger than L2 (q+gate+out 3.2 GB per step), no flush"},
+        "gpu_launches": 3 * args.steps,
+        "e2e": {"value": tokens_step / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "roofline": roof,
+        "stages": stage_roof,
+        "gather": {"per_query_kv_bytes": wc["gather_bytes"], "effective_gather_GBps": gather_gbs,
+                   "compulsory_bytes": wc["kv_bytes"] + wc["qgo_bytes"] + wc["sel_bytes"]},
+        "clocks": clocks,
+    }
+    cpu_in = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        rows = sample_rows_strided(cfg, CPU_STRIDE)
+        full = {n: to_host(dev[n][:1]) for n in ("k", "v", "k_idx")}
+        part = {n: to_host(dev[n][0, rows[:, 1]]).reshape(len(rows), -1) for n in ("q", "q_idx", "gate")}
+        cpu_in = (rows, full, part)
+    # release the prefill buffers before the decode workload
+    del dev, out, sel, kbar, ws, host, out_h
+    torch.cuda.empty_cache()
+    if not args.no_decode:
+        result["decode"] = run_decode(args, world, s)
+    if cpu_in is not None:
+        result["cpu_baseline"] = cpu_baseline(cfg, *cpu_in)
+    return result
+
+
+def run_decode(args, world, s):
+    import torch
+    import block_sparse_long_kbar_b200 as sg
+    from sgqa_inputs import gen_device
+    cfg = CONFIGS["decode_1m"]
+    shape_of = lambda c, n, **kw: c.shape(n, **kw)
+    n_new = DECODE_NEW
+    cache_len = cfg.T
+    T_cap = cache_len + cfg.B
+    dims = sg.sgqa_dims(cfg.batch, T_cap, cfg.Hq, cfg.G, cfg.d, cfg.d_idx, cfg.B, cfg.k)
+    caches = {}
+    for n in ("k", "v", "k_idx"):
+        caches[n] = torch.zeros(shape_of(cfg, n, T=T_cap), dtype=torch.bfloat16, device="cuda")
+        gen_device(cfg, n, caches[n], t0=0, n_t=cache_len)
+    kbar = torch.zeros((cfg.batch, T_cap // cfg.B, cfg.d_idx), device="cuda")
+    sg.sgqa_compress_keys(dims, caches["k_idx"], kbar, None)
+    new = {}
+    for n in ("q", "k", "v", "gate", "q_idx", "k_idx"):
+        new[n] = torch.empty((cfg.batch, n_new) + shape_of(cfg, n)[2:], dtype=torch.bfloat16, device="cuda")
+        gen_device(cfg, n, new[n], t0=cache_len, n_t=n_new, dst_t0=0)
+    out = torch.empty((cfg.batch, n_new, cfg.Hq, cfg.d), dtype=torch.bfloat16, device="cuda")
+    ws = sg.alloc_workspace(sg.sgqa_decode_workspace_size(dims, n_new))
+    sg.sgqa_reset_device_status(ws)
+    torch.cuda.synchronize()
+
+    def step():
+        sg.sgqa_decode(dims, cache_len, n_new, caches["k"], caches["v"], caches["k_idx"], kbar, new["q"], new["k"],
+                       new["v"], new["q_idx"], new["k_idx"], new["gate"], out, ws, stream=s)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    steps = max(args.steps, 10)
+    e0.record(s)
+    for _ in range(steps):
+        step()
+    e1.record(s)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
+    assert sg.sgqa_get_device_status(ws) == 0
+    toks = world * cfg.batch * n_new
+    kbar_bytes = cfg.batch * (cache_len // cfg.B) * cfg.d_idx * 4
+    visits = cfg.batch * cfg.G * sum((cfg.Kb - 1) * cfg.B + i + 1 for i in range(n_new))
+    gather = visits * 2 * cfg.d * 2
+    res = {"metric": "decode query tokens/s at 1M context (32 seqs x 4 new tokens)", "value": toks / (ms / 1e3),
+           "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+           "workload": f"decode: {cfg.batch} seqs x {n_new} new tokens after {cache_len} cached, Hq={cfg.Hq}, "
+                       f"G={cfg.G}, d={cfg.d}, d_idx={cfg.d_idx}, B={cfg.B}, k={cfg.k}, span {cfg.span}, seed {cfg.seed}",
+           "algorithmic_bytes": kbar_bytes + gather,
+           "hbm_frac": (kbar_bytes + gather) / (ms / 1e3) / 1e9 / load_peaks()["hbm_gbs"],
+           "gpu_launches_per_step": 7}
+    del caches, kbar, new, out, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+CPU_STRIDE = 64
+
+
+def cpu_baseline(cfg, rows, full, part):
+    """The oracle, as it stands, timed on the host cores on a strided sample of the same
+    workload (the very bytes the GPU consumed)."""
+    import oracle
+    oracle.build()
+    stride = CPU_STRIDE
+    secs = oracle_sample_time(cfg, stride, full, part, rows)
+    return {"value": len(rows) / secs, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"every {stride}th query row of the {cfg.name} sequence ({len(rows)} rows, all heads and "
+                      f"groups; block means of the whole sequence), {secs:.1f} s"}
+
+
+def run_reference(args, world, rank):
+    """The fp64 oracle as it stands, on the host cores, on bounded strided samples of the workload."""
+    import oracle
+    oracle.build()
+    cfg = CONFIGS[args.config]
+    stride = 256
+    rows0 = sample_rows_strided(cfg, stride)
+    full, _ = oracle_inputs_host(cfg, rows0)
+    times = []
+    for i in range(args.warmup + args.steps):
+        rows = sample_rows_strided(cfg, stride, offset=i * 37)
+        part = {n: gen_rows(cfg, n, 0, rows[:, 1]) for n in ("q", "q_idx", "gate")}
+        secs = oracle_sample_time(cfg, stride, full, part, rows)
+        if i >= args.warmup:
+            times.append((len(rows), secs))
+    n = sum(r for r, _ in times)
+    tot = sum(s for _, s in times)
+    value = n / tot
+    ms = 1e3 * cfg.T / value
+    sample = (f"per step every {stride}th query row of the {cfg.name} sequence (rotating offset, "
+              f"{len(rows0)} rows), fp64 oracle on {oracle.max_threads()} host threads")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded topic-structured generator)",
+            "config": {"workload": f"prefill {cfg.name}: batch {cfg.batch}, T={cfg.T}, Hq={cfg.Hq}, G={cfg.G}, "
+                                   f"d={cfg.d}, d_idx={cfg.d_idx}, B={cfg.B}, k={cfg.k}, topic span {cfg.span}, "
+                                   f"seed {cfg.seed}", "global_batch": cfg.batch, "seq_len": cfg.T,
+                       "parallelism": "host cores (OpenMP)"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="128k", choices=["tiny", "32k", "128k", "64k_b8", "64k_b1"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, world, rank)), flush=True)
+        return
+    world, rank, _ = dist_setup(args.gpus)
+    try:
+        res = run_ours(args, world, rank)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

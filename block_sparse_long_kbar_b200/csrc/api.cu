@@ -1,0 +1,275 @@
+// C ABI of libsgqa: argument validation, workspace layout and the kernel sequence of every
+// entry point declared in include/sgqa.h. No allocation, no host synchronisation (except the
+// explicit status read), no global state.
+#include <cstdint>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace sgqa;
+
+namespace {
+
+constexpr int kSelChunkT = 32768;  // query rows per selection chunk when sel stays in ws
+
+bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_dims(const sgqa_dims* d) {
+  if (!d) return SGQA_ERR_INVALID_ARG;
+  if (d->batch <= 0 || d->T <= 0 || d->Hq <= 0 || d->G <= 0 || d->d <= 0 || d->d_idx <= 0 || d->B <= 0 ||
+      d->k <= 0)
+    return SGQA_ERR_INVALID_ARG;
+  if (d->T >= (1 << 28) || d->batch > 65535) return SGQA_ERR_UNSUPPORTED;
+  if (d->d != 64 && d->d != 128) return SGQA_ERR_UNSUPPORTED;
+  if (d->d_idx != 32 && d->d_idx != 64) return SGQA_ERR_UNSUPPORTED;
+  if (d->B != 1 && d->B != 2 && d->B != 4 && d->B != 8 && d->B != 16) return SGQA_ERR_UNSUPPORTED;
+  if (d->k % d->B != 0) return SGQA_ERR_UNSUPPORTED;
+  if (d->Hq % d->G != 0 || d->Hq / d->G > 16 || 128 % d->G != 0) return SGQA_ERR_UNSUPPORTED;
+  if (d->k / d->B > 16384) return SGQA_ERR_UNSUPPORTED;
+  return SGQA_OK;
+}
+
+struct PrefillWs {
+  int* status;
+  float* kbar;
+  uint16_t* hi;
+  uint16_t* lo;
+  int32_t* sel;
+  size_t bytes;
+};
+
+PrefillWs prefill_layout(const sgqa_dims* d, void* ws) {
+  PrefillWs w{};
+  const size_t nblk = (size_t)(d->T / d->B);
+  const size_t nk = (size_t)d->batch * nblk * d->d_idx;
+  const size_t chunk = (size_t)(d->T < kSelChunkT ? d->T : kSelChunkT);
+  size_t off = kStatusBytes;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  w.status = reinterpret_cast<int*>(base);
+  w.kbar = reinterpret_cast<float*>(base + off);
+  off += align256(nk * 4);
+  w.hi = reinterpret_cast<uint16_t*>(base + off);
+  off += align256(nk * 2);
+  w.lo = reinterpret_cast<uint16_t*>(base + off);
+  off += align256(nk * 2);
+  w.sel = reinterpret_cast<int32_t*>(base + off);
+  off += align256((size_t)d->batch * chunk * d->G * (d->k / d->B) * 4);
+  w.bytes = off;
+  return w;
+}
+
+int decode_splits(long units) {
+  long s = 4096 / (units > 0 ? units : 1);
+  if (s < 1) s = 1;
+  if (s > 16) s = 16;
+  return (int)s;
+}
+
+struct DecodeWs {
+  int* status;
+  float* scores;
+  int32_t* sel;
+  float* part;
+  size_t bytes;
+};
+
+DecodeWs decode_layout(const sgqa_dims* d, int n_new, void* ws) {
+  DecodeWs w{};
+  const size_t nblk = (size_t)(d->T / d->B);
+  const long units = (long)d->batch * n_new * d->G;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  size_t off = kStatusBytes;
+  w.status = reinterpret_cast<int*>(base);
+  w.scores = reinterpret_cast<float*>(base + off);
+  off += align256((size_t)units * nblk * 4);
+  w.sel = reinterpret_cast<int32_t*>(base + off);
+  off += align256((size_t)units * (d->k / d->B) * 4);
+  w.part = reinterpret_cast<float*>(base + off);
+  off += align256(attend_part_bytes((int)units, decode_splits(units), d->Hq / d->G, d->d));
+  w.bytes = off;
+  return w;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? SGQA_OK : SGQA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* sgqa_status_string(int status) {
+  switch (status) {
+    case SGQA_OK: return "ok";
+    case SGQA_ERR_INVALID_ARG: return "invalid argument";
+    case SGQA_ERR_UNSUPPORTED: return "unsupported shape";
+    case SGQA_ERR_WORKSPACE: return "workspace too small or misaligned";
+    case SGQA_ERR_CUDA: return "CUDA error";
+    case SGQA_ERR_TIMEOUT: return "device wait timed out";
+    case SGQA_ERR_DEVICE_CHECK: return "device-side check failed";
+    default: return "unknown status";
+  }
+}
+
+const char* sgqa_version(void) { return "sgqa 0.1 sm_100a"; }
+
+size_t sgqa_workspace_size(const sgqa_dims* dims) {
+  if (check_dims(dims) != SGQA_OK) return 0;
+  return prefill_layout(dims, nullptr).bytes;
+}
+
+size_t sgqa_decode_workspace_size(const sgqa_dims* dims, int n_new) {
+  if (check_dims(dims) != SGQA_OK || n_new <= 0 || n_new * dims->G > 32) return 0;
+  return decode_layout(dims, n_new, nullptr).bytes;
+}
+
+int sgqa_reset_device_status(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || ws_bytes < kStatusBytes) return SGQA_ERR_WORKSPACE;
+  return cuda_status(cudaMemsetAsync(ws, 0, sizeof(int), static_cast<cudaStream_t>(stream)));
+}
+
+int sgqa_get_device_status(const void* ws, size_t ws_bytes, int* status) {
+  if (!ws || ws_bytes < kStatusBytes || !status) return SGQA_ERR_INVALID_ARG;
+  int v = 0;
+  const cudaError_t e = cudaMemcpy(&v, ws, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return SGQA_ERR_CUDA;
+  *status = v;
+  return SGQA_OK;
+}
+
+int sgqa_compress_keys(const sgqa_dims* dims, const uint16_t* k_idx, float* kbar, void* ws, size_t ws_bytes,
+                       void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (!aligned16(k_idx) || !aligned16(kbar)) return SGQA_ERR_INVALID_ARG;
+  (void)ws;
+  (void)ws_bytes;
+  return cuda_status(launch_compress(k_idx, kbar, nullptr, nullptr, dims->batch, dims->T, dims->d_idx, dims->B, 0,
+                                     dims->T / dims->B, static_cast<cudaStream_t>(stream)));
+}
+
+int sgqa_select(const sgqa_dims* dims, const uint16_t* q_idx, const float* kbar, int32_t* sel, void* ws,
+                size_t ws_bytes, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (!aligned16(q_idx) || !aligned16(kbar) || !aligned16(sel)) return SGQA_ERR_INVALID_ARG;
+  const PrefillWs w = prefill_layout(dims, ws);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < (size_t)((uint8_t*)w.sel - (uint8_t*)ws))
+    return SGQA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  SelectArgs a{};
+  a.q_idx = q_idx; a.kbar = kbar; a.kbar_hi = w.hi; a.kbar_lo = w.lo; a.sel = sel;
+  a.batch = dims->batch; a.T = dims->T; a.G = dims->G; a.d_idx = dims->d_idx; a.B = dims->B;
+  a.Kb = dims->k / dims->B; a.t_begin = 0; a.t_end = dims->T; a.sel_T = dims->T; a.sel_t0 = 0;
+  a.status = w.status;
+  return cuda_status(launch_select(a, s));
+}
+
+static AttendArgs prefill_attend_args(const sgqa_dims* d, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                      const uint16_t* gate, uint16_t* out, int* status) {
+  AttendArgs a{};
+  a.q = q; a.gate = gate; a.out = out; a.k = k; a.v = v;
+  a.batch = d->batch; a.nQ = d->T; a.q_t0 = 0; a.T_kv = d->T; a.Hq = d->Hq; a.G = d->G; a.d = d->d;
+  a.B = d->B; a.Kb = d->k / d->B; a.splits = 1; a.status = status;
+  return a;
+}
+
+int sgqa_attend(const sgqa_dims* dims, const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* gate,
+                const int32_t* sel, uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gate) || !aligned16(sel) || !aligned16(out))
+    return SGQA_ERR_INVALID_ARG;
+  const PrefillWs w = prefill_layout(dims, ws);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < (size_t)kStatusBytes) return SGQA_ERR_WORKSPACE;
+  AttendArgs a = prefill_attend_args(dims, q, k, v, gate, out, w.status);
+  a.sel = sel; a.sel_T = dims->T; a.sel_t0 = 0; a.t_begin = 0; a.t_end = dims->T;
+  return cuda_status(launch_attend(a, static_cast<cudaStream_t>(stream)));
+}
+
+int sgqa_forward(const sgqa_dims* dims, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                 const uint16_t* q_idx, const uint16_t* k_idx, const uint16_t* gate, uint16_t* out,
+                 int32_t* sel_out, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_idx) || !aligned16(k_idx) ||
+      !aligned16(gate) || !aligned16(out) || (sel_out && !aligned16(sel_out)))
+    return SGQA_ERR_INVALID_ARG;
+  const PrefillWs w = prefill_layout(dims, ws);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < w.bytes) return SGQA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (launch_compress(k_idx, w.kbar, w.hi, w.lo, dims->batch, dims->T, dims->d_idx, dims->B, 0, dims->T / dims->B,
+                      s) != cudaSuccess)
+    return SGQA_ERR_CUDA;
+  SelectArgs sa{};
+  sa.q_idx = q_idx; sa.kbar = w.kbar; sa.kbar_hi = w.hi; sa.kbar_lo = w.lo;
+  sa.batch = dims->batch; sa.T = dims->T; sa.G = dims->G; sa.d_idx = dims->d_idx; sa.B = dims->B;
+  sa.Kb = dims->k / dims->B; sa.status = w.status;
+  AttendArgs aa = prefill_attend_args(dims, q, k, v, gate, out, w.status);
+  const int chunk = sel_out ? dims->T : (dims->T < kSelChunkT ? dims->T : kSelChunkT);
+  for (int t0 = 0; t0 < dims->T; t0 += chunk) {
+    const int t1 = t0 + chunk < dims->T ? t0 + chunk : dims->T;
+    sa.sel = sel_out ? sel_out : w.sel;
+    sa.sel_T = sel_out ? dims->T : chunk;
+    sa.sel_t0 = sel_out ? 0 : t0;
+    sa.t_begin = t0; sa.t_end = t1;
+    if (launch_select(sa, s) != cudaSuccess) return SGQA_ERR_CUDA;
+    aa.sel = sa.sel; aa.sel_T = sa.sel_T; aa.sel_t0 = sa.sel_t0; aa.t_begin = t0; aa.t_end = t1;
+    if (launch_attend(aa, s) != cudaSuccess) return SGQA_ERR_CUDA;
+  }
+  return SGQA_OK;
+}
+
+int sgqa_decode(const sgqa_dims* dims, int cache_len, int n_new, uint16_t* k_cache, uint16_t* v_cache,
+                uint16_t* kidx_cache, float* kbar_cache, const uint16_t* q_new, const uint16_t* k_new,
+                const uint16_t* v_new, const uint16_t* qidx_new, const uint16_t* kidx_new, const uint16_t* gate_new,
+                uint16_t* out, int32_t* sel_out, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (n_new <= 0 || cache_len < 0 || (long)cache_len + n_new > dims->T || n_new * dims->G > 32)
+    return SGQA_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(kidx_cache) || !aligned16(kbar_cache) ||
+      !aligned16(q_new) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(qidx_new) || !aligned16(kidx_new) ||
+      !aligned16(gate_new) || !aligned16(out) || (sel_out && !aligned16(sel_out)))
+    return SGQA_ERR_INVALID_ARG;
+  const DecodeWs w = decode_layout(dims, n_new, ws);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < w.bytes) return SGQA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int T = dims->T, G = dims->G, d = dims->d, di = dims->d_idx, B = dims->B, Kb = dims->k / dims->B;
+  const int nblk = T / B;
+  cudaError_t e;
+  // 1. append the new rows
+  if ((e = launch_append(k_cache, k_new, dims->batch, (long)G * d, (long)T * G * d, (long)cache_len * G * d,
+                         (long)n_new * G * d, s)) != cudaSuccess)
+    return SGQA_ERR_CUDA;
+  if ((e = launch_append(v_cache, v_new, dims->batch, (long)G * d, (long)T * G * d, (long)cache_len * G * d,
+                         (long)n_new * G * d, s)) != cudaSuccess)
+    return SGQA_ERR_CUDA;
+  if ((e = launch_append(kidx_cache, kidx_new, dims->batch, di, (long)T * di, (long)cache_len * di, (long)n_new * di,
+                         s)) != cudaSuccess)
+    return SGQA_ERR_CUDA;
+  // 2. block means of the blocks the new rows complete
+  const int j0 = cache_len / B, j1 = (cache_len + n_new) / B;
+  if (j1 > j0 && (e = launch_compress(kidx_cache, kbar_cache, nullptr, nullptr, dims->batch, T, di, B, j0, j1, s)) !=
+                     cudaSuccess)
+    return SGQA_ERR_CUDA;
+  // 3. indexer scores and selection
+  if ((e = launch_decode_scores(qidx_new, kbar_cache, w.scores, dims->batch, n_new, G, di, B, nblk, cache_len, s)) !=
+      cudaSuccess)
+    return SGQA_ERR_CUDA;
+  int32_t* sel = sel_out ? sel_out : w.sel;
+  if ((e = launch_decode_select(w.scores, sel, dims->batch, n_new, G, B, Kb, nblk, cache_len, w.status, s)) !=
+      cudaSuccess)
+    return SGQA_ERR_CUDA;
+  // 4. split-K gated attention
+  AttendArgs a{};
+  a.q = q_new; a.gate = gate_new; a.out = out; a.k = k_cache; a.v = v_cache; a.sel = sel; a.part = w.part;
+  a.batch = dims->batch; a.nQ = n_new; a.q_t0 = cache_len; a.T_kv = T; a.Hq = dims->Hq; a.G = G; a.d = d; a.B = B;
+  a.Kb = Kb; a.sel_T = n_new; a.sel_t0 = cache_len; a.t_begin = cache_len; a.t_end = cache_len + n_new;
+  a.splits = decode_splits((long)dims->batch * n_new * G);
+  a.status = w.status;
+  if ((e = launch_attend(a, s)) != cudaSuccess) return SGQA_ERR_CUDA;
+  if ((e = launch_attend_merge(a, s)) != cudaSuccess) return SGQA_ERR_CUDA;
+  return SGQA_OK;
+}
+
+}  // extern "C"

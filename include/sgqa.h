@@ -1,0 +1,143 @@
+/* sgqa.h — C ABI of libsgqa.so: Sparse GQA (Step 5 Preview's full-context attention layer)
+ * on NVIDIA B200 (sm_100a).
+ *
+ * What the layer computes. The pages give prose, not formulas; these are the readings used:
+ *   mo.ai.kr, "Step 5 Preview agentic work design", section "model structure and training
+ *   stability" — the full-context layers use Sparse GQA on top of Gated GQA; shared index keys
+ *   are compressed per block of B = 8 tokens; every KV group selects its own relevant past
+ *   context; the final setting is k = 4096 tokens, i.e. 512 blocks.
+ *   ai.info, "StepFun illustrates the 92-block architecture of Step 5 Preview", section "Sparse
+ *   GQA aims at a 1 million token context" — relevant past blocks are selected instead of the
+ *   whole history; blocks of eight cut indexing and selection cost eightfold.
+ *
+ *   (1) compress  kbar[b,j,:] = (1/B) sum_{i<B} k_idx[b, jB+i, :]   for complete blocks j < T/B
+ *   (2) select    per (b,t,g): c = floor(t/B) (own block); candidates j < c scored by
+ *                 s_j = q_idx[b,t,g,:] . kbar[b,j,:]; keep the best m = min(k/B - 1, c) by
+ *                 (s desc, j asc) plus the own block c; ascending, padded with -1 to k/B
+ *   (3) attend    for each head h of group g = floor(h / (Hq/G)), over the selected tokens
+ *                 U = {u <= t : floor(u/B) in S}: o = softmax_U(q[b,t,h] . k[b,u,g] / sqrt(d)) v
+ *   (4) gate      out[b,t,h,:] = o * sigmoid(gate_logits[b,t,h,:])      (elementwise, bf16 RNE)
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller, contiguous row-major with the
+ *     batch index leading, and 16-byte aligned. bf16 tensors are passed as uint16_t bit patterns.
+ *       q, gate_logits, out  [batch, T, Hq, d]      k, v   [batch, T, G, d]
+ *       q_idx                [batch, T, G, d_idx]   k_idx  [batch, T, d_idx]
+ *       kbar (fp32)          [batch, T/B, d_idx]    sel (int32) [batch, T, G, k/B]
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Every call only enqueues
+ *     work on it: no host synchronisation, no allocation, no freeing.
+ *   - `ws` is caller-owned device workspace of at least the size the matching *_workspace_size
+ *     call returns (256-byte aligned; sgqa_compress_keys needs none). Its first 256 bytes hold a
+ *     sticky device status word; zero it once with sgqa_reset_device_status before first use.
+ *     Calls that share one ws must not overlap on the device.
+ *   - The return value reports argument validation and launch errors only (sgqa_status).
+ *     Errors found on the device (a selection naming a block outside [0, t/B], a bounded wait
+ *     that ran out) are recorded in the status word; read it with sgqa_get_device_status after
+ *     synchronising the stream.
+ *   - Supported shapes (else SGQA_ERR_UNSUPPORTED): d in {64, 128}; d_idx in {32, 64};
+ *     B in {1, 2, 4, 8, 16}; k % B == 0; Hq % G == 0 with 1 <= Hq/G <= 16; 128 % G == 0;
+ *     1 <= T < 2^28. A trailing partial block is never a candidate.
+ *   - Results are deterministic: the same inputs give the same bits, run after run.
+ */
+#ifndef SGQA_H
+#define SGQA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SGQA_OK = 0,
+  SGQA_ERR_INVALID_ARG = 1,   /* null pointer, misaligned pointer, negative size, ... */
+  SGQA_ERR_UNSUPPORTED = 2,   /* shape outside the supported set above */
+  SGQA_ERR_WORKSPACE = 3,     /* ws too small or misaligned */
+  SGQA_ERR_CUDA = 4,          /* a CUDA launch or runtime call failed */
+  SGQA_ERR_TIMEOUT = 5,       /* device status: a bounded wait ran out */
+  SGQA_ERR_DEVICE_CHECK = 6   /* device status: a device-side argument check failed */
+} sgqa_status;
+
+typedef struct {
+  int batch; /* sequences */
+  int T;     /* tokens per sequence (for decode: cache capacity) */
+  int Hq;    /* query heads */
+  int G;     /* KV groups; head h uses group h / (Hq / G) */
+  int d;     /* head dim of q, k, v, gate, out */
+  int d_idx; /* indexer dim of q_idx, k_idx, kbar */
+  int B;     /* block size (tokens per compressed index key) */
+  int k;     /* selection budget in tokens; k / B blocks including the own block */
+} sgqa_dims;
+
+/* Human-readable text of a status code (static storage). */
+const char* sgqa_status_string(int status);
+
+/* Library version and build target (static storage), e.g. "sgqa 0.1 sm_100a". */
+const char* sgqa_version(void);
+
+/* Bytes of workspace that sgqa_compress_keys, sgqa_select, sgqa_attend and sgqa_forward need
+ * for these dims; 0 if the dims are invalid or unsupported. */
+size_t sgqa_workspace_size(const sgqa_dims* dims);
+
+/* Bytes of workspace sgqa_decode needs for n_new new tokens per sequence; 0 if invalid. */
+size_t sgqa_decode_workspace_size(const sgqa_dims* dims, int n_new);
+
+/* Zero the device status word at the start of ws (async on stream). */
+int sgqa_reset_device_status(void* ws, size_t ws_bytes, void* stream);
+
+/* Copy the device status word to *status (a blocking device-to-host copy; call after the
+ * stream that ran the kernels has been synchronised). *status is SGQA_OK or an error code. */
+int sgqa_get_device_status(const void* ws, size_t ws_bytes, int* status);
+
+/* Step (1): block-mean compression of the shared index keys (see the header comment).
+ * k_idx [batch, T, d_idx] bf16 -> kbar [batch, T/B, d_idx] fp32. The block's keys are summed
+ * in fp64 in token order and rounded once, so kbar is the fp32 rounding (RNE) of the block
+ * mean. This call uses no workspace: ws may be NULL and ws_bytes 0. */
+int sgqa_compress_keys(const sgqa_dims* dims, const uint16_t* k_idx, float* kbar, void* ws,
+                       size_t ws_bytes, void* stream);
+
+/* Step (2): per-(token, group) block selection.
+ * q_idx [batch, T, G, d_idx] bf16, kbar [batch, T/B, d_idx] fp32 -> sel [batch, T, G, k/B]
+ * int32: ascending block ids, own block last among the valid entries, -1 padding; exactly
+ * min(k/B, floor(t/B) + 1) valid entries per row. Scores are accumulated in fp32; candidates
+ * whose fp32 scores tie go to the lower block index. */
+int sgqa_select(const sgqa_dims* dims, const uint16_t* q_idx, const float* kbar, int32_t* sel,
+                void* ws, size_t ws_bytes, void* stream);
+
+/* Steps (3)+(4): gated attention of every query row over a given selection.
+ * q, gate [batch, T, Hq, d], k, v [batch, T, G, d] bf16; sel [batch, T, G, k/B] int32 in the
+ * format sgqa_select writes (any order of valid entries is accepted; entries > t/B are
+ * rejected by a device check and skipped) -> out [batch, T, Hq, d] bf16. */
+int sgqa_attend(const sgqa_dims* dims, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                const uint16_t* gate, const int32_t* sel, uint16_t* out, void* ws,
+                size_t ws_bytes, void* stream);
+
+/* The whole layer, steps (1)-(4), for all T rows of every sequence. If sel_out is not NULL it
+ * receives the selection [batch, T, G, k/B]; otherwise the selection is kept in ws, in query
+ * chunks (index selection chunked to bound memory, as the pages describe for training). */
+int sgqa_forward(const sgqa_dims* dims, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                 const uint16_t* q_idx, const uint16_t* k_idx, const uint16_t* gate,
+                 uint16_t* out, int32_t* sel_out, void* ws, size_t ws_bytes, void* stream);
+
+/* One decode step for dims.batch sequences sharing one cache length.
+ * Caches (dims.T = capacity): k_cache, v_cache [batch, T, G, d], kidx_cache [batch, T, d_idx]
+ * bf16, kbar_cache [batch, T/B, d_idx] fp32 holding the block means of every block complete in
+ * the first cache_len tokens. New tokens: q_new, gate_new [batch, n_new, Hq, d], k_new, v_new
+ * [batch, n_new, G, d], qidx_new [batch, n_new, G, d_idx], kidx_new [batch, n_new, d_idx].
+ * The step writes the new k, v, k_idx rows at positions [cache_len, cache_len + n_new), adds
+ * kbar for the blocks they complete, and writes out [batch, n_new, Hq, d] (and, if not NULL,
+ * sel_out [batch, n_new, G, k/B]) exactly as sgqa_forward would give for the last n_new rows of
+ * the concatenated sequence. Requires cache_len + n_new <= T. Repeating a step at the same
+ * cache_len rewrites the same rows, so it is idempotent. */
+int sgqa_decode(const sgqa_dims* dims, int cache_len, int n_new, uint16_t* k_cache,
+                uint16_t* v_cache, uint16_t* kidx_cache, float* kbar_cache, const uint16_t* q_new,
+                const uint16_t* k_new, const uint16_t* v_new, const uint16_t* qidx_new,
+                const uint16_t* kidx_new, const uint16_t* gate_new, uint16_t* out,
+                int32_t* sel_out, void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SGQA_H */

@@ -76,6 +76,14 @@ class Config:
     def replace(self, **kw) -> "Config":
         return dataclasses.replace(self, **kw)
 
+    def shape(self, name: str, T: int | None = None, batch: int | None = None) -> tuple:
+        """Natural layout of tensor `name`: q/gate [b,T,Hq,d], k/v [b,T,G,d], q_idx [b,T,G,d_idx],
+        k_idx [b,T,d_idx]."""
+        T = self.T if T is None else T
+        b = self.batch if batch is None else batch
+        return {"q": (b, T, self.Hq, self.d), "gate": (b, T, self.Hq, self.d), "k": (b, T, self.G, self.d),
+                "v": (b, T, self.G, self.d), "q_idx": (b, T, self.G, self.d_idx), "k_idx": (b, T, self.d_idx)}[name]
+
 
 # The five workloads of the hot path (prefill tiny / 32K / 128K, the B=1 vs B=8 ablation at
 # 64K, and MTP-style decode at 1M context with 4 new tokens per sequence).
@@ -216,22 +224,24 @@ def _lib():
         _gen_lib.sgqa_gen_fill.restype = ctypes.c_int
         _gen_lib.sgqa_gen_fill.argtypes = [
             ctypes.c_int, ctypes.c_uint64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]
     return _gen_lib
 
 
-def gen_device(cfg: Config, name: str, out, t0: int = 0, n_t: int | None = None, stream=None):
-    """Fill a torch CUDA tensor `out` laid out [batch, T_alloc, W] (bf16 or int16) with tokens
-    [t0, t0 + n_t) of tensor `name`, rows written at positions t0.. of each sequence."""
+def gen_device(cfg: Config, name: str, out, t0: int = 0, n_t: int | None = None, dst_t0: int | None = None,
+               stream=None):
+    """Fill a torch CUDA tensor `out` laid out [batch, T_alloc, W] (bf16 or int16) with the values
+    of positions [t0, t0 + n_t) of tensor `name`, written at rows dst_t0.. (default t0)."""
     import torch
     n_t = cfg.T - t0 if n_t is None else n_t
+    dst_t0 = t0 if dst_t0 is None else dst_t0
     W = cfg.width(name)
     assert out.is_cuda and out.is_contiguous() and out.element_size() == 2
     T_alloc = out.numel() // (cfg.batch * W)
-    assert out.numel() == cfg.batch * T_alloc * W and t0 + n_t <= T_alloc
+    assert out.numel() == cfg.batch * T_alloc * W and dst_t0 + n_t <= T_alloc
     s = torch.cuda.current_stream().cuda_stream if stream is None else stream
     rc = _lib().sgqa_gen_fill(KIND_CODES[name], cfg.seed, cfg.span, cfg.G, cfg.d_idx, W,
-                              cfg.batch, t0, n_t, T_alloc * W, ctypes.c_void_p(out.data_ptr()),
+                              cfg.batch, t0, n_t, dst_t0, T_alloc * W, ctypes.c_void_p(out.data_ptr()),
                               ctypes.c_void_p(s))
     if rc != 0:
         raise RuntimeError(f"sgqa_gen_fill failed with CUDA error {rc}")

@@ -49,7 +49,7 @@ __device__ __forceinline__ uint16_t to_bf16_bits(double v) {
 // kind: 0 q, 1 k, 2 v, 3 gate, 4 q_idx, 5 k_idx (streams 1..6); topics stream 7, r stream 8
 __global__ void gen_fill_kernel(int kind, uint64_t key, uint64_t topic_key, uint64_t r_key,
                                 int span, int G, int d_idx, int W, int batch, int t0, int n_t,
-                                int64_t batch_stride, uint16_t* __restrict__ out) {
+                                int dst_t0, int64_t batch_stride, uint16_t* __restrict__ out) {
   const int64_t total = (int64_t)batch * n_t * W;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
        e += (int64_t)gridDim.x * blockDim.x) {
@@ -69,14 +69,16 @@ __global__ void gen_fill_kernel(int kind, uint64_t key, uint64_t topic_key, uint
       const uint64_t r = wr % (t / (uint64_t)span + 1);
       v = __dadd_rn(v, 2.0 * normal_at(topic_key, ((((uint64_t)b) << 32) + r) * (uint64_t)d_idx + (uint64_t)i));
     }
-    out[(int64_t)b * batch_stride + (int64_t)(t0 + tt) * W + w] = to_bf16_bits(v);
+    out[(int64_t)b * batch_stride + (int64_t)(dst_t0 + tt) * W + w] = to_bf16_bits(v);
   }
 }
 
 }  // namespace
 
+// Fills out[b, dst_t0 + i, :] (rows W wide, sequences batch_stride elements apart) with the
+// values of positions t0 + i, i < n_t, of tensor `kind` of every sequence b < batch.
 extern "C" int sgqa_gen_fill(int kind, uint64_t seed, int span, int G, int d_idx, int W, int batch,
-                             int t0, int n_t, int64_t batch_stride, void* out, void* stream) {
+                             int t0, int n_t, int dst_t0, int64_t batch_stride, void* out, void* stream) {
   if (kind < 0 || kind > 5 || W <= 0 || batch <= 0 || n_t < 0 || span <= 0) return (int)cudaErrorInvalidValue;
   if (n_t == 0) return 0;
   const uint64_t key = stream_key(seed, (uint64_t)kind + 1);
@@ -86,6 +88,6 @@ extern "C" int sgqa_gen_fill(int kind, uint64_t seed, int span, int G, int d_idx
   int64_t blocks = (total + 255) / 256;
   if (blocks > 148 * 64) blocks = 148 * 64;
   gen_fill_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(
-      kind, key, topic_key, r_key, span, G, d_idx, W, batch, t0, n_t, batch_stride, (uint16_t*)out);
+      kind, key, topic_key, r_key, span, G, d_idx, W, batch, t0, n_t, dst_t0, batch_stride, (uint16_t*)out);
   return (int)cudaGetLastError();
 }

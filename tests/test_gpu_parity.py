@@ -1,0 +1,308 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the same seeded inputs.
+
+* kbar: bit-exact against the oracle's fp64 block mean rounded once to fp32.
+* selection: identical block sets, except near-ties (every swapped block's oracle score within
+  1e-4 * |s_m| of the oracle's m-th best score s_m), which are counted.
+* outputs with the oracle's selection replayed (sgqa_attend): max-abs <= 1e-2, mean-abs <= 1e-3.
+* the whole layer (sgqa_forward) and a decode step (sgqa_decode) likewise.
+
+Small workloads are compared in full (several tiles and a ragged tail); the full-size
+workloads, in the launch configuration the benchmark times, on seeded samples of rows.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import oracle
+import block_sparse_long_kbar_b200 as sg
+from sgqa_inputs import CONFIGS, DECODE_NEW, Config, gen_device, gen_rows
+from tests._helpers import (NAMES, all_rows, assert_outputs_close, compare_selection, device_inputs, host_inputs,
+                            output_errors, sample_rows, shape_of, to_dev, to_host)
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "tiny": CONFIGS["tiny"],
+    "ragged_g4": Config("ragged_g4", 2, 3001, 32, 4, 128, 64, 8, 512, 400, 7),
+    "b1": Config("b1", 1, 1500, 8, 2, 64, 32, 1, 128, 200, 8),
+    "b16_r16": Config("b16_r16", 1, 1000, 16, 1, 128, 64, 16, 256, 160, 9),
+    "g8_r1": Config("g8_r1", 1, 777, 8, 8, 64, 32, 4, 64, 100, 10),
+    "dense": Config("dense", 1, 300, 8, 2, 64, 32, 8, 304, 64, 11),
+    "t9": Config("t9", 3, 9, 8, 2, 64, 32, 8, 16, 4, 12),
+    "t1": Config("t1", 2, 1, 4, 4, 128, 64, 8, 64, 4, 13),
+}
+
+
+def _ws(dims):
+    ws = sg.alloc_workspace(sg.sgqa_workspace_size(dims))
+    sg.sgqa_reset_device_status(ws)
+    return ws
+
+
+def _status_ok(ws):
+    torch.cuda.synchronize()
+    assert sg.sgqa_get_device_status(ws) == 0
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    sg.load_library()
+    oracle.build()
+
+
+@pytest.fixture(scope="module")
+def small_cases():
+    cache = {}
+
+    def get(name):
+        if name not in cache:
+            cfg = SMALL[name]
+            h = host_inputs(cfg)
+            d = {n: to_dev(h[n], shape_of(cfg, n)) for n in NAMES}
+            dm = oracle.dims_of(cfg)
+            kbar64 = oracle.compress(dm, h["k_idx"])
+            rows = all_rows(cfg)
+            qi = h["q_idx"].reshape(cfg.batch * cfg.T, -1)
+            sel_o, s_m, s_m1 = oracle.select(dm, kbar64, rows, qi)
+            cache[name] = (cfg, h, d, dm, kbar64, rows, sel_o, s_m)
+        return cache[name]
+    return get
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_compress_bit_exact(small_cases, name):
+    cfg, h, d, dm, kbar64, *_ = small_cases(name)
+    dims = sg.sgqa_dims.of(cfg)
+    kbar = torch.full((cfg.batch, cfg.T // cfg.B, cfg.d_idx), float("nan"), device="cuda")
+    sg.sgqa_compress_keys(dims, d["k_idx"], kbar, None)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(kbar.cpu().numpy().view(np.uint32), kbar64.astype(np.float32).view(np.uint32))
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_select_matches_oracle(small_cases, name):
+    cfg, h, d, dm, kbar64, rows, sel_o, s_m = small_cases(name)
+    dims = sg.sgqa_dims.of(cfg)
+    ws = _ws(dims)
+    kbar = torch.empty((cfg.batch, cfg.T // cfg.B, cfg.d_idx), device="cuda")
+    sg.sgqa_compress_keys(dims, d["k_idx"], kbar, None)
+    sel = torch.full((cfg.batch, cfg.T, cfg.G, cfg.Kb), -7, dtype=torch.int32, device="cuda")
+    sg.sgqa_select(dims, d["q_idx"], kbar, sel, ws)
+    _status_ok(ws)
+    gsel = sel.cpu().numpy().reshape(-1, cfg.G, cfg.Kb)
+    n_tie = compare_selection(dm, kbar64, rows, h["q_idx"].reshape(len(rows), -1), gsel, sel_o, s_m)
+    assert n_tie <= max(2, len(rows) * cfg.G // 100), f"{n_tie} near-tie rows"
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_attend_with_oracle_selection(small_cases, name):
+    cfg, h, d, dm, kbar64, rows, sel_o, s_m = small_cases(name)
+    dims = sg.sgqa_dims.of(cfg)
+    ws = _ws(dims)
+    sel = torch.from_numpy(sel_o.reshape(cfg.batch, cfg.T, cfg.G, cfg.Kb)).cuda()
+    out = torch.full(shape_of(cfg, "q"), float("nan"), dtype=torch.bfloat16, device="cuda")
+    sg.sgqa_attend(dims, d["q"], d["k"], d["v"], d["gate"], sel, out, ws)
+    _status_ok(ws)
+    ref = oracle.attend(dm, rows, h["q"].reshape(len(rows), -1), h["k"], h["v"], h["gate"].reshape(len(rows), -1),
+                        sel_o)
+    assert_outputs_close(to_host(out), ref.reshape(shape_of(cfg, "q")), name)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_forward_matches_oracle(small_cases, name):
+    cfg, h, d, dm, kbar64, rows, sel_o, s_m = small_cases(name)
+    dims = sg.sgqa_dims.of(cfg)
+    ws = _ws(dims)
+    out = torch.full(shape_of(cfg, "q"), float("nan"), dtype=torch.bfloat16, device="cuda")
+    sel = torch.full((cfg.batch, cfg.T, cfg.G, cfg.Kb), -7, dtype=torch.int32, device="cuda")
+    sg.sgqa_forward(dims, d["q"], d["k"], d["v"], d["q_idx"], d["k_idx"], d["gate"], out, ws, sel_out=sel)
+    _status_ok(ws)
+    gsel = sel.cpu().numpy().reshape(-1, cfg.G, cfg.Kb)
+    compare_selection(dm, kbar64, rows, h["q_idx"].reshape(len(rows), -1), gsel, sel_o, s_m)
+    ref = oracle.attend(dm, rows, h["q"].reshape(len(rows), -1), h["k"], h["v"], h["gate"].reshape(len(rows), -1),
+                        gsel)
+    assert_outputs_close(to_host(out), ref.reshape(shape_of(cfg, "q")), name)
+    # same result without sel_out (selection kept in the workspace) and run to run
+    out2 = torch.empty_like(out)
+    sg.sgqa_forward(dims, d["q"], d["k"], d["v"], d["q_idx"], d["k_idx"], d["gate"], out2, ws)
+    _status_ok(ws)
+    assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
+
+
+def test_forward_chunked_selection_is_identical():
+    # T above the 32768-row selection chunk: the chunked path must give the same bits
+    cfg = Config("chunked", 1, 40000, 4, 1, 64, 32, 8, 256, 3000, 14)
+    dims = sg.sgqa_dims.of(cfg)
+    d = device_inputs(cfg)
+    ws = _ws(dims)
+    out1 = torch.empty(shape_of(cfg, "q"), dtype=torch.bfloat16, device="cuda")
+    out2 = torch.empty_like(out1)
+    sel = torch.empty((1, cfg.T, cfg.G, cfg.Kb), dtype=torch.int32, device="cuda")
+    sg.sgqa_forward(dims, d["q"], d["k"], d["v"], d["q_idx"], d["k_idx"], d["gate"], out1, ws, sel_out=sel)
+    sg.sgqa_forward(dims, d["q"], d["k"], d["v"], d["q_idx"], d["k_idx"], d["gate"], out2, ws)
+    _status_ok(ws)
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+
+
+def test_causality_on_gpu():
+    cfg = Config("causal", 1, 2500, 8, 2, 64, 32, 8, 256, 300, 15)
+    dims = sg.sgqa_dims.of(cfg)
+    h = host_inputs(cfg)
+    cut = 1234
+    h2 = {n: a.copy() for n, a in h.items()}
+    rng = np.random.default_rng(1)
+    for n in NAMES:
+        h2[n][:, cut + 1:] = rng.integers(0, 2 ** 15, size=h2[n][:, cut + 1:].shape, dtype=np.uint16) & 0x3F7F
+    outs = []
+    for hh in (h, h2):
+        d = {n: to_dev(hh[n], shape_of(cfg, n)) for n in NAMES}
+        ws = _ws(dims)
+        out = torch.empty(shape_of(cfg, "q"), dtype=torch.bfloat16, device="cuda")
+        sg.sgqa_forward(dims, d["q"], d["k"], d["v"], d["q_idx"], d["k_idx"], d["gate"], out, ws)
+        _status_ok(ws)
+        outs.append(to_host(out))
+    np.testing.assert_array_equal(outs[0][:, :cut + 1], outs[1][:, :cut + 1])
+    assert not np.array_equal(outs[0][:, cut + 1:], outs[1][:, cut + 1:])
+
+
+def test_invalid_selection_is_reported_not_faulted():
+    cfg = SMALL["tiny"]
+    dims = sg.sgqa_dims.of(cfg)
+    d = device_inputs(cfg)
+    ws = _ws(dims)
+    sel = torch.full((1, cfg.T, cfg.G, cfg.Kb), -1, dtype=torch.int32, device="cuda")
+    t = torch.arange(cfg.T, device="cuda")
+    sel[0, :, :, 0] = (t // cfg.B)[:, None].int()
+    sel[0, 100, 1, 1] = 10 ** 6          # a block far beyond row 100's own block
+    out = torch.empty(shape_of(cfg, "q"), dtype=torch.bfloat16, device="cuda")
+    sg.sgqa_attend(dims, d["q"], d["k"], d["v"], d["gate"], sel, out, ws)
+    torch.cuda.synchronize()
+    assert sg.sgqa_get_device_status(ws) == 6
+    sg.sgqa_reset_device_status(ws)
+    torch.cuda.synchronize()
+    assert sg.sgqa_get_device_status(ws) == 0
+    assert torch.isfinite(out.float()).all()
+
+
+def test_device_generator_matches_host_generator():
+    cfg = CONFIGS["128k"]
+    for name in NAMES:
+        t = torch.empty(shape_of(cfg, name, T=4096), dtype=torch.bfloat16, device="cuda")
+        c4 = cfg.replace(T=4096)
+        gen_device(c4, name, t)
+        got = to_host(t).reshape(4096, -1)
+        want = gen_rows(cfg, name, 0, np.arange(4096))
+        np.testing.assert_array_equal(got, want)
+
+
+def _decode_case(cfg, cache_len, n_new, check_seqs):
+    """Run one decode step after a cache of cache_len tokens and check sequences check_seqs."""
+    n_seq = cfg.batch
+    T_cap = ((cache_len + n_new + cfg.B - 1) // cfg.B) * cfg.B
+    dims = sg.sgqa_dims(n_seq, T_cap, cfg.Hq, cfg.G, cfg.d, cfg.d_idx, cfg.B, cfg.k)
+    caches = {}
+    for n in ("k", "v", "k_idx"):
+        caches[n] = torch.zeros(shape_of(cfg, n, T=T_cap, batch=n_seq), dtype=torch.bfloat16, device="cuda")
+        gen_device(cfg, n, caches[n], t0=0, n_t=cache_len)
+    kbar = torch.zeros((n_seq, T_cap // cfg.B, cfg.d_idx), device="cuda")
+    sg.sgqa_compress_keys(dims, caches["k_idx"], kbar, None)
+    new = {}
+    for n in NAMES:
+        new[n] = torch.empty((n_seq, n_new) + shape_of(cfg, n)[2:], dtype=torch.bfloat16, device="cuda")
+        gen_device(cfg, n, new[n], t0=cache_len, n_t=n_new, dst_t0=0)
+    ws = sg.alloc_workspace(sg.sgqa_decode_workspace_size(dims, n_new))
+    sg.sgqa_reset_device_status(ws)
+    out = torch.full((n_seq, n_new, cfg.Hq, cfg.d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    sel = torch.full((n_seq, n_new, cfg.G, cfg.Kb), -7, dtype=torch.int32, device="cuda")
+    sg.sgqa_decode(dims, cache_len, n_new, caches["k"], caches["v"], caches["k_idx"], kbar, new["q"], new["k"],
+                   new["v"], new["q_idx"], new["k_idx"], new["gate"], out, ws, sel_out=sel)
+    _status_ok(ws)
+    # idempotent at a fixed cache_len
+    out2 = torch.empty_like(out)
+    sg.sgqa_decode(dims, cache_len, n_new, caches["k"], caches["v"], caches["k_idx"], kbar, new["q"], new["k"],
+                   new["v"], new["q_idx"], new["k_idx"], new["gate"], out2, ws)
+    _status_ok(ws)
+    assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
+    Tn = cache_len + n_new
+    dm = oracle.dims(1, Tn, cfg.Hq, cfg.G, cfg.d, cfg.d_idx, cfg.B, cfg.k)
+    errs = []
+    for b in check_seqs:
+        kh = to_host(caches["k"][b:b + 1, :Tn])
+        vh = to_host(caches["v"][b:b + 1, :Tn])
+        kih = to_host(caches["k_idx"][b:b + 1, :Tn])
+        # the caches hold exactly the generator's rows (append included)
+        np.testing.assert_array_equal(kih[0, cache_len:], gen_rows(cfg, "k_idx", b, np.arange(cache_len, Tn)))
+        kbar64 = oracle.compress(dm, kih)
+        # the decode step's kbar update matches for the blocks it completed
+        j0, j1 = cache_len // cfg.B, Tn // cfg.B
+        if j1 > j0:
+            np.testing.assert_array_equal(kbar[b, j0:j1].cpu().numpy(), kbar64[0, j0:j1].astype(np.float32))
+        rows = np.array([[0, cache_len + i] for i in range(n_new)], dtype=np.int32)
+        qi = to_host(new["q_idx"][b]).reshape(n_new, -1)
+        sel_o, s_m, _ = oracle.select(dm, kbar64, rows, qi)
+        gsel = sel[b].cpu().numpy()
+        compare_selection(dm, kbar64, rows, qi, gsel, sel_o, s_m)
+        ref = oracle.attend(dm, rows, to_host(new["q"][b]).reshape(n_new, -1), kh, vh,
+                            to_host(new["gate"][b]).reshape(n_new, -1), gsel)
+        errs.append(assert_outputs_close(to_host(out[b]), ref.reshape(n_new, cfg.Hq, cfg.d), f"decode seq {b}"))
+    return errs
+
+
+def test_decode_small_matches_oracle():
+    cfg = Config("dec_small", 3, 5000, 32, 4, 128, 64, 8, 512, 600, 16)
+    _decode_case(cfg, 4996, 4, [0, 2])          # new tokens complete block 624
+    _decode_case(cfg, 4000, 4, [1])             # all new tokens in one partial block
+    _decode_case(cfg, 3, 4, [0])                # tiny cache: fewer candidates than the budget
+
+
+def test_decode_n1_and_b1():
+    _decode_case(Config("dec_b1", 2, 3000, 8, 2, 64, 32, 1, 64, 300, 17), 2500, 3, [1])
+    _decode_case(Config("dec_n1", 2, 3000, 8, 2, 64, 32, 8, 128, 300, 18), 2999, 1, [0])
+
+
+# ---- full-size workloads, sampled rows, the benchmark's launch configuration ----------------
+
+def _full_size_forward(cfg, n_rows, seed):
+    dims = sg.sgqa_dims.of(cfg)
+    d = device_inputs(cfg)
+    ws = _ws(dims)
+    out = torch.full(shape_of(cfg, "q"), float("nan"), dtype=torch.bfloat16, device="cuda")
+    sel = torch.full((cfg.batch, cfg.T, cfg.G, cfg.Kb), -7, dtype=torch.int32, device="cuda")
+    sg.sgqa_forward(dims, d["q"], d["k"], d["v"], d["q_idx"], d["k_idx"], d["gate"], out, ws, sel_out=sel)
+    _status_ok(ws)
+    rows = sample_rows(cfg, n_rows, seed)
+    dm = oracle.dims_of(cfg)
+    kih, kh, vh = to_host(d["k_idx"]), to_host(d["k"]), to_host(d["v"])
+    kbar64 = oracle.compress(dm, kih)
+    pick = lambda n: to_host(d[n][rows[:, 0], rows[:, 1]]).reshape(len(rows), -1)
+    qi, qh, gh = pick("q_idx"), pick("q"), pick("gate")
+    sel_o, s_m, _ = oracle.select(dm, kbar64, rows, qi)
+    gsel = sel[rows[:, 0], rows[:, 1]].cpu().numpy()
+    n_tie = compare_selection(dm, kbar64, rows, qi, gsel, sel_o, s_m)
+    ref = oracle.attend(dm, rows, qh, kh, vh, gh, gsel)
+    err = assert_outputs_close(to_host(out[rows[:, 0], rows[:, 1]]), ref.reshape(len(rows), cfg.Hq, cfg.d), cfg.name)
+    # replay the oracle's selection through sgqa_attend
+    sel[rows[:, 0], rows[:, 1]] = torch.from_numpy(sel_o).cuda()
+    out2 = torch.empty_like(out)
+    sg.sgqa_attend(dims, d["q"], d["k"], d["v"], d["gate"], sel, out2, ws)
+    _status_ok(ws)
+    ref2 = oracle.attend(dm, rows, qh, kh, vh, gh, sel_o)
+    assert_outputs_close(to_host(out2[rows[:, 0], rows[:, 1]]), ref2.reshape(len(rows), cfg.Hq, cfg.d), cfg.name)
+    del d, out, out2, sel, ws
+    torch.cuda.empty_cache()
+    return n_tie, err
+
+
+@pytest.mark.parametrize("name", ["32k", "128k", "64k_b8", "64k_b1"])
+def test_full_size_prefill_sampled(name):
+    n_tie, err = _full_size_forward(CONFIGS[name], 48, 100)
+    print(f"{name}: near-tie rows {n_tie}; max-abs/mean-abs/rel-rms {err}")
+
+
+def test_full_size_decode_1m_sampled():
+    cfg = CONFIGS["decode_1m"]
+    errs = _decode_case(cfg, cfg.T, DECODE_NEW, [0, 31])
+    print(f"decode 1M: {errs}")
