@@ -140,6 +140,7 @@ int sgqa_compress_keys(const sgqa_dims* dims, const uint16_t* k_idx, float* kbar
                        void* stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
+  if (dims->T / dims->B == 0) return SGQA_OK;  // no complete block: nothing to write
   if (!aligned16(k_idx) || !aligned16(kbar)) return SGQA_ERR_INVALID_ARG;
   (void)ws;
   (void)ws_bytes;
@@ -151,7 +152,7 @@ int sgqa_select(const sgqa_dims* dims, const uint16_t* q_idx, const float* kbar,
                 size_t ws_bytes, void* stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
-  if (!aligned16(q_idx) || !aligned16(kbar) || !aligned16(sel)) return SGQA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || (dims->T >= dims->B && !aligned16(kbar)) || !aligned16(sel)) return SGQA_ERR_INVALID_ARG;
   const PrefillWs w = prefill_layout(dims, ws);
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < (size_t)((uint8_t*)w.sel - (uint8_t*)ws))
     return SGQA_ERR_WORKSPACE;

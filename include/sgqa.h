@@ -93,7 +93,8 @@ int sgqa_get_device_status(const void* ws, size_t ws_bytes, int* status);
 /* Step (1): block-mean compression of the shared index keys (see the header comment).
  * k_idx [batch, T, d_idx] bf16 -> kbar [batch, T/B, d_idx] fp32. The block's keys are summed
  * in fp64 in token order and rounded once, so kbar is the fp32 rounding (RNE) of the block
- * mean. This call uses no workspace: ws may be NULL and ws_bytes 0. */
+ * mean. This call uses no workspace: ws may be NULL and ws_bytes 0. With T < B there is no
+ * complete block and kbar may be NULL. */
 int sgqa_compress_keys(const sgqa_dims* dims, const uint16_t* k_idx, float* kbar, void* ws,
                        size_t ws_bytes, void* stream);
 
