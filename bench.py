@@ -327,7 +327,8 @@ def run_ours(args, world, rank):
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         rows = sample_rows_strided(cfg, CPU_STRIDE)
         full = {n: to_host(dev[n][:1]) for n in ("k", "v", "k_idx")}
-        part = {n: to_host(dev[n][0, rows[:, 1]]).reshape(len(rows), -1) for n in ("q", "q_idx", "gate")}
+        ti = torch.from_numpy(rows[:, 1].astype(np.int64)).cuda()
+        part = {n: to_host(dev[n][0].index_select(0, ti)).reshape(len(rows), -1) for n in ("q", "q_idx", "gate")}
         cpu_in = (rows, full, part)
     # release the prefill buffers before the decode workload
     del dev, out, sel, kbar, ws, host, out_h
