@@ -26,7 +26,7 @@ STATUS_NAMES = {0: "SGQA_OK", 1: "SGQA_ERR_INVALID_ARG", 2: "SGQA_ERR_UNSUPPORTE
 # every symbol include/sgqa.h declares
 EXPORTS = ["sgqa_status_string", "sgqa_version", "sgqa_workspace_size", "sgqa_decode_workspace_size",
            "sgqa_reset_device_status", "sgqa_get_device_status", "sgqa_compress_keys", "sgqa_select",
-           "sgqa_attend", "sgqa_forward", "sgqa_decode"]
+           "sgqa_attend", "sgqa_forward", "sgqa_decode", "sgqa_decode_noalloc"]
 
 
 class SgqaError(RuntimeError):
@@ -72,8 +72,9 @@ def load_library():
     L.sgqa_attend.argtypes = [D, P, P, P, P, P, P, P, S, P]
     L.sgqa_forward.argtypes = [D, P, P, P, P, P, P, P, P, P, S, P]
     L.sgqa_decode.argtypes = [D, I, I] + [P] * 13 + [S, P]
+    L.sgqa_decode_noalloc.argtypes = [D, I, I] + [P] * 12 + [P]
     for n in ("sgqa_reset_device_status", "sgqa_get_device_status", "sgqa_compress_keys", "sgqa_select",
-              "sgqa_attend", "sgqa_forward", "sgqa_decode"):
+              "sgqa_attend", "sgqa_forward", "sgqa_decode", "sgqa_decode_noalloc"):
         getattr(L, n).restype = I
     _lib = L
     return L
@@ -171,3 +172,17 @@ def sgqa_decode(dims, cache_len, n_new, k_cache, v_cache, kidx_cache, kbar_cache
         _ptr(kidx_cache, "kidx_cache"), _ptr(kbar_cache, "kbar_cache"), _ptr(q_new, "q_new"), _ptr(k_new, "k_new"),
         _ptr(v_new, "v_new"), _ptr(qidx_new, "qidx_new"), _ptr(kidx_new, "kidx_new"), _ptr(gate_new, "gate_new"),
         _ptr(out, "out"), _ptr(sel_out, "sel_out"), _ptr(ws, "ws"), ws.numel(), _stream(stream)))
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def sgqa_decode_noalloc(dims, cache_len, n_new, k_cache, v_cache, kidx_cache, kbar_cache, q_new, k_new, v_new,
+                        qidx_new, kidx_new, gate_new, out, sel_out=None, stream=None):
+    """sgqa_decode without a workspace: the library's fixed device scratch array is used instead
+    (for callers that cannot allocate device memory; see include/sgqa.h)."""
+    _check("sgqa_decode_noalloc", load_library().sgqa_decode_noalloc(
+        ctypes.byref(dims), int(cache_len), int(n_new), _ptr(k_cache, "k_cache"), _ptr(v_cache, "v_cache"),
+        _ptr(kidx_cache, "kidx_cache"), _ptr(kbar_cache, "kbar_cache"), _ptr(q_new, "q_new"), _ptr(k_new, "k_new"),
+        _ptr(v_new, "v_new"), _ptr(qidx_new, "qidx_new"), _ptr(kidx_new, "kidx_new"), _ptr(gate_new, "gate_new"),
+        _ptr(out, "out"), _ptr(sel_out, "sel_out"), _stream(stream)))

@@ -137,6 +137,30 @@ int sgqa_decode(const sgqa_dims* dims, int cache_len, int n_new, uint16_t* k_cac
                 const uint16_t* kidx_new, const uint16_t* gate_new, uint16_t* out,
                 int32_t* sel_out, void* ws, size_t ws_bytes, void* stream);
 
+/* Size of the library-owned scratch array that sgqa_decode_noalloc uses (16 MiB). */
+#define SGQA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* A decode step for callers that cannot allocate device memory. No counterpart on the pages:
+ * this is a deployment variant of sgqa_decode, not a step of the method.
+ * Same arguments, results and cache updates as sgqa_decode, but no ws: the step's scratch (status
+ * word, indexer scores, selection, split-K partials) lives in one file-scope __device__ array of
+ * SGQA_NOALLOC_SCRATCH_BYTES bytes that every GPU using the library holds until the process ends.
+ * Nothing is allocated or freed: no cudaMalloc/cudaFree and no allocating library routine.
+ *   - Returns SGQA_ERR_WORKSPACE if sgqa_decode_workspace_size(dims, n_new) exceeds
+ *     SGQA_NOALLOC_SCRATCH_BYTES (e.g. 32 sequences at a 1M-token cache need more; use sgqa_decode),
+ *     SGQA_ERR_INVALID_ARG / SGQA_ERR_UNSUPPORTED as sgqa_decode does.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
+ *     that device current) and caches it; make that first call before any stream capture.
+ *   - Each call zeroes the status word (on `stream`) before its kernels; the device status is not
+ *     readable through this entry point (use sgqa_decode with a workspace when it is needed).
+ *   - All calls share the array and it keeps the last call's contents: calls that overlap on the
+ *     GPU (other streams, other host threads) race; serialise them. */
+int sgqa_decode_noalloc(const sgqa_dims* dims, int cache_len, int n_new, uint16_t* k_cache,
+                        uint16_t* v_cache, uint16_t* kidx_cache, float* kbar_cache,
+                        const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new,
+                        const uint16_t* qidx_new, const uint16_t* kidx_new,
+                        const uint16_t* gate_new, uint16_t* out, int32_t* sel_out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
