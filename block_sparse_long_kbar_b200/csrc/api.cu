@@ -32,6 +32,7 @@ int check_dims(const sgqa_dims* d) {
 
 struct PrefillWs {
   int* status;
+  void* plan;
   float* kbar;
   uint16_t* hi;
   uint16_t* lo;
@@ -47,6 +48,8 @@ PrefillWs prefill_layout(const sgqa_dims* d, void* ws) {
   size_t off = kStatusBytes;
   uint8_t* base = static_cast<uint8_t*>(ws);
   w.status = reinterpret_cast<int*>(base);
+  w.plan = base + off;
+  off += plan_bytes((long)d->batch * d->T * d->G, d->batch * d->G, d->T);
   w.kbar = reinterpret_cast<float*>(base + off);
   off += align256(nk * 4);
   w.hi = reinterpret_cast<uint16_t*>(base + off);
@@ -92,6 +95,16 @@ DecodeWs decode_layout(const sgqa_dims* d, int n_new, void* ws) {
 }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? SGQA_OK : SGQA_ERR_CUDA; }
+
+// Prefill attention for query rows [a.t_begin, a.t_end): schedule the rows by selection
+// similarity, then the tiled union kernel; shapes it does not cover use the per-row kernel.
+cudaError_t launch_prefill_attend(const AttendArgs& a, void* plan_ws, cudaStream_t s) {
+  if (!attend_tiles_supported(a.Hq, a.G, a.B)) return launch_attend(a, s);
+  const uint32_t* perm = nullptr;
+  cudaError_t e = launch_plan(a.sel, a.sel_T, a.sel_t0, a.batch, a.G, a.Kb, a.B, a.t_begin, a.t_end, plan_ws, &perm, s);
+  if (e != cudaSuccess) return e;
+  return launch_attend_tiles(a, perm, s);
+}
 
 }  // namespace
 
@@ -181,10 +194,10 @@ int sgqa_attend(const sgqa_dims* dims, const uint16_t* q, const uint16_t* k, con
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gate) || !aligned16(sel) || !aligned16(out))
     return SGQA_ERR_INVALID_ARG;
   const PrefillWs w = prefill_layout(dims, ws);
-  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < (size_t)kStatusBytes) return SGQA_ERR_WORKSPACE;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < w.bytes) return SGQA_ERR_WORKSPACE;
   AttendArgs a = prefill_attend_args(dims, q, k, v, gate, out, w.status);
   a.sel = sel; a.sel_T = dims->T; a.sel_t0 = 0; a.t_begin = 0; a.t_end = dims->T;
-  return cuda_status(launch_attend(a, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_prefill_attend(a, w.plan, static_cast<cudaStream_t>(stream)));
 }
 
 int sgqa_forward(const sgqa_dims* dims, const uint16_t* q, const uint16_t* k, const uint16_t* v,
@@ -215,7 +228,7 @@ int sgqa_forward(const sgqa_dims* dims, const uint16_t* q, const uint16_t* k, co
     sa.t_begin = t0; sa.t_end = t1;
     if (launch_select(sa, s) != cudaSuccess) return SGQA_ERR_CUDA;
     aa.sel = sa.sel; aa.sel_T = sa.sel_T; aa.sel_t0 = sa.sel_t0; aa.t_begin = t0; aa.t_end = t1;
-    if (launch_attend(aa, s) != cudaSuccess) return SGQA_ERR_CUDA;
+    if (launch_prefill_attend(aa, w.plan, s) != cudaSuccess) return SGQA_ERR_CUDA;
   }
   return SGQA_OK;
 }

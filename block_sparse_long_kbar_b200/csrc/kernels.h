@@ -51,6 +51,16 @@ cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s);
 cudaError_t launch_attend_merge(const AttendArgs& a, cudaStream_t s);
 size_t attend_part_bytes(int units, int splits, int R, int d);
 
+// Query scheduling for the tiled attention: per (sequence, group) segment, the rows of
+// [t_begin, t_end) ordered by a MinHash signature of their selection (stable in t).
+// *perm_out receives [batch * G][t_end - t_begin] row offsets (t - t_begin), inside ws.
+size_t plan_bytes(long units, int n_seg, int n_per_seg);
+cudaError_t launch_plan(const int32_t* sel, int sel_T, int sel_t0, int batch, int G, int Kb, int B, int t_begin,
+                        int t_end, void* ws, const uint32_t** perm_out, cudaStream_t s);
+// K3 tiled: tiles of consecutive rows of perm, union of their selections (requires ascending rows).
+bool attend_tiles_supported(int Hq, int G, int B);
+cudaError_t launch_attend_tiles(const AttendArgs& a, const uint32_t* perm, cudaStream_t s);
+
 // Decode helpers.
 cudaError_t launch_append(uint16_t* dst, const uint16_t* src, int batch, long row_elems, long dst_seq_stride,
                           long dst_off, long n_elems_per_seq, cudaStream_t s);

@@ -108,8 +108,10 @@ int sgqa_select(const sgqa_dims* dims, const uint16_t* q_idx, const float* kbar,
 
 /* Steps (3)+(4): gated attention of every query row over a given selection.
  * q, gate [batch, T, Hq, d], k, v [batch, T, G, d] bf16; sel [batch, T, G, k/B] int32 in the
- * format sgqa_select writes (any order of valid entries is accepted; entries > t/B are
- * rejected by a device check and skipped) -> out [batch, T, Hq, d] bf16. */
+ * format sgqa_select writes: strictly ascending block ids <= t/B, then -1 padding (entries that
+ * break this are flagged by a device check (SGQA_ERR_DEVICE_CHECK) and skipped)
+ * -> out [batch, T, Hq, d] bf16. Rows are scheduled in tiles of rows with similar selections
+ * (a deterministic function of sel); each tile gathers the union of its rows' blocks once. */
 int sgqa_attend(const sgqa_dims* dims, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                 const uint16_t* gate, const int32_t* sel, uint16_t* out, void* ws,
                 size_t ws_bytes, void* stream);

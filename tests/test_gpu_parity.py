@@ -31,6 +31,7 @@ SMALL = {
     "dense": Config("dense", 1, 300, 8, 2, 64, 32, 8, 304, 64, 11),
     "t9": Config("t9", 3, 9, 8, 2, 64, 32, 8, 16, 4, 12),
     "t1": Config("t1", 2, 1, 4, 4, 128, 64, 8, 64, 4, 13),
+    "r3_rowkernel": Config("r3_rowkernel", 1, 1200, 12, 4, 64, 32, 8, 256, 150, 19),
 }
 
 
