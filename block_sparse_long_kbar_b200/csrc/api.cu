@@ -175,6 +175,9 @@ int sgqa_select(const sgqa_dims* dims, const uint16_t* q_idx, const float* kbar,
   a.batch = dims->batch; a.T = dims->T; a.G = dims->G; a.d_idx = dims->d_idx; a.B = dims->B;
   a.Kb = dims->k / dims->B; a.t_begin = 0; a.t_end = dims->T; a.sel_T = dims->T; a.sel_t0 = 0;
   a.status = w.status;
+  if (launch_split_planes(kbar, w.hi, w.lo, (long)dims->batch * (dims->T / dims->B) * dims->d_idx, s) !=
+      cudaSuccess)
+    return SGQA_ERR_CUDA;
   return cuda_status(launch_select(a, s));
 }
 
@@ -250,7 +253,7 @@ int sgqa_decode(const sgqa_dims* dims, int cache_len, int n_new, uint16_t* k_cac
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int T = dims->T, G = dims->G, d = dims->d, di = dims->d_idx, B = dims->B, Kb = dims->k / dims->B;
   const int nblk = T / B;
-  cudaError_t e;
+  cudaError_t e = cudaSuccess;
   // 1. append the new rows
   if ((e = launch_append(k_cache, k_new, dims->batch, (long)G * d, (long)T * G * d, (long)cache_len * G * d,
                          (long)n_new * G * d, s)) != cudaSuccess)
