@@ -40,7 +40,9 @@ constexpr int kRows = 128;
 constexpr int kN = 128;          // candidate blocks per MMA tile
 constexpr int kStages = 2;
 constexpr int kHistStride = 257;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;     // two per TMEM lane quadrant: each histograms half the columns
+constexpr int kThreads = (kEpiWarps + 2) * 32;
+constexpr int kProducerWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
 constexpr int kMaxPasses = 5;
 
 template <int DI>
@@ -59,29 +61,30 @@ struct SelShared {
   volatile int signals;
   volatile int abort_flag;
   int more[kMaxPasses + 1];
-  int vote_cnt[kMaxPasses];
-  int vote_any[kMaxPasses];
+  int vote_cnt[3 * kMaxPasses];
+  int vote_any[3 * kMaxPasses];
 };
 
-// "Is any epilogue row still unresolved before pass p?": every epilogue warp adds its vote and
-// waits (bounded, abort-aware) until all four have voted. Returns 1/0, or -1 on giving up.
-__device__ __forceinline__ int epi_vote_any(SelShared* sh, int p, bool v) {
+// Bounded barrier + "any" vote among the epilogue warps (slot = a fresh index per use): every
+// epilogue warp adds its vote and waits (bounded, abort-aware) until all have voted. Returns 1/0,
+// or -1 on giving up.
+__device__ __forceinline__ int epi_vote_any(SelShared* sh, int slot, bool v) {
   const int lane = threadIdx.x & 31;
   const unsigned any = __any_sync(0xFFFFFFFFu, v);
   int res = 0;
   if (lane == 0) {
-    if (any) atomicOr(&sh->vote_any[p], 1);
+    if (any) atomicOr(&sh->vote_any[slot], 1);
     __threadfence_block();
-    atomicAdd(&sh->vote_cnt[p], 1);
+    atomicAdd(&sh->vote_cnt[slot], 1);
     const uint64_t t0 = tc::globaltimer();
-    volatile int* cnt = &sh->vote_cnt[p];
+    volatile int* cnt = &sh->vote_cnt[slot];
     res = 1;
-    while (*cnt < 4) {
+    while (*cnt < kEpiWarps) {
       if (sh->abort_flag || tc::globaltimer() - t0 > tc::kWaitLimitNs) { res = -1; break; }
     }
     if (res > 0) {
       __threadfence_block();
-      res = *(volatile int*)&sh->vote_any[p] ? 1 : 0;
+      res = *(volatile int*)&sh->vote_any[slot] ? 1 : 0;
     }
   }
   return __shfl_sync(0xFFFFFFFFu, res, 0);
@@ -137,21 +140,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&sh->acc_full[s], 1);
-      tc::mbar_init(&sh->acc_empty[s], 4);
+      tc::mbar_init(&sh->acc_empty[s], kEpiWarps);
     }
     tc::mbar_init(&sh->a_full, 1);
     sh->signals = 0;
     sh->abort_flag = 0;
-    for (int p = 0; p < kMaxPasses; ++p) sh->vote_cnt[p] = sh->vote_any[p] = 0;
+    for (int p = 0; p < 3 * kMaxPasses; ++p) sh->vote_cnt[p] = sh->vote_any[p] = 0;
     tc::fence_mbar_init();
   }
-  if (warp == 5) tc::tmem_alloc(&sh->tmem, 256);
+  if (warp == kMmaWarp) tc::tmem_alloc(&sh->tmem, 256);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = sh->tmem;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ---------------- TMA producer ----------------
     if (lane == 0 && n_nt > 0) {
       tc::prefetch_tensormap(&map_q);
@@ -193,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mbar_wait(&sh->a_full, 0, &no_abort);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
     if (lane == 0 && n_nt > 0) {
       const uint32_t idesc = tc::idesc_bf16_f32(kRows, kN);
@@ -240,8 +243,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ---------------- epilogue: one row per thread ----------------
-    const int r = tid;
+    // ---------------- epilogue: one row per thread pair ----------------
+    // Warps w and w + 4 read TMEM lane quadrant w % 4 (row r = 32 * (w % 4) + lane); in histogram
+    // passes each takes half of every tile's columns (atomics on the row's shared histogram); in
+    // the emit pass the lower warp streams all columns in order and the upper one only releases
+    // the accumulators.
+    const int quad = warp & 3, half = warp >> 2;
+    const int r = quad * 32 + lane;
     const int t = tq0 + r / G, g = r % G;
     const bool valid = t <= t_last;
     const int c = valid ? t / a.B : 0;
@@ -252,26 +260,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (rem == 0) { prefix = 0xFFFFFFFFu; mask = 0xFFFFFFFFu; done = true; }
     uint32_t* my_hist = hist + r * kHistStride;
     int32_t* out = a.sel + (((long)b * a.sel_T + (t - a.sel_t0)) * G + g) * (long)a.Kb;
-    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
     long k = 0;
     int pos = 0, eq_taken = 0;
     bool aborted = false;
     for (int pass = 0; pass < kMaxPasses; ++pass) {
-      const int vote = epi_vote_any(sh, pass, !done);
+      // zero the histograms for this pass, then a barrier+vote: is any row still unresolved?
+      if (half == 0 && !done && pass < kMaxPasses - 1)
+        for (int i = 0; i < 256; ++i) my_hist[i] = 0;
+      const int vote = epi_vote_any(sh, 3 * pass, !done);
       if (vote < 0) {
-        if (!sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
+        if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
         sh->abort_flag = 1;
         break;
       }
       const bool is_emit = vote == 0 || pass == kMaxPasses - 1;
-      if (r == 0) {
+      if (warp == 0 && lane == 0) {
         sh->more[pass] = is_emit ? 0 : 1;
         __threadfence_block();
         sh->signals = pass + 1;
       }
       const int shift = 24 - 8 * pass;
-      if (!is_emit && !done)
-        for (int i = 0; i < 256; ++i) my_hist[i] = 0;
       for (int i = 0; i < n_nt; ++i, ++k) {
         const int buf = (int)(k & 1);
         if (!warp_wait(&sh->acc_full[buf], (uint32_t)((k >> 1) & 1), &sh->abort_flag)) {
@@ -281,29 +290,43 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc::fence_after_sync();
-#pragma unroll 1
-        for (int chunk = 0; chunk < kN / 32; ++chunk) {
-          uint32_t v[32];
-          tc::tmem_ld32(tmem + lane_base + (uint32_t)(buf * kN + chunk * 32), v);
-          const int j0 = i * kN + chunk * 32;
+        if (!is_emit) {
+          uint32_t v[64];
+          tc::tmem_ld64(tmem + lane_base + (uint32_t)(buf * kN + half * 64), v);
+          const int j0 = i * kN + half * 64;
           const int lim = c - j0;
-          if (!is_emit) {
-            if (!done) {
+          if (!done && lim > 0) {
+            if (pass == 0) {  // every key matches the empty prefix
+              if (lim >= 64) {
 #pragma unroll
-              for (int q = 0; q < 32; ++q) {
-                if (q < lim) {
-                  const uint32_t key = score_key(__uint_as_float(v[q]));
-                  if ((key & mask) == prefix) atomicAdd(&my_hist[(key >> shift) & 255u], 1u);
-                }
+                for (int q = 0; q < 64; ++q) atomicAdd(&my_hist[score_key(__uint_as_float(v[q])) >> 24], 1u);
+              } else {
+#pragma unroll
+                for (int q = 0; q < 64; ++q)
+                  if (q < lim) atomicAdd(&my_hist[score_key(__uint_as_float(v[q])) >> 24], 1u);
+              }
+            } else {
+#pragma unroll
+              for (int q = 0; q < 64; ++q) {
+                const uint32_t key = score_key(__uint_as_float(v[q]));
+                if (q < lim && (key & mask) == prefix) atomicAdd(&my_hist[(key >> shift) & 255u], 1u);
               }
             }
-          } else if (valid) {
+          }
+        } else if (half == 0) {
+#pragma unroll 1
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t v[64];
+            tc::tmem_ld64(tmem + lane_base + (uint32_t)(buf * kN + hh * 64), v);
+            const int j0 = i * kN + hh * 64;
+            const int lim = c - j0;
+            if (valid && lim > 0) {
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
-              if (q < lim) {
+              for (int q = 0; q < 64; ++q) {
                 const uint32_t key = score_key(__uint_as_float(v[q])) & mask;
-                bool take = key > prefix;
-                if (key == prefix) take = eq_taken++ < rem;
+                const bool eq = key == prefix;
+                const bool take = q < lim && (key > prefix || (eq && eq_taken < rem));
+                eq_taken += (q < lim && eq) ? 1 : 0;
                 if (take && pos < m) out[pos++] = j0 + q;
               }
             }
@@ -315,11 +338,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (aborted) break;
       if (is_emit) {
-        if (valid) {
+        if (half == 0 && valid) {
           if (pos != m) report(a.status, SGQA_ERR_DEVICE_CHECK);
           out[pos++] = c;
           for (; pos < a.Kb; ++pos) out[pos] = -1;
         }
+        break;
+      }
+      // both halves' histogram updates are complete before either reads the histogram
+      if (epi_vote_any(sh, 3 * pass + 1, false) < 0) {
+        if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
+        sh->abort_flag = 1;
         break;
       }
       if (!done) {
@@ -337,12 +366,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         done = (rem == nb) || (mask == 0xFFFFFFFFu);
       }
+      // both halves have read the histogram before the next pass zeroes it
+      if (epi_vote_any(sh, 3 * pass + 2, false) < 0) {
+        if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
+        sh->abort_flag = 1;
+        break;
+      }
     }
   }
 
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, 256);
   }
