@@ -103,6 +103,7 @@ cudaError_t launch_prefill_attend(const AttendArgs& a, void* plan_ws, cudaStream
   const uint32_t* perm = nullptr;
   cudaError_t e = launch_plan(a.sel, a.sel_T, a.sel_t0, a.batch, a.G, a.Kb, a.B, a.t_begin, a.t_end, plan_ws, &perm, s);
   if (e != cudaSuccess) return e;
+  if (attend_tc_supported(a.Hq, a.G, a.B, a.d)) return launch_attend_tc(a, perm, s);
   return launch_attend_tiles(a, perm, s);
 }
 

@@ -1,0 +1,490 @@
+// K3 on the 5th-generation tensor cores: gated attention for a tile of 128 query rows (128/R
+// queries x R heads of one KV group) over the union of their selected blocks.
+//
+// Step 5 Preview pages (mo.ai.kr, "Step 5 Preview agentic work design", section "model
+// structure and training stability"): the full-context layer is Sparse GQA on top of Gated GQA;
+// every KV group attends only to its selected blocks, and queries whose selections overlap are
+// batched for GPU utilisation. The rows of a tile come from the scheduling permutation (plan.cu)
+// that puts rows with similar selections together.
+//
+// Data movement and math:
+//   * Q tile: 128 rows x d bf16 in shared memory (K-major, 128B swizzle), loaded once.
+//   * The union of the tile's selections is built window by window over block ids (a shared
+//     bitmap of 32-bit query masks per block, one cursor per query) and consumed as 16-token
+//     superblocks aligned on block ids. Each superblock's K and V rows of the group arrive by
+//     3-D TMA boxes (16 tokens x 64 dims, 128B swizzle) into a 4-stage ring.
+//   * S[128 x 16] = Q K^T: tcgen05.mma (kind::f16, M=128, N=16) into TMEM, double-buffered.
+//   * Softmax: one thread per row (TMEM lane), masks from the bitmap (query selected the block,
+//     token <= query position). Pass 1 streams the union once for the exact row maxima (S only);
+//     pass 2 streams it again, forms P = exp2((S - max) * log2e / sqrt(d)) in bf16 into shared
+//     memory and accumulates O[128 x d] += P V with tcgen05.mma (V as an MN-major operand) in
+//     TMEM. With the exact maximum known up front there is no rescaling of O, and because
+//     superblocks are aligned on block ids and unselected slots contribute exact zeros, every
+//     row's arithmetic is the same whatever rows share its tile (bitwise causal, chunk-invariant).
+//   * Epilogue: O / l times sigmoid(gate_logits), bf16.
+// Warp roles: warp 0 issues TMA, warp 1 allocates TMEM and issues MMAs, warps 2-5 run the
+// softmax and the epilogue; all six build the union. Every wait is bounded by %globaltimer: on
+// expiry the kernel records SGQA_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and
+// returns.
+#include <cmath>
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_common.cuh"
+
+namespace sgqa {
+namespace {
+
+constexpr int kUnit = 16;    // tokens per superblock
+constexpr int kWin = 2048;   // block ids per union window
+constexpr int kNS = 4;       // K/V stages
+constexpr int kThreads = 192;
+constexpr int kM = 128;
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct AtcCfg {
+  static constexpr int kHalves = D / 64;
+  static constexpr int kQ = kM * D * 2;                 // [half][128 rows][128 B]
+  static constexpr int kKsb = kHalves * kUnit * 128;    // one superblock of K (or V): [half][16][128 B]
+  static constexpr int kStage = 2 * kKsb;               // K then V
+  static constexpr int kP = kM * kUnit * 2;             // P tile 128 x 16 bf16
+  static constexpr int kSmem = 1024 + kQ + kNS * kStage + 2 * kP + 2 * kWin * 4 + 1024;
+};
+
+struct AtcShared {
+  uint64_t kv_full[kNS], kv_empty[kNS], s_full[2], s_empty[2], p_full[2], p_empty[2], o_done;
+  uint32_t tmem;
+  volatile int abort_flag;
+  int t[32];
+  int cur[32];
+  int scan[8];
+  int nu, maxc;
+};
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = tc::mbar_wait(bar, parity, abort) ? 1 : 0;
+  return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
+}
+
+template <int D, int R>
+__global__ void __launch_bounds__(kThreads, 2)
+    attend_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+                     AttendArgs a, const uint32_t* __restrict__ perm, int n_per_seg, int tiles_per_seg, int lb) {
+  using C = AtcCfg<D>;
+  constexpr int QT = kM / R;  // queries per tile (<= 32)
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* sQ = smem;
+  uint8_t* sKV = sQ + C::kQ;                             // [stage][K|V][half][16][128 B]
+  uint8_t* sP = sKV + kNS * C::kStage;                   // [2][16 groups][2 chunks][8 rows][16 B]
+  uint32_t* wmask = reinterpret_cast<uint32_t*>(sP + 2 * C::kP);
+  int32_t* usb = reinterpret_cast<int32_t*>(wmask + kWin);
+  AtcShared* sh = reinterpret_cast<AtcShared*>(usb + kWin);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int B = a.B, G = a.G;
+  const int seg = blockIdx.x / tiles_per_seg, tile = blockIdx.x % tiles_per_seg;
+  const int b = seg / G, g = seg % G;
+
+  if (tid == 0) {
+    for (int i = 0; i < kNS; ++i) {
+      tc::mbar_init(&sh->kv_full[i], 1);
+      tc::mbar_init(&sh->kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&sh->s_full[i], 1);
+      tc::mbar_init(&sh->s_empty[i], 4);
+      tc::mbar_init(&sh->p_full[i], 4);
+      tc::mbar_init(&sh->p_empty[i], 1);
+    }
+    tc::mbar_init(&sh->o_done, 1);
+    sh->abort_flag = 0;
+    sh->maxc = -1;
+    tc::fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid < QT) {
+    const int idx = tile * QT + tid;
+    const int t = idx < n_per_seg ? a.t_begin + (int)__ldg(perm + (long)seg * n_per_seg + idx) : -1;
+    sh->t[tid] = t;
+    if (t >= 0) atomicMax(&sh->maxc, t / B);
+  }
+  if (warp == 1) tc::tmem_alloc(&sh->tmem, 256);
+
+  // Q tile: row r = query r / R, head r % R; 16-byte chunk c of half h at
+  // h * 16 KB + r * 128 + ((c ^ (r & 7)) * 16) (the 128B-swizzled K-major layout).
+  __syncthreads();
+  for (int idx = tid; idx < kM * (D / 8); idx += kThreads) {
+    const int r = idx / (D / 8), cc = idx % (D / 8);
+    const int h = cc >> 3, c = cc & 7;
+    const int tq = sh->t[r / R];
+    const long row = tq >= 0 ? ((long)b * a.nQ + (tq - a.q_t0)) * a.Hq + (long)g * R + (r % R) : 0;
+    cp_async16(smem_u32(sQ + h * (kM * 128) + r * 128 + ((c ^ (r & 7)) * 16)), a.q + row * D + cc * 8,
+               tq >= 0 ? 16 : 0);
+  }
+  cp_async_commit();
+  cp_async_wait<0>();
+  tc::fence_proxy_async();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = sh->tmem;
+  const uint32_t tmem_o = tmem + 128;  // O: columns 128 .. 128 + D - 1; S buffers: columns 0 .. 31
+
+  // softmax role state (warps 2-5): TMEM lane quadrant warp % 4
+  const bool is_sm = warp >= 2;
+  const int quad = warp & 3;
+  const int r = quad * 32 + lane;
+  const int q_r = r / R, h_r = r % R;
+  const int t_r = is_sm ? sh->t[q_r] : -1;
+  float m_r = -INFINITY, l_r = 0.f;
+  const float sc = kLog2e / sqrtf((float)D);
+  const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
+
+  const int nwin = sh->maxc < 0 ? 0 : sh->maxc / kWin + 1;
+  const int spb = kUnit >> lb;  // blocks per superblock
+  long kc = 0;                  // superblocks streamed (producer & MMA ring position)
+  long scnt = 0;                // S buffer uses (MMA & softmax)
+  long pcnt = 0;                // P buffer uses (MMA & softmax, pass 2)
+  bool first_pv = true;
+  const uint32_t idesc_s = tc::idesc_bf16_f32(kM, kUnit);
+  const uint32_t idesc_pv = tc::idesc_bf16_f32(kM, D, true);
+
+  for (int pass = 0; pass < 2; ++pass) {
+    if (tid < QT) sh->cur[tid] = 0;
+    for (int win = 0; win < nwin; ++win) {
+      const int w0 = win * kWin, w1 = w0 + kWin;
+      // ---- union of this window (all warps) ----
+      for (int i = tid; i < kWin; i += kThreads) wmask[i] = 0;
+      __syncthreads();
+      for (int q = warp; q < QT; q += kThreads / 32) {
+        const int t = sh->t[q];
+        if (t < 0) continue;
+        const int cq = t / B;
+        const int32_t* row = a.sel + (((long)b * a.sel_T + (t - a.sel_t0)) * G + g) * (long)a.Kb;
+        int cur = sh->cur[q];
+        while (cur < a.Kb) {
+          const int e = cur + lane;
+          int j = e < a.Kb ? __ldg(row + e) : -1;
+          const int prev = __shfl_up_sync(0xFFFFFFFFu, j, 1);
+          const int before = lane > 0 ? prev : (cur > 0 ? __ldg(row + cur - 1) : -1);
+          if (j > cq || j < -1 || (j >= 0 && j <= before) || (j >= 0 && j < w0)) {
+            if (pass == 0) report(a.status, SGQA_ERR_DEVICE_CHECK);
+            j = -1;
+          }
+          const bool in = j >= w0 && j < w1;
+          const bool past = j < 0 || j >= w1;
+          if (in) atomicOr(&wmask[j - w0], 1u << q);
+          const unsigned stop = __ballot_sync(0xFFFFFFFFu, past);
+          const int adv = stop ? __ffs(stop) - 1 : 32;
+          cur += adv;
+          if (stop) {
+            const int first = __shfl_sync(0xFFFFFFFFu, j, adv);
+            if (first < 0) cur = a.Kb;
+            break;
+          }
+        }
+        if (lane == 0) sh->cur[q] = cur;
+      }
+      __syncthreads();
+      {
+        const int nsb_win = kWin / spb;
+        const int per = (nsb_win + kThreads - 1) / kThreads;
+        const int sb0 = min(nsb_win, tid * per), sb1 = min(nsb_win, sb0 + per);
+        int cnt = 0;
+        for (int sb = sb0; sb < sb1; ++sb) {
+          uint32_t any = 0;
+          for (int i = 0; i < spb; ++i) any |= wmask[sb * spb + i];
+          cnt += any != 0u;
+        }
+        int x = cnt;
+#pragma unroll
+        for (int o2 = 1; o2 < 32; o2 <<= 1) {
+          const int y = __shfl_up_sync(0xFFFFFFFFu, x, o2);
+          if (lane >= o2) x += y;
+        }
+        if (lane == 31) sh->scan[warp] = x;
+        __syncthreads();
+        if (tid == 0) {
+          int run = 0;
+          for (int w = 0; w < kThreads / 32; ++w) {
+            const int v = sh->scan[w];
+            sh->scan[w] = run;
+            run += v;
+          }
+          sh->nu = run;
+        }
+        __syncthreads();
+        int pos = sh->scan[warp] + x - cnt;
+        for (int sb = sb0; sb < sb1; ++sb) {
+          uint32_t any = 0;
+          for (int i = 0; i < spb; ++i) any |= wmask[sb * spb + i];
+          if (any) usb[pos++] = (w0 >> (4 - lb)) + sb;
+        }
+      }
+      __syncthreads();
+      const int nu = sh->nu;
+
+      if (warp == 0) {
+        // ---- TMA producer ----
+        if (lane == 0) {
+          for (int u = 0; u < nu && !sh->abort_flag; ++u, ++kc) {
+            const int st = (int)(kc % kNS);
+            if (kc >= kNS && !tc::mbar_wait(&sh->kv_empty[st], (uint32_t)(((kc / kNS) - 1) & 1), &sh->abort_flag)) {
+              if (!sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
+              sh->abort_flag = 1;
+              break;
+            }
+            uint8_t* dst = sKV + st * C::kStage;
+            tc::mbar_arrive_expect_tx(&sh->kv_full[st], pass == 0 ? C::kKsb : C::kStage);
+            const int z = b * a.T_kv + usb[u] * kUnit;
+#pragma unroll
+            for (int h = 0; h < C::kHalves; ++h) {
+              tc::tma_load_3d(dst + h * (kUnit * 128), &map_k, &sh->kv_full[st], h * 64, g, z);
+              if (pass == 1) tc::tma_load_3d(dst + C::kKsb + h * (kUnit * 128), &map_v, &sh->kv_full[st], h * 64, g, z);
+            }
+          }
+        }
+      } else if (warp == 1) {
+        // ---- MMA issuer ----
+        if (lane == 0) {
+          long pend_stage = -1;  // stage of the superblock whose P V is still to issue (pass 2)
+          auto issue_pv = [&](long stage_of) -> bool {
+            const int pb = (int)(pcnt & 1);
+            if (!tc::mbar_wait(&sh->p_full[pb], (uint32_t)((pcnt >> 1) & 1), &sh->abort_flag)) return false;
+            tc::fence_after_sync();
+            const int st = (int)(stage_of % kNS);
+            const uint64_t dp = tc::smem_desc_kmajor_noswz(sP + pb * C::kP, 128, 256);
+            const uint64_t dv = tc::smem_desc_mnmajor_sw128(sKV + st * C::kStage + C::kKsb, kUnit * 128, 1024);
+            tc::mma_bf16_ss(tmem_o, dp, dv, idesc_pv, first_pv ? 0u : 1u);
+            first_pv = false;
+            tc::mma_commit(&sh->kv_empty[st]);
+            tc::mma_commit(&sh->p_empty[pb]);
+            ++pcnt;
+            return true;
+          };
+          bool ok = true;
+          for (int u = 0; u < nu && ok && !sh->abort_flag; ++u, ++kc, ++scnt) {
+            const int st = (int)(kc % kNS);
+            const int sb = (int)(scnt & 1);
+            if (!tc::mbar_wait(&sh->kv_full[st], (uint32_t)((kc / kNS) & 1), &sh->abort_flag) ||
+                (scnt >= 2 && !tc::mbar_wait(&sh->s_empty[sb], (uint32_t)(((scnt >> 1) - 1) & 1), &sh->abort_flag))) {
+              ok = false;
+              break;
+            }
+            tc::fence_after_sync();
+            const uint8_t* kst = sKV + st * C::kStage;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const int h = kk >> 2, off = (kk & 3) * 32;
+              const uint64_t da = tc::smem_desc_kmajor(sQ + h * (kM * 128) + off, 128);
+              const uint64_t db = tc::smem_desc_kmajor(kst + h * (kUnit * 128) + off, 128);
+              tc::mma_bf16_ss(tmem + (uint32_t)(sb * kUnit), da, db, idesc_s, kk > 0 ? 1u : 0u);
+            }
+            tc::mma_commit(&sh->s_full[sb]);
+            if (pass == 0) {
+              tc::mma_commit(&sh->kv_empty[st]);
+            } else {
+              if (pend_stage >= 0 && !issue_pv(pend_stage)) { ok = false; break; }
+              pend_stage = kc;
+            }
+          }
+          if (ok && pass == 1 && pend_stage >= 0 && !sh->abort_flag) ok = issue_pv(pend_stage);
+          if (!ok) {
+            if (!sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
+            sh->abort_flag = 1;
+          }
+        }
+      } else {
+        // ---- softmax (one row per thread) ----
+        for (int u = 0; u < nu; ++u, ++scnt) {
+          const int sb = (int)(scnt & 1);
+          if (!warp_wait(&sh->s_full[sb], (uint32_t)((scnt >> 1) & 1), &sh->abort_flag)) {
+            if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
+            sh->abort_flag = 1;
+            break;
+          }
+          tc::fence_after_sync();
+          uint32_t v[16];
+          tc::tmem_ld16(tmem + lane_base + (uint32_t)(sb * kUnit), v);
+          tc::fence_before_sync();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&sh->s_empty[sb]);
+          const int u0 = usb[u] * kUnit;
+          float s[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int tok = u0 + i;
+            const uint32_t mk = wmask[(tok >> lb) - w0];
+            const bool valid = ((mk >> q_r) & 1u) && tok <= t_r;
+            s[i] = valid ? __uint_as_float(v[i]) : -INFINITY;
+          }
+          if (pass == 0) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) m_r = fmaxf(m_r, s[i]);
+          } else {
+            const float base = m_r == -INFINITY ? 0.f : m_r * sc;
+            uint32_t pk[8];
+            float psum = 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              pk[i] = pack_bf16x2(exp2f(fmaf(s[2 * i], sc, -base)), exp2f(fmaf(s[2 * i + 1], sc, -base)));
+              psum += bf16_lo(pk[i]) + bf16_hi(pk[i]);
+            }
+            l_r += psum;
+            const int pb = (int)(pcnt & 1);
+            if (pcnt >= 2 && !warp_wait(&sh->p_empty[pb], (uint32_t)(((pcnt >> 1) - 1) & 1), &sh->abort_flag)) {
+              if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
+              sh->abort_flag = 1;
+              break;
+            }
+            // P row r: two 16-byte core-matrix rows (tokens 0-7, 8-15) of the no-swizzle K-major layout
+            uint8_t* prow = sP + pb * C::kP + (r >> 3) * 256 + (r & 7) * 16;
+            *reinterpret_cast<uint4*>(prow) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            *reinterpret_cast<uint4*>(prow + 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            tc::fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&sh->p_full[pb]);
+            ++pcnt;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+
+  // ---- epilogue ----
+  // o_done arrives once every MMA this thread issued has completed (at once if none was issued)
+  if (warp == 1 && lane == 0) tc::mma_commit(&sh->o_done);
+  if (is_sm) {
+    bool ok = warp_wait(&sh->o_done, 0, &sh->abort_flag);
+    if (ok) {
+      tc::fence_after_sync();
+      const float inv = l_r > 0.f ? 1.f / l_r : 0.f;
+      const long orow = t_r >= 0 ? ((long)b * a.nQ + (t_r - a.q_t0)) * a.Hq + (long)g * R + h_r : -1;
+#pragma unroll 1
+      for (int h = 0; h < D / 64; ++h) {
+        uint32_t o[64];
+        tc::tmem_ld64(tmem_o + lane_base + (uint32_t)(h * 64), o);
+        if (orow >= 0) {
+#pragma unroll
+          for (int c8 = 0; c8 < 8; ++c8) {
+            const long off = orow * D + h * 64 + c8 * 8;
+            const uint4 gv = __ldg(reinterpret_cast<const uint4*>(a.gate + off));
+            const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+            uint32_t ov[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float o0 = inv > 0.f ? __uint_as_float(o[c8 * 8 + 2 * i]) * inv : 0.f;
+              const float o1 = inv > 0.f ? __uint_as_float(o[c8 * 8 + 2 * i + 1]) * inv : 0.f;
+              const float y0 = o0 * (1.f / (1.f + expf(-bf16_lo(gw[i]))));
+              const float y1 = o1 * (1.f / (1.f + expf(-bf16_hi(gw[i]))));
+              ov[i] = pack_bf16x2(y0, y1);
+            }
+            *reinterpret_cast<uint4*>(a.out + off) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
+          }
+        }
+      }
+    } else if (lane == 0 && !sh->abort_flag) {
+      report(a.status, SGQA_ERR_TIMEOUT);
+      sh->abort_flag = 1;
+    }
+  }
+
+  // ---- drain and release ----
+  if (warp == 0 && lane == 0) {
+    // copies issued for the last stages must land before the CTA exits
+    for (long k2 = kc - kNS; k2 < kc; ++k2) {
+      if (k2 < 0) continue;
+      volatile int no_abort = 0;
+      tc::mbar_wait(&sh->kv_full[k2 % kNS], (uint32_t)((k2 / kNS) & 1), &no_abort);
+    }
+  }
+  if (warp == 1 && lane == 0) {
+    volatile int no_abort = 0;
+    tc::mbar_wait(&sh->o_done, 0, &no_abort);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 256);
+  }
+}
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled get_encode() {
+  static EncodeTiled fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiled>(p);
+  }
+  return fn;
+}
+
+// 3-D map over k or v [batch * T_kv tokens][G][d] bf16: box = 64 dims x 1 group x 16 tokens,
+// 128B swizzle (one 128-byte row per token).
+bool make_kv_map(CUtensorMap* map, const void* base, long tokens, int G, int d) {
+  EncodeTiled enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)G, (cuuint64_t)tokens};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)G * d * 2};
+  const cuuint32_t box[3] = {64, 1, (cuuint32_t)kUnit};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int R>
+cudaError_t launch_dr(const AttendArgs& a, const uint32_t* perm, cudaStream_t s) {
+  using C = AtcCfg<D>;
+  constexpr int QT = kM / R;
+  const int n = a.t_end - a.t_begin;
+  const int tiles = (n + QT - 1) / QT;
+  const int n_seg = a.batch * a.G;
+  int lb = 0;
+  while ((1 << lb) < a.B) ++lb;
+  CUtensorMap mk, mv;
+  if (!make_kv_map(&mk, a.k, (long)a.batch * a.T_kv, a.G, D) || !make_kv_map(&mv, a.v, (long)a.batch * a.T_kv, a.G, D))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  attend_tc_kernel<D, R><<<(unsigned)((long)tiles * n_seg), kThreads, C::kSmem, s>>>(mk, mv, a, perm, n, tiles, lb);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_d(const AttendArgs& a, const uint32_t* perm, cudaStream_t s) {
+  switch (a.Hq / a.G) {
+    case 4: return launch_dr<D, 4>(a, perm, s);
+    case 8: return launch_dr<D, 8>(a, perm, s);
+    case 16: return launch_dr<D, 16>(a, perm, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+bool attend_tc_supported(int Hq, int G, int B, int d) {
+  const int R = Hq / G;
+  return (R == 4 || R == 8 || R == 16) && B <= kUnit && (d == 64 || d == 128);
+}
+
+cudaError_t launch_attend_tc(const AttendArgs& a, const uint32_t* perm, cudaStream_t s) {
+  if (a.t_end <= a.t_begin) return cudaSuccess;
+  if (a.d == 128) return launch_d<128>(a, perm, s);
+  if (a.d == 64) return launch_d<64>(a, perm, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace sgqa

@@ -61,6 +61,10 @@ cudaError_t launch_plan(const int32_t* sel, int sel_T, int sel_t0, int batch, in
 bool attend_tiles_supported(int Hq, int G, int B);
 cudaError_t launch_attend_tiles(const AttendArgs& a, const uint32_t* perm, cudaStream_t s);
 
+// K3 on tcgen05 (R in {4, 8, 16}): same contract as launch_attend_tiles.
+bool attend_tc_supported(int Hq, int G, int B, int d);
+cudaError_t launch_attend_tc(const AttendArgs& a, const uint32_t* perm, cudaStream_t s);
+
 // Decode helpers.
 cudaError_t launch_append(uint16_t* dst, const uint16_t* src, int batch, long row_elems, long dst_seq_stride,
                           long dst_off, long n_elems_per_seq, cudaStream_t s);
