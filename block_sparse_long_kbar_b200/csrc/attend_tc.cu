@@ -37,9 +37,12 @@ namespace sgqa {
 namespace {
 
 constexpr int kUnit = 16;    // tokens per superblock
+constexpr int kCH = 4;       // superblocks per chunk (one handshake between MMA and softmax)
+constexpr int kCT = kCH * kUnit;  // token slots per chunk
 constexpr int kWin = 2048;   // block ids per union window
-constexpr int kNS = 4;       // K/V stages
-constexpr int kThreads = 192;
+constexpr int kNS = 3;       // K/V chunk stages
+constexpr int kSmWarps = 8;  // softmax warps: two per TMEM lane quadrant, each half of every chunk
+constexpr int kThreads = (2 + kSmWarps) * 32;
 constexpr int kM = 128;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -47,19 +50,22 @@ template <int D>
 struct AtcCfg {
   static constexpr int kHalves = D / 64;
   static constexpr int kQ = kM * D * 2;                 // [half][128 rows][128 B]
-  static constexpr int kKsb = kHalves * kUnit * 128;    // one superblock of K (or V): [half][16][128 B]
-  static constexpr int kStage = 2 * kKsb;               // K then V
-  static constexpr int kP = kM * kUnit * 2;             // P tile 128 x 16 bf16
-  static constexpr int kSmem = 1024 + kQ + kNS * kStage + 2 * kP + 2 * kWin * 4 + 1024;
+  static constexpr int kHalfRows = kCT * 128;           // one 64-dim half of a chunk: [64 tokens][128 B]
+  static constexpr int kKc = kHalves * kHalfRows;       // K (or V) of one chunk: [half][64][128 B]
+  static constexpr int kStage = 2 * kKc;                // K then V
+  static constexpr int kPsb = kM * kUnit * 2;           // P of one superblock: 128 x 16 bf16
+  static constexpr int kP = kCH * kPsb;                 // P of one chunk
+  static constexpr int kSmem = 1024 + kQ + kNS * kStage + 2 * kP + 2 * kWin * 4 + 2048 + 2048;
 };
 
 struct AtcShared {
   uint64_t kv_full[kNS], kv_empty[kNS], s_full[2], s_empty[2], p_full[2], p_empty[2], o_done;
+  long long l_part[2][kM];   // per-row fixed-point partial sums of the two softmax halves
+  float m_part[2][kM];       // per-row partial maxima of the two softmax halves
   uint32_t tmem;
   volatile int abort_flag;
   int t[32];
-  int cur[32];
-  int scan[8];
+  int scan[kThreads / 32];
   int nu, maxc;
 };
 
@@ -70,7 +76,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 template <int D, int R>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
                      AttendArgs a, const uint32_t* __restrict__ perm, int n_per_seg, int tiles_per_seg, int lb) {
   using C = AtcCfg<D>;
@@ -78,8 +84,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = smem;
-  uint8_t* sKV = sQ + C::kQ;                             // [stage][K|V][half][16][128 B]
-  uint8_t* sP = sKV + kNS * C::kStage;                   // [2][16 groups][2 chunks][8 rows][16 B]
+  uint8_t* sKV = sQ + C::kQ;                             // [stage][K|V][half][64 tokens][128 B]
+  uint8_t* sP = sKV + kNS * C::kStage;                   // [2][superblock][16 groups][2][8 rows][16 B]
   uint32_t* wmask = reinterpret_cast<uint32_t*>(sP + 2 * C::kP);
   int32_t* usb = reinterpret_cast<int32_t*>(wmask + kWin);
   AtcShared* sh = reinterpret_cast<AtcShared*>(usb + kWin);
@@ -96,8 +102,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&sh->s_full[i], 1);
-      tc::mbar_init(&sh->s_empty[i], 4);
-      tc::mbar_init(&sh->p_full[i], 4);
+      tc::mbar_init(&sh->s_empty[i], kSmWarps);
+      tc::mbar_init(&sh->p_full[i], kSmWarps);
       tc::mbar_init(&sh->p_empty[i], 1);
     }
     tc::mbar_init(&sh->o_done, 1);
@@ -113,6 +119,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (t >= 0) atomicMax(&sh->maxc, t / B);
   }
   if (warp == 1) tc::tmem_alloc(&sh->tmem, 256);
+  (void)sh->scan;
 
   // Q tile: row r = query r / R, head r % R; 16-byte chunk c of half h at
   // h * 16 KB + r * 128 + ((c ^ (r & 7)) * 16) (the 128B-swizzled K-major layout).
@@ -132,29 +139,30 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = sh->tmem;
-  const uint32_t tmem_o = tmem + 128;  // O: columns 128 .. 128 + D - 1; S buffers: columns 0 .. 31
+  const uint32_t tmem_o = tmem + 128;  // O: columns 128 .. 128 + D - 1; S buffers: columns 0 .. 127
 
-  // softmax role state (warps 2-5): TMEM lane quadrant warp % 4
+  // softmax role state (warps 2..9): TMEM lane quadrant warp % 4, half (warp - 2) / 4 of every chunk
   const bool is_sm = warp >= 2;
   const int quad = warp & 3;
+  const int shalf = is_sm ? (warp - 2) / 4 : 0;
   const int r = quad * 32 + lane;
   const int q_r = r / R, h_r = r % R;
   const int t_r = is_sm ? sh->t[q_r] : -1;
-  float m_r = -INFINITY, l_r = 0.f;
+  float m_r = -INFINITY;
+  long long l_fx = 0;  // row sum of P in fixed point (2^-40 units): exact, order-independent
   const float sc = kLog2e / sqrtf((float)D);
   const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
 
   const int nwin = sh->maxc < 0 ? 0 : sh->maxc / kWin + 1;
   const int spb = kUnit >> lb;  // blocks per superblock
-  long kc = 0;                  // superblocks streamed (producer & MMA ring position)
+  long kc = 0;                  // chunks streamed (producer & MMA ring position)
   long scnt = 0;                // S buffer uses (MMA & softmax)
   long pcnt = 0;                // P buffer uses (MMA & softmax, pass 2)
   bool first_pv = true;
-  const uint32_t idesc_s = tc::idesc_bf16_f32(kM, kUnit);
+  const uint32_t idesc_s = tc::idesc_bf16_f32(kM, kCT);
   const uint32_t idesc_pv = tc::idesc_bf16_f32(kM, D, true);
 
   for (int pass = 0; pass < 2; ++pass) {
-    if (tid < QT) sh->cur[tid] = 0;
     for (int win = 0; win < nwin; ++win) {
       const int w0 = win * kWin, w1 = w0 + kWin;
       // ---- union of this window (all warps) ----
@@ -165,29 +173,33 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (t < 0) continue;
         const int cq = t / B;
         const int32_t* row = a.sel + (((long)b * a.sel_T + (t - a.sel_t0)) * G + g) * (long)a.Kb;
-        int cur = sh->cur[q];
-        while (cur < a.Kb) {
-          const int e = cur + lane;
-          int j = e < a.Kb ? __ldg(row + e) : -1;
-          const int prev = __shfl_up_sync(0xFFFFFFFFu, j, 1);
-          const int before = lane > 0 ? prev : (cur > 0 ? __ldg(row + cur - 1) : -1);
-          if (j > cq || j < -1 || (j >= 0 && j <= before) || (j >= 0 && j < w0)) {
-            if (pass == 0) report(a.status, SGQA_ERR_DEVICE_CHECK);
-            j = -1;
+        int before_batch = -1;  // last entry of the previous batch (rows are strictly ascending)
+        for (int base = 0; base < a.Kb; base += 512) {
+          int jv[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int e = base + i * 32 + lane;
+            jv[i] = e < a.Kb ? __ldg(row + e) : -1;
           }
-          const bool in = j >= w0 && j < w1;
-          const bool past = j < 0 || j >= w1;
-          if (in) atomicOr(&wmask[j - w0], 1u << q);
-          const unsigned stop = __ballot_sync(0xFFFFFFFFu, past);
-          const int adv = stop ? __ffs(stop) - 1 : 32;
-          cur += adv;
-          if (stop) {
-            const int first = __shfl_sync(0xFFFFFFFFu, j, adv);
-            if (first < 0) cur = a.Kb;
-            break;
+          bool stop = false;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            int j = jv[i];
+            // every lane takes part in both shuffles (they are warp-collective)
+            const int prev = __shfl_up_sync(0xFFFFFFFFu, j, 1);
+            const int last_prev = __shfl_sync(0xFFFFFFFFu, i > 0 ? jv[i > 0 ? i - 1 : 0] : before_batch, 31);
+            const int before = lane > 0 ? prev : last_prev;
+            if (j > cq || j < -1 || (j >= 0 && j <= before)) {
+              if (pass == 0 && win == 0) report(a.status, SGQA_ERR_DEVICE_CHECK);
+              j = -1;
+            }
+            if (j >= w0 && j < w1) atomicOr(&wmask[j - w0], 1u << q);
+            jv[i] = j;
+            stop |= __any_sync(0xFFFFFFFFu, j < 0 || j >= w1);
           }
+          before_batch = __shfl_sync(0xFFFFFFFFu, jv[15], 31);
+          if (stop) break;  // end of row, or past this window
         }
-        if (lane == 0) sh->cur[q] = cur;
       }
       __syncthreads();
       {
@@ -227,11 +239,13 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       __syncthreads();
       const int nu = sh->nu;
+      const int nch = (nu + kCH - 1) / kCH;
 
       if (warp == 0) {
-        // ---- TMA producer ----
+        // ---- TMA producer: one chunk = kCH superblocks; missing ones (partial last chunk) are
+        // loaded from out of bounds, which fills zeros ----
         if (lane == 0) {
-          for (int u = 0; u < nu && !sh->abort_flag; ++u, ++kc) {
+          for (int ch = 0; ch < nch && !sh->abort_flag; ++ch, ++kc) {
             const int st = (int)(kc % kNS);
             if (kc >= kNS && !tc::mbar_wait(&sh->kv_empty[st], (uint32_t)(((kc / kNS) - 1) & 1), &sh->abort_flag)) {
               if (!sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
@@ -239,35 +253,45 @@ __global__ void __launch_bounds__(kThreads, 2)
               break;
             }
             uint8_t* dst = sKV + st * C::kStage;
-            tc::mbar_arrive_expect_tx(&sh->kv_full[st], pass == 0 ? C::kKsb : C::kStage);
-            const int z = b * a.T_kv + usb[u] * kUnit;
+            tc::mbar_arrive_expect_tx(&sh->kv_full[st], pass == 0 ? C::kKc : C::kStage);
 #pragma unroll
-            for (int h = 0; h < C::kHalves; ++h) {
-              tc::tma_load_3d(dst + h * (kUnit * 128), &map_k, &sh->kv_full[st], h * 64, g, z);
-              if (pass == 1) tc::tma_load_3d(dst + C::kKsb + h * (kUnit * 128), &map_v, &sh->kv_full[st], h * 64, g, z);
+            for (int i = 0; i < kCH; ++i) {
+              const int e = ch * kCH + i;
+              const int z = e < nu ? b * a.T_kv + usb[e] * kUnit : 0x7FFFFFF0;
+#pragma unroll
+              for (int h = 0; h < C::kHalves; ++h) {
+                tc::tma_load_3d(dst + h * C::kHalfRows + i * (kUnit * 128), &map_k, &sh->kv_full[st], h * 64, g, z);
+                if (pass == 1)
+                  tc::tma_load_3d(dst + C::kKc + h * C::kHalfRows + i * (kUnit * 128), &map_v, &sh->kv_full[st], h * 64,
+                                  g, z);
+              }
             }
           }
         }
       } else if (warp == 1) {
         // ---- MMA issuer ----
         if (lane == 0) {
-          long pend_stage = -1;  // stage of the superblock whose P V is still to issue (pass 2)
+          long pend_stage = -1;  // ring position of the chunk whose P V is still to issue (pass 2)
           auto issue_pv = [&](long stage_of) -> bool {
             const int pb = (int)(pcnt & 1);
             if (!tc::mbar_wait(&sh->p_full[pb], (uint32_t)((pcnt >> 1) & 1), &sh->abort_flag)) return false;
             tc::fence_after_sync();
             const int st = (int)(stage_of % kNS);
-            const uint64_t dp = tc::smem_desc_kmajor_noswz(sP + pb * C::kP, 128, 256);
-            const uint64_t dv = tc::smem_desc_mnmajor_sw128(sKV + st * C::kStage + C::kKsb, kUnit * 128, 1024);
-            tc::mma_bf16_ss(tmem_o, dp, dv, idesc_pv, first_pv ? 0u : 1u);
-            first_pv = false;
+            const uint8_t* vbase = sKV + st * C::kStage + C::kKc;
+#pragma unroll
+            for (int i = 0; i < kCH; ++i) {
+              const uint64_t dp = tc::smem_desc_kmajor_noswz(sP + pb * C::kP + i * C::kPsb, 128, 256);
+              const uint64_t dv = tc::smem_desc_mnmajor_sw128(vbase + i * (kUnit * 128), C::kHalfRows, 1024);
+              tc::mma_bf16_ss(tmem_o, dp, dv, idesc_pv, first_pv ? 0u : 1u);
+              first_pv = false;
+            }
             tc::mma_commit(&sh->kv_empty[st]);
             tc::mma_commit(&sh->p_empty[pb]);
             ++pcnt;
             return true;
           };
           bool ok = true;
-          for (int u = 0; u < nu && ok && !sh->abort_flag; ++u, ++kc, ++scnt) {
+          for (int ch = 0; ch < nch && ok && !sh->abort_flag; ++ch, ++kc, ++scnt) {
             const int st = (int)(kc % kNS);
             const int sb = (int)(scnt & 1);
             if (!tc::mbar_wait(&sh->kv_full[st], (uint32_t)((kc / kNS) & 1), &sh->abort_flag) ||
@@ -281,8 +305,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int kk = 0; kk < D / 16; ++kk) {
               const int h = kk >> 2, off = (kk & 3) * 32;
               const uint64_t da = tc::smem_desc_kmajor(sQ + h * (kM * 128) + off, 128);
-              const uint64_t db = tc::smem_desc_kmajor(kst + h * (kUnit * 128) + off, 128);
-              tc::mma_bf16_ss(tmem + (uint32_t)(sb * kUnit), da, db, idesc_s, kk > 0 ? 1u : 0u);
+              const uint64_t db = tc::smem_desc_kmajor(kst + h * C::kHalfRows + off, 128);
+              tc::mma_bf16_ss(tmem + (uint32_t)(sb * kCT), da, db, idesc_s, kk > 0 ? 1u : 0u);
             }
             tc::mma_commit(&sh->s_full[sb]);
             if (pass == 0) {
@@ -299,8 +323,10 @@ __global__ void __launch_bounds__(kThreads, 2)
           }
         }
       } else {
-        // ---- softmax (one row per thread) ----
-        for (int u = 0; u < nu; ++u, ++scnt) {
+        // ---- softmax: one row per thread; this half handles superblocks 2*shalf, 2*shalf+1 of
+        // every chunk ----
+        constexpr int kHalfCols = kCT / 2;
+        for (int ch = 0; ch < nch; ++ch, ++scnt) {
           const int sb = (int)(scnt & 1);
           if (!warp_wait(&sh->s_full[sb], (uint32_t)((scnt >> 1) & 1), &sh->abort_flag)) {
             if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
@@ -308,43 +334,56 @@ __global__ void __launch_bounds__(kThreads, 2)
             break;
           }
           tc::fence_after_sync();
-          uint32_t v[16];
-          tc::tmem_ld16(tmem + lane_base + (uint32_t)(sb * kUnit), v);
+          uint32_t v[kHalfCols];
+          tc::tmem_ld32(tmem + lane_base + (uint32_t)(sb * kCT + shalf * kHalfCols), v);
           tc::fence_before_sync();
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(&sh->s_empty[sb]);
-          const int u0 = usb[u] * kUnit;
-          float s[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int tok = u0 + i;
-            const uint32_t mk = wmask[(tok >> lb) - w0];
-            const bool valid = ((mk >> q_r) & 1u) && tok <= t_r;
-            s[i] = valid ? __uint_as_float(v[i]) : -INFINITY;
+          for (int i2 = 0; i2 < kCH / 2; ++i2) {
+            const int e = ch * kCH + shalf * (kCH / 2) + i2;
+            const int u0 = e < nu ? usb[e] * kUnit : 0;
+            uint32_t vmask = 0;  // bit k: token u0 + k is valid for this row
+            if (e < nu && t_r >= 0) {
+              for (int blk = 0; blk < spb; ++blk) {
+                const int j = (u0 >> lb) + blk;
+                if ((wmask[j - w0] >> q_r) & 1u) vmask |= ((1u << (1 << lb)) - 1u) << (blk << lb);
+              }
+              const int lim = t_r - u0;
+              if (lim < 15) vmask &= lim < 0 ? 0u : ((2u << lim) - 1u);
+            }
+#pragma unroll
+            for (int k2 = 0; k2 < kUnit; ++k2)
+              if (!((vmask >> k2) & 1u)) v[i2 * kUnit + k2] = __float_as_uint(-INFINITY);
           }
           if (pass == 0) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) m_r = fmaxf(m_r, s[i]);
+            for (int i = 0; i < kHalfCols; ++i) m_r = fmaxf(m_r, __uint_as_float(v[i]));
           } else {
             const float base = m_r == -INFINITY ? 0.f : m_r * sc;
-            uint32_t pk[8];
-            float psum = 0.f;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              pk[i] = pack_bf16x2(exp2f(fmaf(s[2 * i], sc, -base)), exp2f(fmaf(s[2 * i + 1], sc, -base)));
-              psum += bf16_lo(pk[i]) + bf16_hi(pk[i]);
-            }
-            l_r += psum;
             const int pb = (int)(pcnt & 1);
             if (pcnt >= 2 && !warp_wait(&sh->p_empty[pb], (uint32_t)(((pcnt >> 1) - 1) & 1), &sh->abort_flag)) {
               if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
               sh->abort_flag = 1;
               break;
             }
-            // P row r: two 16-byte core-matrix rows (tokens 0-7, 8-15) of the no-swizzle K-major layout
-            uint8_t* prow = sP + pb * C::kP + (r >> 3) * 256 + (r & 7) * 16;
-            *reinterpret_cast<uint4*>(prow) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            *reinterpret_cast<uint4*>(prow + 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+#pragma unroll
+            for (int i2 = 0; i2 < kCH / 2; ++i2) {
+              uint32_t pk[8];
+              float psum = 0.f;
+#pragma unroll
+              for (int k2 = 0; k2 < 8; ++k2) {
+                pk[k2] = pack_bf16x2(exp2f(fmaf(__uint_as_float(v[i2 * kUnit + 2 * k2]), sc, -base)),
+                                     exp2f(fmaf(__uint_as_float(v[i2 * kUnit + 2 * k2 + 1]), sc, -base)));
+                psum += bf16_lo(pk[k2]) + bf16_hi(pk[k2]);
+              }
+              // each superblock's sum (fixed order) enters the row sum exactly, in 2^-40 units
+              l_fx += __float2ll_rz(psum * 1099511627776.0f);
+              const int i = shalf * (kCH / 2) + i2;
+              uint8_t* prow = sP + pb * C::kP + i * C::kPsb + (r >> 3) * 256 + (r & 7) * 16;
+              *reinterpret_cast<uint4*>(prow) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              *reinterpret_cast<uint4*>(prow + 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
             tc::fence_proxy_async();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&sh->p_full[pb]);
@@ -354,7 +393,15 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       __syncthreads();
     }
+    if (pass == 0) {
+      if (is_sm) sh->m_part[shalf][r] = m_r;
+      __syncthreads();
+      if (is_sm) m_r = fmaxf(sh->m_part[0][r], sh->m_part[1][r]);
+    }
   }
+  if (is_sm) sh->l_part[shalf][r] = l_fx;
+  __syncthreads();
+  const float l_r = is_sm ? (float)((double)(sh->l_part[0][r] + sh->l_part[1][r]) * 0x1.0p-40) : 0.f;
 
   // ---- epilogue ----
   // o_done arrives once every MMA this thread issued has completed (at once if none was issued)
@@ -366,13 +413,13 @@ __global__ void __launch_bounds__(kThreads, 2)
       const float inv = l_r > 0.f ? 1.f / l_r : 0.f;
       const long orow = t_r >= 0 ? ((long)b * a.nQ + (t_r - a.q_t0)) * a.Hq + (long)g * R + h_r : -1;
 #pragma unroll 1
-      for (int h = 0; h < D / 64; ++h) {
-        uint32_t o[64];
-        tc::tmem_ld64(tmem_o + lane_base + (uint32_t)(h * 64), o);
+      for (int h = shalf; h < D / 32; h += 2) {
+        uint32_t o[32];
+        tc::tmem_ld32(tmem_o + lane_base + (uint32_t)(h * 32), o);
         if (orow >= 0) {
 #pragma unroll
-          for (int c8 = 0; c8 < 8; ++c8) {
-            const long off = orow * D + h * 64 + c8 * 8;
+          for (int c8 = 0; c8 < 4; ++c8) {
+            const long off = orow * D + h * 32 + c8 * 8;
             const uint4 gv = __ldg(reinterpret_cast<const uint4*>(a.gate + off));
             const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
             uint32_t ov[4];

@@ -81,6 +81,7 @@ __device__ __forceinline__ int epi_vote_any(SelShared* sh, int slot, bool v) {
     res = 1;
     while (*cnt < kEpiWarps) {
       if (sh->abort_flag || tc::globaltimer() - t0 > tc::kWaitLimitNs) { res = -1; break; }
+      __nanosleep(32);
     }
     if (res > 0) {
       __threadfence_block();
