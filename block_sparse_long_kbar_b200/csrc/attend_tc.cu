@@ -40,11 +40,14 @@ constexpr int kUnit = 16;    // tokens per superblock
 constexpr int kCH = 4;       // superblocks per chunk (one handshake between MMA and softmax)
 constexpr int kCT = kCH * kUnit;  // token slots per chunk
 constexpr int kWin = 2048;   // block ids per union window
+constexpr int kWinWords = 16;     // occupancy bits for up to 512 windows
 constexpr int kNS = 3;       // K/V chunk stages
-constexpr int kSmWarps = 8;  // softmax warps: two per TMEM lane quadrant, each half of every chunk
+constexpr int kSmWarps = 8;  // softmax warps: two per TMEM lane quadrant
 constexpr int kThreads = (2 + kSmWarps) * 32;
 constexpr int kM = 128;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRiskLog2 = 60.f;  // a row whose scores exceed its reference by more than this (log2)
+                                   // is recomputed with its exact maximum
 
 template <int D>
 struct AtcCfg {
@@ -55,24 +58,62 @@ struct AtcCfg {
   static constexpr int kStage = 2 * kKc;                // K then V
   static constexpr int kPsb = kM * kUnit * 2;           // P of one superblock: 128 x 16 bf16
   static constexpr int kP = kCH * kPsb;                 // P of one chunk
-  static constexpr int kSmem = 1024 + kQ + kNS * kStage + 2 * kP + 2 * kWin * 4 + 2048 + 2048;
+  static constexpr int kSmem = 1024 + kQ + kNS * kStage + 2 * kP + 2 * kWin * 4 + 4096;
 };
 
 struct AtcShared {
   uint64_t kv_full[kNS], kv_empty[kNS], s_full[2], s_empty[2], p_full[2], p_empty[2], o_done;
-  long long l_part[2][kM];   // per-row fixed-point partial sums of the two softmax halves
-  float m_part[2][kM];       // per-row partial maxima of the two softmax halves
+  float ref_part[2][kM];  // per-row reference maxima from the own block (two halves of its tokens)
+  float max_part[2][kM];  // per-row exact maxima by superblock parity (fallback pass)
+  float l_part[2][kM];    // per-row sums of P by superblock parity
+  uint32_t wbits[kWinWords];
   uint32_t tmem;
   volatile int abort_flag;
   int t[32];
   int scan[kThreads / 32];
-  int nu, maxc;
+  int nu, maxc, all_windows;
 };
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   int ok = 1;
   if ((threadIdx.x & 31) == 0) ok = tc::mbar_wait(bar, parity, abort) ? 1 : 0;
   return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
+}
+
+// Visit every valid entry of a query's selection row (strictly ascending block ids <= cq, then -1
+// padding), 512 entries per batch with all loads in flight; fn(j) per valid entry. Entries that
+// break the format are skipped (and reported when `report_errors`). Must be called by a whole warp.
+template <class Fn>
+__device__ __forceinline__ void for_each_selected(const int32_t* row, int Kb, int cq, int stop_at, bool report_errors,
+                                                  int* status, Fn fn) {
+  const int lane = threadIdx.x & 31;
+  int before_batch = -1;
+  for (int base = 0; base < Kb; base += 512) {
+    int jv[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int e = base + i * 32 + lane;
+      jv[i] = e < Kb ? __ldg(row + e) : -1;
+    }
+    bool stop = false;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      int j = jv[i];
+      // both shuffles are warp-collective: every lane executes them
+      const int prev = __shfl_up_sync(0xFFFFFFFFu, j, 1);
+      const int last_prev = __shfl_sync(0xFFFFFFFFu, i > 0 ? jv[i > 0 ? i - 1 : 0] : before_batch, 31);
+      const int before = lane > 0 ? prev : last_prev;
+      if (j > cq || j < -1 || (j >= 0 && j <= before)) {
+        if (report_errors) report(status, SGQA_ERR_DEVICE_CHECK);
+        j = -1;
+      }
+      if (j >= 0 && j < stop_at) fn(j);
+      jv[i] = j;
+      stop |= __any_sync(0xFFFFFFFFu, j < 0 || j >= stop_at);
+    }
+    before_batch = __shfl_sync(0xFFFFFFFFu, jv[15], 31);
+    if (stop) break;
+  }
 }
 
 template <int D, int R>
@@ -109,8 +150,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::mbar_init(&sh->o_done, 1);
     sh->abort_flag = 0;
     sh->maxc = -1;
+    sh->all_windows = 0;
     tc::fence_mbar_init();
   }
+  if (tid < kWinWords) sh->wbits[tid] = 0;
+  for (int i = tid; i < kWin; i += kThreads) wmask[i] = 0;
   __syncthreads();
   if (tid < QT) {
     const int idx = tile * QT + tid;
@@ -119,7 +163,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (t >= 0) atomicMax(&sh->maxc, t / B);
   }
   if (warp == 1) tc::tmem_alloc(&sh->tmem, 256);
-  (void)sh->scan;
 
   // Q tile: row r = query r / R, head r % R; 16-byte chunk c of half h at
   // h * 16 KB + r * 128 + ((c ^ (r & 7)) * 16) (the 128B-swizzled K-major layout).
@@ -133,6 +176,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                tq >= 0 ? 16 : 0);
   }
   cp_async_commit();
+  // which windows hold any selected block (each row read once; format errors reported here)
+  const int nwin = sh->maxc < 0 ? 0 : sh->maxc / kWin + 1;
+  if (nwin > 32 * kWinWords) {
+    if (tid == 0) sh->all_windows = 1;
+  } else {
+    for (int q = warp; q < QT; q += kThreads / 32) {
+      const int t = sh->t[q];
+      if (t < 0) continue;
+      const int32_t* row = a.sel + (((long)b * a.sel_T + (t - a.sel_t0)) * G + g) * (long)a.Kb;
+      for_each_selected(row, a.Kb, t / B, 0x7FFFFFFF, true, a.status, [&](int j) {
+        const int w = j / kWin;
+        atomicOr(&sh->wbits[w >> 5], 1u << (w & 31));
+      });
+    }
+  }
   cp_async_wait<0>();
   tc::fence_proxy_async();
   tc::fence_before_sync();
@@ -141,65 +199,80 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sh->tmem;
   const uint32_t tmem_o = tmem + 128;  // O: columns 128 .. 128 + D - 1; S buffers: columns 0 .. 127
 
-  // softmax role state (warps 2..9): TMEM lane quadrant warp % 4, half (warp - 2) / 4 of every chunk
+  // softmax role state (warps 2..9): TMEM lane quadrant warp % 4; `shalf` also picks the
+  // superblocks (by block-id parity) and the own-block tokens this thread handles
   const bool is_sm = warp >= 2;
   const int quad = warp & 3;
   const int shalf = is_sm ? (warp - 2) / 4 : 0;
   const int r = quad * 32 + lane;
   const int q_r = r / R, h_r = r % R;
   const int t_r = is_sm ? sh->t[q_r] : -1;
-  float m_r = -INFINITY;
-  long long l_fx = 0;  // row sum of P in fixed point (2^-40 units): exact, order-independent
   const float sc = kLog2e / sqrtf((float)D);
   const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
 
-  const int nwin = sh->maxc < 0 ? 0 : sh->maxc / kWin + 1;
+  // reference maximum of the row: its scores against its own block (always selected, u <= t),
+  // computed on the CUDA cores from the same bf16 operands; a function of the row alone
+  if (is_sm) {
+    float mx = -INFINITY;
+    if (t_r >= 0) {
+      const int u_lo = (t_r / B) * B;
+      const uint8_t* qrow = sQ + r * 128;
+      for (int u = u_lo + shalf; u <= t_r; u += 2) {
+        const uint16_t* krow = a.k + (((long)b * a.T_kv + u) * G + g) * D;
+        float acc = 0.f;
+#pragma unroll
+        for (int cc = 0; cc < D / 8; ++cc) {
+          const int h = cc >> 3, c = cc & 7;
+          const uint4 qv = *reinterpret_cast<const uint4*>(qrow + h * (kM * 128) + ((c ^ (r & 7)) * 16));
+          const uint4 kv = __ldg(reinterpret_cast<const uint4*>(krow + cc * 8));
+          const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w}, kw[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            acc = fmaf(bf16_lo(qw[i]), bf16_lo(kw[i]), acc);
+            acc = fmaf(bf16_hi(qw[i]), bf16_hi(kw[i]), acc);
+          }
+        }
+        mx = fmaxf(mx, acc);
+      }
+    }
+    sh->ref_part[shalf][r] = mx;
+  }
+  __syncthreads();
+  const float m_ref = is_sm ? fmaxf(sh->ref_part[0][r], sh->ref_part[1][r]) : -INFINITY;
+  float m_use = m_ref, m_exact = -INFINITY;
+  bool risky = false;  // this row's scores exceed m_use by more than kRiskLog2
+  float l_half = 0.f;
+
   const int spb = kUnit >> lb;  // blocks per superblock
   long kc = 0;                  // chunks streamed (producer & MMA ring position)
   long scnt = 0;                // S buffer uses (MMA & softmax)
-  long pcnt = 0;                // P buffer uses (MMA & softmax, pass 2)
-  bool first_pv = true;
+  long pcnt = 0;                // P buffer uses (MMA & softmax)
   const uint32_t idesc_s = tc::idesc_bf16_f32(kM, kCT);
   const uint32_t idesc_pv = tc::idesc_bf16_f32(kM, D, true);
+  bool rerun = false;
 
-  for (int pass = 0; pass < 2; ++pass) {
+  // pass 0: main (P V with the reference maximum); passes 1-2 only if some row was risky:
+  // exact maxima, then the main pass again (risky rows use their exact maximum, all other rows
+  // repeat exactly the same arithmetic as in pass 0).
+  for (int pass = 0; pass < 3; ++pass) {
+    if (pass == 1 && !rerun) break;
+    const bool main_pass = pass != 1;
+    bool first_pv = true;
+    if (main_pass) {
+      l_half = 0.f;
+      if (pass == 2) m_use = risky ? m_exact : m_ref;
+    }
     for (int win = 0; win < nwin; ++win) {
+      if (!sh->all_windows && !((sh->wbits[win >> 5] >> (win & 31)) & 1u)) continue;  // uniform
       const int w0 = win * kWin, w1 = w0 + kWin;
       // ---- union of this window (all warps) ----
-      for (int i = tid; i < kWin; i += kThreads) wmask[i] = 0;
-      __syncthreads();
       for (int q = warp; q < QT; q += kThreads / 32) {
         const int t = sh->t[q];
         if (t < 0) continue;
-        const int cq = t / B;
         const int32_t* row = a.sel + (((long)b * a.sel_T + (t - a.sel_t0)) * G + g) * (long)a.Kb;
-        int before_batch = -1;  // last entry of the previous batch (rows are strictly ascending)
-        for (int base = 0; base < a.Kb; base += 512) {
-          int jv[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int e = base + i * 32 + lane;
-            jv[i] = e < a.Kb ? __ldg(row + e) : -1;
-          }
-          bool stop = false;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            int j = jv[i];
-            // every lane takes part in both shuffles (they are warp-collective)
-            const int prev = __shfl_up_sync(0xFFFFFFFFu, j, 1);
-            const int last_prev = __shfl_sync(0xFFFFFFFFu, i > 0 ? jv[i > 0 ? i - 1 : 0] : before_batch, 31);
-            const int before = lane > 0 ? prev : last_prev;
-            if (j > cq || j < -1 || (j >= 0 && j <= before)) {
-              if (pass == 0 && win == 0) report(a.status, SGQA_ERR_DEVICE_CHECK);
-              j = -1;
-            }
-            if (j >= w0 && j < w1) atomicOr(&wmask[j - w0], 1u << q);
-            jv[i] = j;
-            stop |= __any_sync(0xFFFFFFFFu, j < 0 || j >= w1);
-          }
-          before_batch = __shfl_sync(0xFFFFFFFFu, jv[15], 31);
-          if (stop) break;  // end of row, or past this window
-        }
+        for_each_selected(row, a.Kb, t / B, w1, false, a.status, [&](int j) {
+          if (j >= w0) atomicOr(&wmask[j - w0], 1u << q);
+        });
       }
       __syncthreads();
       {
@@ -253,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             uint8_t* dst = sKV + st * C::kStage;
-            tc::mbar_arrive_expect_tx(&sh->kv_full[st], pass == 0 ? C::kKc : C::kStage);
+            tc::mbar_arrive_expect_tx(&sh->kv_full[st], main_pass ? C::kStage : C::kKc);
 #pragma unroll
             for (int i = 0; i < kCH; ++i) {
               const int e = ch * kCH + i;
@@ -261,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int h = 0; h < C::kHalves; ++h) {
                 tc::tma_load_3d(dst + h * C::kHalfRows + i * (kUnit * 128), &map_k, &sh->kv_full[st], h * 64, g, z);
-                if (pass == 1)
+                if (main_pass)
                   tc::tma_load_3d(dst + C::kKc + h * C::kHalfRows + i * (kUnit * 128), &map_v, &sh->kv_full[st], h * 64,
                                   g, z);
               }
@@ -271,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else if (warp == 1) {
         // ---- MMA issuer ----
         if (lane == 0) {
-          long pend_stage = -1;  // ring position of the chunk whose P V is still to issue (pass 2)
+          long pend_stage = -1;  // ring position of the chunk whose P V is still to issue
           auto issue_pv = [&](long stage_of) -> bool {
             const int pb = (int)(pcnt & 1);
             if (!tc::mbar_wait(&sh->p_full[pb], (uint32_t)((pcnt >> 1) & 1), &sh->abort_flag)) return false;
@@ -309,23 +382,22 @@ __global__ void __launch_bounds__(kThreads, 1)
               tc::mma_bf16_ss(tmem + (uint32_t)(sb * kCT), da, db, idesc_s, kk > 0 ? 1u : 0u);
             }
             tc::mma_commit(&sh->s_full[sb]);
-            if (pass == 0) {
+            if (!main_pass) {
               tc::mma_commit(&sh->kv_empty[st]);
             } else {
               if (pend_stage >= 0 && !issue_pv(pend_stage)) { ok = false; break; }
               pend_stage = kc;
             }
           }
-          if (ok && pass == 1 && pend_stage >= 0 && !sh->abort_flag) ok = issue_pv(pend_stage);
+          if (ok && main_pass && pend_stage >= 0 && !sh->abort_flag) ok = issue_pv(pend_stage);
           if (!ok) {
             if (!sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
             sh->abort_flag = 1;
           }
         }
       } else {
-        // ---- softmax: one row per thread; this half handles superblocks 2*shalf, 2*shalf+1 of
-        // every chunk ----
-        constexpr int kHalfCols = kCT / 2;
+        // ---- softmax: one row per thread pair; each handles the superblocks whose id parity
+        // is `shalf` (a fixed, tile-independent split of the row's work) ----
         for (int ch = 0; ch < nch; ++ch, ++scnt) {
           const int sb = (int)(scnt & 1);
           if (!warp_wait(&sh->s_full[sb], (uint32_t)((scnt >> 1) & 1), &sh->abort_flag)) {
@@ -334,17 +406,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc::fence_after_sync();
-          uint32_t v[kHalfCols];
-          tc::tmem_ld32(tmem + lane_base + (uint32_t)(sb * kCT + shalf * kHalfCols), v);
+          uint32_t v[kCT];
+          tc::tmem_ld64(tmem + lane_base + (uint32_t)(sb * kCT), v);
           tc::fence_before_sync();
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(&sh->s_empty[sb]);
+          const int pb = (int)(pcnt & 1);
+          if (main_pass && pcnt >= 2 &&
+              !warp_wait(&sh->p_empty[pb], (uint32_t)(((pcnt >> 1) - 1) & 1), &sh->abort_flag)) {
+            if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
+            sh->abort_flag = 1;
+            break;
+          }
+          const float base = m_use * sc;
 #pragma unroll
-          for (int i2 = 0; i2 < kCH / 2; ++i2) {
-            const int e = ch * kCH + shalf * (kCH / 2) + i2;
-            const int u0 = e < nu ? usb[e] * kUnit : 0;
-            uint32_t vmask = 0;  // bit k: token u0 + k is valid for this row
-            if (e < nu && t_r >= 0) {
+          for (int i = 0; i < kCH; ++i) {
+            const int e = ch * kCH + i;
+            const int sbid = e < nu ? usb[e] : -1;
+            const bool mine = sbid >= 0 ? ((sbid & 1) == shalf) : (shalf == 0);
+            if (!mine) continue;
+            uint32_t vmask = 0;  // bit k: token sbid * 16 + k is valid for this row
+            if (sbid >= 0 && t_r >= 0) {
+              const int u0 = sbid * kUnit;
               for (int blk = 0; blk < spb; ++blk) {
                 const int j = (u0 >> lb) + blk;
                 if ((wmask[j - w0] >> q_r) & 1u) vmask |= ((1u << (1 << lb)) - 1u) << (blk << lb);
@@ -352,38 +435,29 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int lim = t_r - u0;
               if (lim < 15) vmask &= lim < 0 ? 0u : ((2u << lim) - 1u);
             }
+            if (!main_pass) {
 #pragma unroll
-            for (int k2 = 0; k2 < kUnit; ++k2)
-              if (!((vmask >> k2) & 1u)) v[i2 * kUnit + k2] = __float_as_uint(-INFINITY);
+              for (int k2 = 0; k2 < kUnit; ++k2)
+                if ((vmask >> k2) & 1u) m_exact = fmaxf(m_exact, __uint_as_float(v[i * kUnit + k2]));
+              continue;
+            }
+            uint32_t pk[8];
+            float psum = 0.f, smax = -INFINITY;
+#pragma unroll
+            for (int k2 = 0; k2 < 8; ++k2) {
+              const bool va = (vmask >> (2 * k2)) & 1u, vb = (vmask >> (2 * k2 + 1)) & 1u;
+              const float sa = __uint_as_float(v[i * kUnit + 2 * k2]), sbv = __uint_as_float(v[i * kUnit + 2 * k2 + 1]);
+              smax = fmaxf(smax, fmaxf(va ? sa : -INFINITY, vb ? sbv : -INFINITY));
+              pk[k2] = pack_bf16x2(va ? exp2f(fmaf(sa, sc, -base)) : 0.f, vb ? exp2f(fmaf(sbv, sc, -base)) : 0.f);
+              psum += bf16_lo(pk[k2]) + bf16_hi(pk[k2]);
+            }
+            if (smax * sc - base > kRiskLog2) risky = true;
+            l_half += psum;  // this half's superblocks in ascending order: a canonical order
+            uint8_t* prow = sP + pb * C::kP + i * C::kPsb + (r >> 3) * 256 + (r & 7) * 16;
+            *reinterpret_cast<uint4*>(prow) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            *reinterpret_cast<uint4*>(prow + 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
           }
-          if (pass == 0) {
-#pragma unroll
-            for (int i = 0; i < kHalfCols; ++i) m_r = fmaxf(m_r, __uint_as_float(v[i]));
-          } else {
-            const float base = m_r == -INFINITY ? 0.f : m_r * sc;
-            const int pb = (int)(pcnt & 1);
-            if (pcnt >= 2 && !warp_wait(&sh->p_empty[pb], (uint32_t)(((pcnt >> 1) - 1) & 1), &sh->abort_flag)) {
-              if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
-              sh->abort_flag = 1;
-              break;
-            }
-#pragma unroll
-            for (int i2 = 0; i2 < kCH / 2; ++i2) {
-              uint32_t pk[8];
-              float psum = 0.f;
-#pragma unroll
-              for (int k2 = 0; k2 < 8; ++k2) {
-                pk[k2] = pack_bf16x2(exp2f(fmaf(__uint_as_float(v[i2 * kUnit + 2 * k2]), sc, -base)),
-                                     exp2f(fmaf(__uint_as_float(v[i2 * kUnit + 2 * k2 + 1]), sc, -base)));
-                psum += bf16_lo(pk[k2]) + bf16_hi(pk[k2]);
-              }
-              // each superblock's sum (fixed order) enters the row sum exactly, in 2^-40 units
-              l_fx += __float2ll_rz(psum * 1099511627776.0f);
-              const int i = shalf * (kCH / 2) + i2;
-              uint8_t* prow = sP + pb * C::kP + i * C::kPsb + (r >> 3) * 256 + (r & 7) * 16;
-              *reinterpret_cast<uint4*>(prow) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-              *reinterpret_cast<uint4*>(prow + 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-            }
+          if (main_pass) {
             tc::fence_proxy_async();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&sh->p_full[pb]);
@@ -392,16 +466,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       __syncthreads();
+      // clear this window's bitmap words through its union list
+      for (int e = tid; e < nu; e += kThreads)
+        for (int i = 0; i < spb; ++i) wmask[(usb[e] * spb + i) - w0] = 0u;
+      __syncthreads();
     }
     if (pass == 0) {
-      if (is_sm) sh->m_part[shalf][r] = m_r;
+      rerun = __syncthreads_or(is_sm && risky) != 0;
+    } else if (pass == 1) {
+      if (is_sm) sh->max_part[shalf][r] = m_exact;
       __syncthreads();
-      if (is_sm) m_r = fmaxf(sh->m_part[0][r], sh->m_part[1][r]);
+      if (is_sm) m_exact = fmaxf(sh->max_part[0][r], sh->max_part[1][r]);
     }
   }
-  if (is_sm) sh->l_part[shalf][r] = l_fx;
+  if (is_sm) sh->l_part[shalf][r] = l_half;
   __syncthreads();
-  const float l_r = is_sm ? (float)((double)(sh->l_part[0][r] + sh->l_part[1][r]) * 0x1.0p-40) : 0.f;
+  const float l_r = is_sm ? sh->l_part[0][r] + sh->l_part[1][r] : 0.f;
 
   // ---- epilogue ----
   // o_done arrives once every MMA this thread issued has completed (at once if none was issued)
