@@ -147,14 +147,20 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """The step time every rank reports is the slowest rank's (weak scaling: one sequence per rank)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_tokens(cfg, world: int) -> int:
+    """Tokens one timed step processes across the job: every rank runs its own sequence(s)."""
+    return world * cfg.batch * cfg.T
 
 
 # ---- the CPU oracle on a bounded sample (cpu_baseline and the reference arm) ------------------
@@ -238,7 +244,7 @@ def run_ours(args, world, rank):
     status = sg.sgqa_get_device_status(ws)
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
-    tokens_step = world * cfg.batch * cfg.T
+    tokens_step = job_tokens(cfg, world)
     value = tokens_step / (ms / 1e3)
 
     # per-stage times: the same kernels through the per-stage entry points, events on the launch stream

@@ -193,8 +193,8 @@ __global__ void __launch_bounds__(kWarps * 32) attend_kernel(AttendArgs a) {
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int nt = 2 * kk + h;
-        const uint32_t lo = pack_bf16x2(exp2f(fmaf(sacc[nt][0], sc, -base0)), exp2f(fmaf(sacc[nt][1], sc, -base0)));
-        const uint32_t hi = pack_bf16x2(exp2f(fmaf(sacc[nt][2], sc, -base1)), exp2f(fmaf(sacc[nt][3], sc, -base1)));
+        const uint32_t lo = pack_bf16x2(ex2_approx(fmaf(sacc[nt][0], sc, -base0)), ex2_approx(fmaf(sacc[nt][1], sc, -base0)));
+        const uint32_t hi = pack_bf16x2(ex2_approx(fmaf(sacc[nt][2], sc, -base1)), ex2_approx(fmaf(sacc[nt][3], sc, -base1)));
         pa[kk][2 * h] = lo;       // row gid
         pa[kk][2 * h + 1] = hi;   // row gid + 8
         ps0 += bf16_lo(lo) + bf16_hi(lo);

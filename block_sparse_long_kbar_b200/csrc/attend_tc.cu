@@ -448,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const bool va = (vmask >> (2 * k2)) & 1u, vb = (vmask >> (2 * k2 + 1)) & 1u;
               const float sa = __uint_as_float(v[i * kUnit + 2 * k2]), sbv = __uint_as_float(v[i * kUnit + 2 * k2 + 1]);
               smax = fmaxf(smax, fmaxf(va ? sa : -INFINITY, vb ? sbv : -INFINITY));
-              pk[k2] = pack_bf16x2(va ? exp2f(fmaf(sa, sc, -base)) : 0.f, vb ? exp2f(fmaf(sbv, sc, -base)) : 0.f);
+              pk[k2] = pack_bf16x2(va ? ex2_approx(fmaf(sa, sc, -base)) : 0.f, vb ? ex2_approx(fmaf(sbv, sc, -base)) : 0.f);
               psum += bf16_lo(pk[k2]) + bf16_hi(pk[k2]);
             }
             if (smax * sc - base > kRiskLog2) risky = true;

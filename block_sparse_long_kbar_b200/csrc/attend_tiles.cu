@@ -300,8 +300,8 @@ __global__ void __launch_bounds__(TileCfg<D, R>::NT, 1)
         uint32_t pa[4];
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
-          pa[2 * nt] = pack_bf16x2(exp2f(fmaf(sacc[nt][0], sc, -base0)), exp2f(fmaf(sacc[nt][1], sc, -base0)));
-          pa[2 * nt + 1] = pack_bf16x2(exp2f(fmaf(sacc[nt][2], sc, -base1)), exp2f(fmaf(sacc[nt][3], sc, -base1)));
+          pa[2 * nt] = pack_bf16x2(ex2_approx(fmaf(sacc[nt][0], sc, -base0)), ex2_approx(fmaf(sacc[nt][1], sc, -base0)));
+          pa[2 * nt + 1] = pack_bf16x2(ex2_approx(fmaf(sacc[nt][2], sc, -base1)), ex2_approx(fmaf(sacc[nt][3], sc, -base1)));
         }
         l0 += (bf16_lo(pa[0]) + bf16_hi(pa[0])) + (bf16_lo(pa[2]) + bf16_hi(pa[2]));
         l1 += (bf16_lo(pa[1]) + bf16_hi(pa[1])) + (bf16_lo(pa[3]) + bf16_hi(pa[3]));

@@ -29,6 +29,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// 2^x with the hardware's approximate base-2 exponential (relative error ~2^-22, subnormal
+// results flushed to zero); used for attention probabilities, which are rounded to bf16 next.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Order-preserving map of an fp32 score to uint32 (larger score -> larger key). -0 is first
 // folded into +0 so that equal scores give equal keys.
 __device__ __forceinline__ uint32_t score_key(float s) {
