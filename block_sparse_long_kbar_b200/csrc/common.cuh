@@ -49,6 +49,13 @@ __device__ __forceinline__ uint32_t score_key(float s) {
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
+// Round a dynamic shared-memory base up to A bytes by pointer arithmetic on the shared array
+// itself, so pointers derived from it stay in the shared state space (ld/st/atom.shared rather
+// than generic accesses).
+template <int A>
+__device__ __forceinline__ uint8_t* smem_align(uint8_t* base) {
+  return base + ((A - (smem_u32(base) & (A - 1))) & (A - 1));
+}
 // 16-byte global->shared copy; src_bytes = 0 zero-fills the destination without reading.
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes));

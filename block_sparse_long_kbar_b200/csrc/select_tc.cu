@@ -44,6 +44,7 @@ constexpr int kEpiWarps = 8;     // two per TMEM lane quadrant: each histograms 
 constexpr int kThreads = (kEpiWarps + 2) * 32;
 constexpr int kProducerWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
 constexpr int kMaxPasses = 5;
+constexpr int kCap = 128;        // bucket keys a row may collect for an early exact finish (8 B each)
 
 template <int DI>
 struct SelCfg {
@@ -61,8 +62,8 @@ struct SelShared {
   volatile int signals;
   volatile int abort_flag;
   int more[kMaxPasses + 1];
-  int vote_cnt[3 * kMaxPasses];
-  int vote_any[3 * kMaxPasses];
+  int vote_cnt[4 * kMaxPasses];
+  int vote_any[4 * kMaxPasses];
 };
 
 // Bounded barrier + "any" vote among the epilogue warps (slot = a fresh index per use): every
@@ -111,13 +112,69 @@ __device__ __forceinline__ int pass_exists(SelShared* sh, int p) {
   return sh->more[p - 1];
 }
 
+// ---- branch-free per-key epilogue steps (64 consecutive candidates of one row per call) ----
+// Shared-memory histogram increment / pair store, predicated in PTX so that the per-key loop
+// has no branches.
+__device__ __forceinline__ void red_shared_inc(uint32_t addr) {
+  asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(addr) : "memory");
+}
+__device__ __forceinline__ void red_shared_inc_if_eq(uint32_t addr, uint32_t a, uint32_t b) {
+  asm volatile("{ .reg .pred p; setp.eq.u32 p, %1, %2; @p red.shared.add.u32 [%0], 1; }" ::"r"(addr), "r"(a),
+               "r"(b)
+               : "memory");
+}
+// (addr is only 4-byte aligned: row histograms are 257 words apart)
+__device__ __forceinline__ void st_shared_pair_if(uint32_t addr, uint32_t x, uint32_t y, uint32_t pred) {
+  asm volatile("{ .reg .pred p; setp.ne.u32 p, %3, 0; @p st.shared.u32 [%0], %1; @p st.shared.u32 [%0+4], %2; }" ::"r"(
+                   addr),
+               "r"(x), "r"(y), "r"(pred)
+               : "memory");
+}
+
+// Histogram pass: count, in the row's 256 bins, the next 8 key bits (at `shift`) of the keys
+// whose resolved bits (mask) equal prefix. kFull: all 64 candidates exist (else only q < lim).
+template <bool kFull, bool kFirst>
+__device__ __forceinline__ void hist_chunk(const uint32_t (&v)[64], int lim, uint32_t mask, uint32_t prefix, int shift,
+                                           uint32_t hbase) {
+#pragma unroll
+  for (int q = 0; q < 64; ++q) {
+    const uint32_t key = score_key(__uint_as_float(v[q]));
+    const uint32_t addr = hbase + (((key >> shift) & 255u) << 2);
+    if (kFull) {
+      if (kFirst) red_shared_inc(addr);
+      else red_shared_inc_if_eq(addr, key & mask, prefix);
+    } else {
+      red_shared_inc_if_eq(addr, (q < lim && (kFirst || (key & mask) == prefix)) ? 1u : 0u, 1u);
+    }
+  }
+}
+
+// Emit pass: mark (bits of tb) the candidates taken: keys >= thr, plus, among the keys of the
+// bucket [blo, blo + bw], the first tie_lim in j order; the first col_lim bucket keys are also
+// stored as (key, j) pairs at cbase. eqn counts the bucket keys seen so far in this row.
+template <bool kFull>
+__device__ __forceinline__ void emit_chunk(const uint32_t (&v)[64], int lim, uint32_t thr, uint32_t blo, uint32_t bw,
+                                           int tie_lim, int col_lim, uint32_t cbase, int j0, int& eqn,
+                                           uint32_t (&tb)[2]) {
+#pragma unroll
+  for (int q = 0; q < 64; ++q) {
+    const uint32_t key = score_key(__uint_as_float(v[q]));
+    const bool in = kFull || q < lim;
+    const bool inb = in && key - blo <= bw;
+    const bool take = in && (key >= thr || (inb && eqn < tie_lim));
+    st_shared_pair_if(cbase + 8u * (uint32_t)eqn, key, (uint32_t)(j0 + q), (inb && eqn < col_lim) ? 1u : 0u);
+    eqn += inb ? 1 : 0;
+    tb[q >> 5] |= take ? (1u << (q & 31)) : 0u;
+  }
+}
+
 template <int DI>
 __global__ void __launch_bounds__(kThreads, 1)
     select_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_hi,
                      const __grid_constant__ CUtensorMap map_lo, SelectArgs a) {
   using C = SelCfg<DI>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* smem = smem_align<1024>(smem_raw);
   uint8_t* sA = smem;
   uint8_t* sB = sA + C::kA;                                               // [stage][hi|lo][kN][DI]
   uint32_t* hist = reinterpret_cast<uint32_t*>(sB + kStages * C::kStage);
@@ -146,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::mbar_init(&sh->a_full, 1);
     sh->signals = 0;
     sh->abort_flag = 0;
-    for (int p = 0; p < 3 * kMaxPasses; ++p) sh->vote_cnt[p] = sh->vote_any[p] = 0;
+    for (int p = 0; p < 4 * kMaxPasses; ++p) sh->vote_cnt[p] = sh->vote_any[p] = 0;
     tc::fence_mbar_init();
   }
   if (warp == kMmaWarp) tc::tmem_alloc(&sh->tmem, 256);
@@ -262,25 +319,46 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* my_hist = hist + r * kHistStride;
     int32_t* out = a.sel + (((long)b * a.sel_T + (t - a.sel_t0)) * G + g) * (long)a.Kb;
     const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
+    const uint32_t hbase = smem_u32(my_hist);
     long k = 0;
-    int pos = 0, eq_taken = 0;
+    int pos = 0;
     bool aborted = false;
     for (int pass = 0; pass < kMaxPasses; ++pass) {
       // zero the histograms for this pass, then a barrier+vote: is any row still unresolved?
       if (half == 0 && !done && pass < kMaxPasses - 1)
         for (int i = 0; i < 256; ++i) my_hist[i] = 0;
-      const int vote = epi_vote_any(sh, 3 * pass, !done);
-      if (vote < 0) {
+      const int vote = epi_vote_any(sh, 4 * pass, !done);
+      // from the third pass on, if every unresolved row's threshold bucket is small, this pass is
+      // the last: it also collects those buckets' keys, which are then resolved exactly
+      const int vote_big = (pass >= 2 && vote > 0) ? epi_vote_any(sh, 4 * pass + 3, !done && nb > kCap) : 1;
+      if (vote < 0 || vote_big < 0) {
         if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
         sh->abort_flag = 1;
         break;
       }
-      const bool is_emit = vote == 0 || pass == kMaxPasses - 1;
+      const bool is_emit = vote == 0 || vote_big == 0 || pass == kMaxPasses - 1;
       if (warp == 0 && lane == 0) {
         sh->more[pass] = is_emit ? 0 : 1;
         __threadfence_block();
         sh->signals = pass + 1;
       }
+      // emit rule of this row: take keys >= thr; bucket [blo, blo + bw] handled by ties or collection
+      uint32_t thr = 0xFFFFFFFFu, blo = 0xFFFFFFFFu, bw = 0u;
+      int tie_lim = 0, col_lim = 0;
+      if (!done) {  // collecting: everything above the bucket, the bucket's keys kept aside
+        const uint32_t pend = prefix | ~mask;
+        thr = pend == 0xFFFFFFFFu ? 0xFFFFFFFFu : pend + 1u;
+        blo = prefix;
+        bw = ~mask;
+        col_lim = kCap;
+      } else if (rem == nb) {  // the whole bucket is taken
+        thr = prefix;
+      } else {  // fully resolved key with ties: the first rem of them in j order
+        thr = prefix == 0xFFFFFFFFu ? 0xFFFFFFFFu : prefix + 1u;
+        blo = prefix;
+        tie_lim = rem;
+      }
+      int eqn = 0;
       const int shift = 24 - 8 * pass;
       for (int i = 0; i < n_nt; ++i, ++k) {
         const int buf = (int)(k & 1);
@@ -296,23 +374,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::tmem_ld64(tmem + lane_base + (uint32_t)(buf * kN + half * 64), v);
           const int j0 = i * kN + half * 64;
           const int lim = c - j0;
-          if (!done && lim > 0) {
-            if (pass == 0) {  // every key matches the empty prefix
-              if (lim >= 64) {
-#pragma unroll
-                for (int q = 0; q < 64; ++q) atomicAdd(&my_hist[score_key(__uint_as_float(v[q])) >> 24], 1u);
-              } else {
-#pragma unroll
-                for (int q = 0; q < 64; ++q)
-                  if (q < lim) atomicAdd(&my_hist[score_key(__uint_as_float(v[q])) >> 24], 1u);
-              }
-            } else {
-#pragma unroll
-              for (int q = 0; q < 64; ++q) {
-                const uint32_t key = score_key(__uint_as_float(v[q]));
-                if (q < lim && (key & mask) == prefix) atomicAdd(&my_hist[(key >> shift) & 255u], 1u);
-              }
-            }
+          // a resolved row matches nothing (its histogram is not read; in the first pass it may
+          // count, harmlessly)
+          const uint32_t mk = done ? 0u : mask, pf = done ? 1u : prefix;
+          if (__all_sync(0xFFFFFFFFu, lim >= 64)) {
+            if (pass == 0) hist_chunk<true, true>(v, lim, mk, pf, shift, hbase);
+            else hist_chunk<true, false>(v, lim, mk, pf, shift, hbase);
+          } else if (lim > 0) {
+            if (pass == 0) hist_chunk<false, true>(v, lim, mk, pf, shift, hbase);
+            else hist_chunk<false, false>(v, lim, mk, pf, shift, hbase);
           }
         } else if (half == 0) {
 #pragma unroll 1
@@ -320,15 +390,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t v[64];
             tc::tmem_ld64(tmem + lane_base + (uint32_t)(buf * kN + hh * 64), v);
             const int j0 = i * kN + hh * 64;
-            const int lim = c - j0;
-            if (valid && lim > 0) {
+            const int lim = valid ? c - j0 : 0;
+            uint32_t tb[2] = {0u, 0u};
+            if (__all_sync(0xFFFFFFFFu, lim >= 64))
+              emit_chunk<true>(v, lim, thr, blo, bw, tie_lim, col_lim, hbase, j0, eqn, tb);
+            else if (lim > 0)
+              emit_chunk<false>(v, lim, thr, blo, bw, tie_lim, col_lim, hbase, j0, eqn, tb);
 #pragma unroll
-              for (int q = 0; q < 64; ++q) {
-                const uint32_t key = score_key(__uint_as_float(v[q])) & mask;
-                const bool eq = key == prefix;
-                const bool take = q < lim && (key > prefix || (eq && eq_taken < rem));
-                eq_taken += (q < lim && eq) ? 1 : 0;
-                if (take && pos < m) out[pos++] = j0 + q;
+            for (int w = 0; w < 2; ++w) {
+              uint32_t bits = tb[w];
+              while (bits) {
+                const int q = __ffs(bits) - 1;
+                bits &= bits - 1u;
+                if (pos < m) out[pos++] = j0 + 32 * w + q;
               }
             }
           }
@@ -339,6 +413,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (aborted) break;
       if (is_emit) {
+        if (half == 0 && valid && !done) {
+          // the collected bucket (ascending j): candidate i ranks behind every larger key and every
+          // equal key of lower j, and is chosen when fewer than rem rank ahead of it
+          const uint32_t* cand = my_hist;
+          uint32_t* cj = my_hist;
+          int nch = 0;
+          if (eqn > kCap) report(a.status, SGQA_ERR_DEVICE_CHECK);
+          const int ncand = min(eqn, kCap);
+          for (int ci = 0; ci < ncand; ++ci) {
+            const uint32_t key = cand[2 * ci];
+            int ahead = 0;
+            for (int c2 = 0; c2 < ncand; ++c2) {
+              const uint32_t k2 = cand[2 * c2];
+              ahead += (k2 > key || (k2 == key && c2 < ci)) ? 1 : 0;
+            }
+            if (ahead < rem) cj[2 * nch++ + 1] = cand[2 * ci + 1];  // keys stay; only j slots move down
+          }
+          if (pos + nch > m) {
+            report(a.status, SGQA_ERR_DEVICE_CHECK);
+            nch = m - pos;
+          }
+          // merge the chosen (ascending j) into the row written so far, from the back
+          int rd = pos - 1, wr = pos + nch - 1;
+          for (int kk = nch - 1; kk >= 0 && wr >= 0; --wr) {
+            const int jc = (int)cj[2 * kk + 1];
+            if (rd >= 0 && out[rd] > jc) out[wr] = out[rd--];
+            else { out[wr] = jc; --kk; }
+          }
+          pos += nch;
+        }
         if (half == 0 && valid) {
           if (pos != m) report(a.status, SGQA_ERR_DEVICE_CHECK);
           out[pos++] = c;
@@ -347,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       // both halves' histogram updates are complete before either reads the histogram
-      if (epi_vote_any(sh, 3 * pass + 1, false) < 0) {
+      if (epi_vote_any(sh, 4 * pass + 1, false) < 0) {
         if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
         sh->abort_flag = 1;
         break;
@@ -368,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         done = (rem == nb) || (mask == 0xFFFFFFFFu);
       }
       // both halves have read the histogram before the next pass zeroes it
-      if (epi_vote_any(sh, 3 * pass + 2, false) < 0) {
+      if (epi_vote_any(sh, 4 * pass + 2, false) < 0) {
         if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
         sh->abort_flag = 1;
         break;
