@@ -44,7 +44,8 @@ constexpr int kEpiWarps = 8;     // two per TMEM lane quadrant: each histograms 
 constexpr int kThreads = (kEpiWarps + 2) * 32;
 constexpr int kProducerWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
 constexpr int kMaxPasses = 5;
-constexpr int kCap = 128;        // bucket keys a row may collect for an early exact finish (8 B each)
+constexpr int kCap = 42;         // bucket keys a row may collect for an early exact finish (3 words each)
+constexpr int kRing = 129;       // the row's output staging ring (128 words) starts at this word
 
 template <int DI>
 struct SelCfg {
@@ -113,22 +114,13 @@ __device__ __forceinline__ int pass_exists(SelShared* sh, int p) {
 }
 
 // ---- branch-free per-key epilogue steps (64 consecutive candidates of one row per call) ----
-// Shared-memory histogram increment / pair store, predicated in PTX so that the per-key loop
-// has no branches.
+// Shared-memory histogram updates for the branch-free per-key loops.
 __device__ __forceinline__ void red_shared_inc(uint32_t addr) {
   asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(addr) : "memory");
 }
-__device__ __forceinline__ void red_shared_inc_if_eq(uint32_t addr, uint32_t a, uint32_t b) {
-  asm volatile("{ .reg .pred p; setp.eq.u32 p, %1, %2; @p red.shared.add.u32 [%0], 1; }" ::"r"(addr), "r"(a),
-               "r"(b)
-               : "memory");
-}
-// (addr is only 4-byte aligned: row histograms are 257 words apart)
-__device__ __forceinline__ void st_shared_pair_if(uint32_t addr, uint32_t x, uint32_t y, uint32_t pred) {
-  asm volatile("{ .reg .pred p; setp.ne.u32 p, %3, 0; @p st.shared.u32 [%0], %1; @p st.shared.u32 [%0+4], %2; }" ::"r"(
-                   addr),
-               "r"(x), "r"(y), "r"(pred)
-               : "memory");
+// Adds 0 or 1: every lane stays active, which measured faster than a predicated reduction.
+__device__ __forceinline__ void red_shared_add(uint32_t addr, uint32_t val) {
+  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(addr), "r"(val) : "memory");
 }
 
 // Histogram pass: count, in the row's 256 bins, the next 8 key bits (at `shift`) of the keys
@@ -140,31 +132,151 @@ __device__ __forceinline__ void hist_chunk(const uint32_t (&v)[64], int lim, uin
   for (int q = 0; q < 64; ++q) {
     const uint32_t key = score_key(__uint_as_float(v[q]));
     const uint32_t addr = hbase + (((key >> shift) & 255u) << 2);
-    if (kFull) {
-      if (kFirst) red_shared_inc(addr);
-      else red_shared_inc_if_eq(addr, key & mask, prefix);
-    } else {
-      red_shared_inc_if_eq(addr, (q < lim && (kFirst || (key & mask) == prefix)) ? 1u : 0u, 1u);
-    }
+    if (kFull && kFirst) red_shared_inc(addr);
+    else red_shared_add(addr, ((kFull || q < lim) && (kFirst || (key & mask) == prefix)) ? 1u : 0u);
+  }
+}
+
+// v[q] for a run-time q, keeping the array in registers (used only for the rare bucket keys)
+__device__ __forceinline__ uint32_t pick64(const uint32_t (&v)[64], int q) {
+  switch (q) {
+    case 0: return v[0];
+    case 1: return v[1];
+    case 2: return v[2];
+    case 3: return v[3];
+    case 4: return v[4];
+    case 5: return v[5];
+    case 6: return v[6];
+    case 7: return v[7];
+    case 8: return v[8];
+    case 9: return v[9];
+    case 10: return v[10];
+    case 11: return v[11];
+    case 12: return v[12];
+    case 13: return v[13];
+    case 14: return v[14];
+    case 15: return v[15];
+    case 16: return v[16];
+    case 17: return v[17];
+    case 18: return v[18];
+    case 19: return v[19];
+    case 20: return v[20];
+    case 21: return v[21];
+    case 22: return v[22];
+    case 23: return v[23];
+    case 24: return v[24];
+    case 25: return v[25];
+    case 26: return v[26];
+    case 27: return v[27];
+    case 28: return v[28];
+    case 29: return v[29];
+    case 30: return v[30];
+    case 31: return v[31];
+    case 32: return v[32];
+    case 33: return v[33];
+    case 34: return v[34];
+    case 35: return v[35];
+    case 36: return v[36];
+    case 37: return v[37];
+    case 38: return v[38];
+    case 39: return v[39];
+    case 40: return v[40];
+    case 41: return v[41];
+    case 42: return v[42];
+    case 43: return v[43];
+    case 44: return v[44];
+    case 45: return v[45];
+    case 46: return v[46];
+    case 47: return v[47];
+    case 48: return v[48];
+    case 49: return v[49];
+    case 50: return v[50];
+    case 51: return v[51];
+    case 52: return v[52];
+    case 53: return v[53];
+    case 54: return v[54];
+    case 55: return v[55];
+    case 56: return v[56];
+    case 57: return v[57];
+    case 58: return v[58];
+    case 59: return v[59];
+    case 60: return v[60];
+    case 61: return v[61];
+    case 62: return v[62];
+    case 63: return v[63];
+    default: return 0u;
   }
 }
 
 // Emit pass: mark (bits of tb) the candidates taken: keys >= thr, plus, among the keys of the
 // bucket [blo, blo + bw], the first tie_lim in j order; the first col_lim bucket keys are also
-// stored as (key, j) pairs at cbase. eqn counts the bucket keys seen so far in this row.
+// stored in cand as (key, j, number of taken keys of lower j) triples. eqn counts the bucket keys
+// seen so far in this row; pos0 is the number of keys taken before this chunk. The per-key work
+// is ALU only; the few bucket keys are handled afterwards, one set bit at a time.
 template <bool kFull>
 __device__ __forceinline__ void emit_chunk(const uint32_t (&v)[64], int lim, uint32_t thr, uint32_t blo, uint32_t bw,
-                                           int tie_lim, int col_lim, uint32_t cbase, int j0, int& eqn,
+                                           int tie_lim, int col_lim, uint32_t* cand, int j0, int pos0, int& eqn,
                                            uint32_t (&tb)[2]) {
+  uint32_t bb[2] = {0u, 0u};
 #pragma unroll
   for (int q = 0; q < 64; ++q) {
     const uint32_t key = score_key(__uint_as_float(v[q]));
     const bool in = kFull || q < lim;
-    const bool inb = in && key - blo <= bw;
-    const bool take = in && (key >= thr || (inb && eqn < tie_lim));
-    st_shared_pair_if(cbase + 8u * (uint32_t)eqn, key, (uint32_t)(j0 + q), (inb && eqn < col_lim) ? 1u : 0u);
-    eqn += inb ? 1 : 0;
-    tb[q >> 5] |= take ? (1u << (q & 31)) : 0u;
+    tb[q >> 5] |= (in && key >= thr) ? (1u << (q & 31)) : 0u;
+    bb[q >> 5] |= (in && key - blo <= bw) ? (1u << (q & 31)) : 0u;
+  }
+#pragma unroll
+  for (int w = 0; w < 2; ++w) {
+    uint32_t bits = bb[w];
+    while (bits) {
+      const int q = __ffs(bits) - 1;
+      bits &= bits - 1u;
+      if (eqn < tie_lim) tb[w] |= 1u << q;
+      if (eqn < col_lim) {  // collecting (no ties are taken then, so tb holds only keys above)
+        const int before = pos0 + (w ? __popc(tb[0]) : 0) + __popc(tb[w] & ((1u << q) - 1u));
+        cand[3 * eqn] = score_key(__uint_as_float(pick64(v, 32 * w + q)));
+        cand[3 * eqn + 1] = (uint32_t)(j0 + 32 * w + q);
+        cand[3 * eqn + 2] = (uint32_t)before;
+      }
+      ++eqn;
+    }
+  }
+}
+
+// Writes, cooperatively across the warp, the staged block indices of every row whose staging
+// ring holds at least `least` unwritten entries (all of them when least is 1, else 64): each
+// selected row goes out as whole 128-byte lines instead of one scattered 4-byte store per index.
+// Rows are 32 * quad + lane; `out` and the ring state (pos, flushed) belong to the lane's row.
+__device__ __forceinline__ void flush_rows(const uint32_t* hist, int quad, int lane, int32_t* out, int pos,
+                                           int& flushed, int least) {
+  unsigned need = __ballot_sync(0xFFFFFFFFu, pos - flushed >= least);
+  while (need) {
+    const int L = __ffs(need) - 1;
+    need &= need - 1u;
+    const int fl = __shfl_sync(0xFFFFFFFFu, flushed, L);
+    const int cnt = min(64, __shfl_sync(0xFFFFFFFFu, pos, L) - fl);
+    int32_t* rout = reinterpret_cast<int32_t*>(__shfl_sync(0xFFFFFFFFu, reinterpret_cast<long long>(out), L));
+    const uint32_t* ring = hist + (32 * quad + L) * kHistStride + kRing + (fl & 127);
+    if (lane < cnt) rout[fl + lane] = (int32_t)ring[lane];
+    if (lane + 32 < cnt) rout[fl + 32 + lane] = (int32_t)ring[lane + 32];
+    if (lane == L) flushed = fl + cnt;
+  }
+}
+
+// Moves out[lo, hi) up by sh slots (sh >= 1), top down, eight independent loads at a time.
+__device__ __forceinline__ void shift_up(int32_t* out, int lo, int hi, int sh) {
+  int p = hi;
+  while (p - lo >= 8) {
+    int x[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) x[u] = out[p - 1 - u];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) out[p - 1 - u + sh] = x[u];
+    p -= 8;
+  }
+  while (p > lo) {
+    --p;
+    out[p + sh] = out[p];
   }
 }
 
@@ -321,7 +433,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
     const uint32_t hbase = smem_u32(my_hist);
     long k = 0;
-    int pos = 0;
+    uint32_t* ring = my_hist + kRing;  // emit pass: taken indices staged here, 128 in flight at most
+    int pos = 0, flushed = 0;
     bool aborted = false;
     for (int pass = 0; pass < kMaxPasses; ++pass) {
       // zero the histograms for this pass, then a barrier+vote: is any row still unresolved?
@@ -393,18 +506,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int lim = valid ? c - j0 : 0;
             uint32_t tb[2] = {0u, 0u};
             if (__all_sync(0xFFFFFFFFu, lim >= 64))
-              emit_chunk<true>(v, lim, thr, blo, bw, tie_lim, col_lim, hbase, j0, eqn, tb);
+              emit_chunk<true>(v, lim, thr, blo, bw, tie_lim, col_lim, my_hist, j0, pos, eqn, tb);
             else if (lim > 0)
-              emit_chunk<false>(v, lim, thr, blo, bw, tie_lim, col_lim, hbase, j0, eqn, tb);
+              emit_chunk<false>(v, lim, thr, blo, bw, tie_lim, col_lim, my_hist, j0, pos, eqn, tb);
+            // stage the taken indices in order (warp-uniform trip count: no divergent loop), then
+            // write out the rows that have 64 staged
 #pragma unroll
             for (int w = 0; w < 2; ++w) {
               uint32_t bits = tb[w];
-              while (bits) {
+              const int n_it = (int)__reduce_max_sync(0xFFFFFFFFu, (unsigned)__popc(bits));
+              for (int it = 0; it < n_it; ++it) {
                 const int q = __ffs(bits) - 1;
                 bits &= bits - 1u;
-                if (pos < m) out[pos++] = j0 + 32 * w + q;
+                if (q >= 0 && pos < m) ring[pos++ & 127] = (uint32_t)(j0 + 32 * w + q);
               }
             }
+            flush_rows(hist, quad, lane, out, pos, flushed, 64);
           }
         }
         tc::fence_before_sync();
@@ -413,33 +530,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (aborted) break;
       if (is_emit) {
+        if (half == 0) {
+          flush_rows(hist, quad, lane, out, pos, flushed, 1);
+          __syncwarp();  // the row's lines written by other lanes are visible to its owner below
+        }
         if (half == 0 && valid && !done) {
           // the collected bucket (ascending j): candidate i ranks behind every larger key and every
           // equal key of lower j, and is chosen when fewer than rem rank ahead of it
-          const uint32_t* cand = my_hist;
-          uint32_t* cj = my_hist;
+          uint32_t* cand = my_hist;
           int nch = 0;
           if (eqn > kCap) report(a.status, SGQA_ERR_DEVICE_CHECK);
           const int ncand = min(eqn, kCap);
           for (int ci = 0; ci < ncand; ++ci) {
-            const uint32_t key = cand[2 * ci];
+            const uint32_t key = cand[3 * ci];
             int ahead = 0;
             for (int c2 = 0; c2 < ncand; ++c2) {
-              const uint32_t k2 = cand[2 * c2];
+              const uint32_t k2 = cand[3 * c2];
               ahead += (k2 > key || (k2 == key && c2 < ci)) ? 1 : 0;
             }
-            if (ahead < rem) cj[2 * nch++ + 1] = cand[2 * ci + 1];  // keys stay; only j slots move down
+            if (ahead < rem) {  // keys stay in place; the chosen (j, before) pairs move to the front
+              cand[3 * nch + 1] = cand[3 * ci + 1];
+              cand[3 * nch + 2] = cand[3 * ci + 2];
+              ++nch;
+            }
           }
           if (pos + nch > m) {
             report(a.status, SGQA_ERR_DEVICE_CHECK);
             nch = m - pos;
           }
-          // merge the chosen (ascending j) into the row written so far, from the back
-          int rd = pos - 1, wr = pos + nch - 1;
-          for (int kk = nch - 1; kk >= 0 && wr >= 0; --wr) {
-            const int jc = (int)cj[2 * kk + 1];
-            if (rd >= 0 && out[rd] > jc) out[wr] = out[rd--];
-            else { out[wr] = jc; --kk; }
+          // chosen i (ascending j) lands at before_i + i; the keys taken between before_i and
+          // before_{i+1} move up by i + 1. Done from the last chosen down, so nothing is overwritten.
+          int hi = pos;
+          for (int i = nch - 1; i >= 0; --i) {
+            const int before = min((int)cand[3 * i + 2], hi);
+            shift_up(out, before, hi, i + 1);
+            out[before + i] = (int)cand[3 * i + 1];
+            hi = before;
           }
           pos += nch;
         }
