@@ -10,20 +10,28 @@
 // Data movement and math:
 //   * Q tile: 128 rows x d bf16 in shared memory (K-major, 128B swizzle), loaded once.
 //   * The union of the tile's selections is built window by window over block ids (a shared
-//     bitmap of 32-bit query masks per block, one cursor per query) and consumed as 16-token
-//     superblocks aligned on block ids. Each superblock's K and V rows of the group arrive by
-//     3-D TMA boxes (16 tokens x 64 dims, 128B swizzle) into a 4-stage ring.
-//   * S[128 x 16] = Q K^T: tcgen05.mma (kind::f16, M=128, N=16) into TMEM, double-buffered.
-//   * Softmax: one thread per row (TMEM lane), masks from the bitmap (query selected the block,
-//     token <= query position). Pass 1 streams the union once for the exact row maxima (S only);
-//     pass 2 streams it again, forms P = exp2((S - max) * log2e / sqrt(d)) in bf16 into shared
-//     memory and accumulates O[128 x d] += P V with tcgen05.mma (V as an MN-major operand) in
-//     TMEM. With the exact maximum known up front there is no rescaling of O, and because
-//     superblocks are aligned on block ids and unselected slots contribute exact zeros, every
-//     row's arithmetic is the same whatever rows share its tile (bitwise causal, chunk-invariant).
+//     bitmap of 32-bit query masks per block) and consumed as 16-token superblocks aligned on
+//     block ids, four per chunk. Each chunk's K and V rows of the group arrive by 3-D TMA boxes
+//     (16 tokens x 64 dims, 128B swizzle) into a 3-stage ring; a missing superblock of the last
+//     chunk is loaded from out of bounds, which fills zeros.
+//   * S[128 x 64] = Q K^T per chunk: tcgen05.mma (kind::f16, M=128, N=64) into TMEM, double
+//     buffered.
+//   * Softmax: two threads per row (TMEM lane), each taking the chunk's superblocks of one block-id
+//     parity; masks from the bitmap (the query selected the block, token <= query position).
+//     Every row is scaled by a reference maximum computed up front on the CUDA cores from its
+//     own block (always selected), so there is a single streaming pass and no rescaling of O:
+//     P = exp2((S - m_ref) log2(e) / sqrt(d)), rounded to bf16 into shared memory. A row whose
+//     exponents exceed 2^60 anywhere is flagged, and if any row is, the tile streams the union
+//     again for exact maxima and then repeats the main pass (flagged rows with their exact
+//     maximum, the others with exactly the same arithmetic as before).
+//   * O[128 x d] += P V with tcgen05.mma (V as an MN-major operand) in TMEM, and the row sums
+//     l[128] += P 1 by one more MMA against a tile of ones, so l adds exactly the bf16 P that O
+//     adds, in the same order. Because superblocks are aligned on block ids, each is one K=16
+//     accumulation step, and unselected slots contribute exact zeros, every row's arithmetic is
+//     the same whatever rows share its tile (bitwise causal, chunk-invariant).
 //   * Epilogue: O / l times sigmoid(gate_logits), bf16.
-// Warp roles: warp 0 issues TMA, warp 1 allocates TMEM and issues MMAs, warps 2-5 run the
-// softmax and the epilogue; all six build the union. Every wait is bounded by %globaltimer: on
+// Warp roles: warp 0 issues TMA, warp 1 allocates TMEM and issues MMAs, warps 2-9 run the
+// softmax and the epilogue; all ten build the union. Every wait is bounded by %globaltimer: on
 // expiry the kernel records SGQA_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and
 // returns.
 #include <cmath>
@@ -58,14 +66,14 @@ struct AtcCfg {
   static constexpr int kStage = 2 * kKc;                // K then V
   static constexpr int kPsb = kM * kUnit * 2;           // P of one superblock: 128 x 16 bf16
   static constexpr int kP = kCH * kPsb;                 // P of one chunk
-  static constexpr int kSmem = 1024 + kQ + kNS * kStage + 2 * kP + 2 * kWin * 4 + 4096;
+  static constexpr int kOnes = 16 * 128;                // 16 x 64 bf16 ones: B operand of the row-sum MMA
+  static constexpr int kSmem = 1024 + kQ + kNS * kStage + 2 * kP + kOnes + 2 * kWin * 4 + 4096;
 };
 
 struct AtcShared {
   uint64_t kv_full[kNS], kv_empty[kNS], s_full[2], s_empty[2], p_full[2], p_empty[2], o_done;
   float ref_part[2][kM];  // per-row reference maxima from the own block (two halves of its tokens)
   float max_part[2][kM];  // per-row exact maxima by superblock parity (fallback pass)
-  float l_part[2][kM];    // per-row sums of P by superblock parity
   uint32_t wbits[kWinWords];
   uint32_t tmem;
   volatile int abort_flag;
@@ -123,11 +131,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   using C = AtcCfg<D>;
   constexpr int QT = kM / R;  // queries per tile (<= 32)
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* smem = smem_align<1024>(smem_raw);
   uint8_t* sQ = smem;
   uint8_t* sKV = sQ + C::kQ;                             // [stage][K|V][half][64 tokens][128 B]
   uint8_t* sP = sKV + kNS * C::kStage;                   // [2][superblock][16 groups][2][8 rows][16 B]
-  uint32_t* wmask = reinterpret_cast<uint32_t*>(sP + 2 * C::kP);
+  uint8_t* sOnes = sP + 2 * C::kP;                       // [16 rows][128 B] of bf16 1.0
+  uint32_t* wmask = reinterpret_cast<uint32_t*>(sOnes + C::kOnes);
   int32_t* usb = reinterpret_cast<int32_t*>(wmask + kWin);
   AtcShared* sh = reinterpret_cast<AtcShared*>(usb + kWin);
 
@@ -155,6 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (tid < kWinWords) sh->wbits[tid] = 0;
   for (int i = tid; i < kWin; i += kThreads) wmask[i] = 0;
+  for (int i = tid; i < C::kOnes / 4; i += kThreads) reinterpret_cast<uint32_t*>(sOnes)[i] = 0x3F803F80u;
   __syncthreads();
   if (tid < QT) {
     const int idx = tile * QT + tid;
@@ -162,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     sh->t[tid] = t;
     if (t >= 0) atomicMax(&sh->maxc, t / B);
   }
-  if (warp == 1) tc::tmem_alloc(&sh->tmem, 256);
+  if (warp == 1) tc::tmem_alloc(&sh->tmem, 512);
 
   // Q tile: row r = query r / R, head r % R; 16-byte chunk c of half h at
   // h * 16 KB + r * 128 + ((c ^ (r & 7)) * 16) (the 128B-swizzled K-major layout).
@@ -198,6 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::fence_after_sync();
   const uint32_t tmem = sh->tmem;
   const uint32_t tmem_o = tmem + 128;  // O: columns 128 .. 128 + D - 1; S buffers: columns 0 .. 127
+  const uint32_t tmem_l = tmem + 256;  // row sums of P: columns 256 .. 271 (all equal)
 
   // softmax role state (warps 2..9): TMEM lane quadrant warp % 4; `shalf` also picks the
   // superblocks (by block-id parity) and the own-block tokens this thread handles
@@ -241,7 +252,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const float m_ref = is_sm ? fmaxf(sh->ref_part[0][r], sh->ref_part[1][r]) : -INFINITY;
   float m_use = m_ref, m_exact = -INFINITY;
   bool risky = false;  // this row's scores exceed m_use by more than kRiskLog2
-  float l_half = 0.f;
 
   const int spb = kUnit >> lb;  // blocks per superblock
   long kc = 0;                  // chunks streamed (producer & MMA ring position)
@@ -249,6 +259,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   long pcnt = 0;                // P buffer uses (MMA & softmax)
   const uint32_t idesc_s = tc::idesc_bf16_f32(kM, kCT);
   const uint32_t idesc_pv = tc::idesc_bf16_f32(kM, D, true);
+  const uint32_t idesc_l = tc::idesc_bf16_f32(kM, 16);
+  const uint64_t d_ones = tc::smem_desc_kmajor(sOnes, 128);
   bool rerun = false;
 
   // pass 0: main (P V with the reference maximum); passes 1-2 only if some row was risky:
@@ -258,10 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (pass == 1 && !rerun) break;
     const bool main_pass = pass != 1;
     bool first_pv = true;
-    if (main_pass) {
-      l_half = 0.f;
-      if (pass == 2) m_use = risky ? m_exact : m_ref;
-    }
+    if (main_pass && pass == 2) m_use = risky ? m_exact : m_ref;
     for (int win = 0; win < nwin; ++win) {
       if (!sh->all_windows && !((sh->wbits[win >> 5] >> (win & 31)) & 1u)) continue;  // uniform
       const int w0 = win * kWin, w1 = w0 + kWin;
@@ -355,7 +364,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < kCH; ++i) {
               const uint64_t dp = tc::smem_desc_kmajor_noswz(sP + pb * C::kP + i * C::kPsb, 128, 256);
               const uint64_t dv = tc::smem_desc_mnmajor_sw128(vbase + i * (kUnit * 128), C::kHalfRows, 1024);
-              tc::mma_bf16_ss(tmem_o, dp, dv, idesc_pv, first_pv ? 0u : 1u);
+              const uint32_t acc = first_pv ? 0u : 1u;
+              tc::mma_bf16_ss(tmem_o, dp, dv, idesc_pv, acc);
+              tc::mma_bf16_ss(tmem_l, dp, d_ones, idesc_l, acc);  // l += P 1: the row sums, same order as O
               first_pv = false;
             }
             tc::mma_commit(&sh->kv_empty[st]);
@@ -441,18 +452,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if ((vmask >> k2) & 1u) m_exact = fmaxf(m_exact, __uint_as_float(v[i * kUnit + k2]));
               continue;
             }
+            // masked slots get -inf, whose exp2 is an exact 0; the row sums come from the MMA
             uint32_t pk[8];
-            float psum = 0.f, smax = -INFINITY;
+            float tmax = -INFINITY;
 #pragma unroll
             for (int k2 = 0; k2 < 8; ++k2) {
               const bool va = (vmask >> (2 * k2)) & 1u, vb = (vmask >> (2 * k2 + 1)) & 1u;
-              const float sa = __uint_as_float(v[i * kUnit + 2 * k2]), sbv = __uint_as_float(v[i * kUnit + 2 * k2 + 1]);
-              smax = fmaxf(smax, fmaxf(va ? sa : -INFINITY, vb ? sbv : -INFINITY));
-              pk[k2] = pack_bf16x2(va ? ex2_approx(fmaf(sa, sc, -base)) : 0.f, vb ? ex2_approx(fmaf(sbv, sc, -base)) : 0.f);
-              psum += bf16_lo(pk[k2]) + bf16_hi(pk[k2]);
+              const float ta = va ? fmaf(__uint_as_float(v[i * kUnit + 2 * k2]), sc, -base) : -INFINITY;
+              const float tb = vb ? fmaf(__uint_as_float(v[i * kUnit + 2 * k2 + 1]), sc, -base) : -INFINITY;
+              tmax = fmaxf(tmax, fmaxf(ta, tb));
+              pk[k2] = pack_bf16x2(ex2_approx(ta), ex2_approx(tb));
             }
-            if (smax * sc - base > kRiskLog2) risky = true;
-            l_half += psum;  // this half's superblocks in ascending order: a canonical order
+            if (tmax > kRiskLog2) risky = true;
             uint8_t* prow = sP + pb * C::kP + i * C::kPsb + (r >> 3) * 256 + (r & 7) * 16;
             *reinterpret_cast<uint4*>(prow) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             *reinterpret_cast<uint4*>(prow + 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
@@ -479,9 +490,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (is_sm) m_exact = fmaxf(sh->max_part[0][r], sh->max_part[1][r]);
     }
   }
-  if (is_sm) sh->l_part[shalf][r] = l_half;
-  __syncthreads();
-  const float l_r = is_sm ? sh->l_part[0][r] + sh->l_part[1][r] : 0.f;
 
   // ---- epilogue ----
   // o_done arrives once every MMA this thread issued has completed (at once if none was issued)
@@ -490,6 +498,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = warp_wait(&sh->o_done, 0, &sh->abort_flag);
     if (ok) {
       tc::fence_after_sync();
+      uint32_t lv[16];
+      tc::tmem_ld16(tmem_l + lane_base, lv);
+      const float l_r = __uint_as_float(lv[0]);
       const float inv = l_r > 0.f ? 1.f / l_r : 0.f;
       const long orow = t_r >= 0 ? ((long)b * a.nQ + (t_r - a.q_t0)) * a.Hq + (long)g * R + h_r : -1;
 #pragma unroll 1
@@ -538,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, 256);
+    tc::tmem_dealloc(tmem, 512);
   }
 }
 
