@@ -211,7 +211,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_l = tmem + 256;  // row sums of P: columns 256 .. 271 (all equal)
 
   // softmax role state (warps 2..9): TMEM lane quadrant warp % 4; `shalf` also picks the
-  // superblocks (by block-id parity) and the own-block tokens this thread handles
+  // half of every chunk (superblocks 2 shalf, 2 shalf + 1) and the own-block tokens this thread
+  // handles
   const bool is_sm = warp >= 2;
   const int quad = warp & 3;
   const int shalf = is_sm ? (warp - 2) / 4 : 0;
@@ -407,8 +408,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else {
-        // ---- softmax: one row per thread pair; each handles the superblocks whose id parity
-        // is `shalf` (a fixed, tile-independent split of the row's work) ----
+        // ---- softmax: one row per thread pair, each taking half of every chunk (the split
+        // does not enter the arithmetic: P is elementwise, the row sums come from the MMA) ----
         for (int ch = 0; ch < nch; ++ch, ++scnt) {
           const int sb = (int)(scnt & 1);
           if (!warp_wait(&sh->s_full[sb], (uint32_t)((scnt >> 1) & 1), &sh->abort_flag)) {
@@ -417,8 +418,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc::fence_after_sync();
-          uint32_t v[kCT];
-          tc::tmem_ld64(tmem + lane_base + (uint32_t)(sb * kCT), v);
+          constexpr int kHalfCT = kCT / 2;
+          uint32_t v[kHalfCT];
+          tc::tmem_ld32(tmem + lane_base + (uint32_t)(sb * kCT + shalf * kHalfCT), v);
           tc::fence_before_sync();
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(&sh->s_empty[sb]);
@@ -431,11 +433,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const float base = m_use * sc;
 #pragma unroll
-          for (int i = 0; i < kCH; ++i) {
+          for (int ii = 0; ii < kCH / 2; ++ii) {
+            const int i = shalf * (kCH / 2) + ii;
             const int e = ch * kCH + i;
             const int sbid = e < nu ? usb[e] : -1;
-            const bool mine = sbid >= 0 ? ((sbid & 1) == shalf) : (shalf == 0);
-            if (!mine) continue;
             uint32_t vmask = 0;  // bit k: token sbid * 16 + k is valid for this row
             if (sbid >= 0 && t_r >= 0) {
               const int u0 = sbid * kUnit;
@@ -449,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!main_pass) {
 #pragma unroll
               for (int k2 = 0; k2 < kUnit; ++k2)
-                if ((vmask >> k2) & 1u) m_exact = fmaxf(m_exact, __uint_as_float(v[i * kUnit + k2]));
+                if ((vmask >> k2) & 1u) m_exact = fmaxf(m_exact, __uint_as_float(v[ii * kUnit + k2]));
               continue;
             }
             // masked slots get -inf, whose exp2 is an exact 0; the row sums come from the MMA
@@ -458,8 +459,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k2 = 0; k2 < 8; ++k2) {
               const bool va = (vmask >> (2 * k2)) & 1u, vb = (vmask >> (2 * k2 + 1)) & 1u;
-              const float ta = va ? fmaf(__uint_as_float(v[i * kUnit + 2 * k2]), sc, -base) : -INFINITY;
-              const float tb = vb ? fmaf(__uint_as_float(v[i * kUnit + 2 * k2 + 1]), sc, -base) : -INFINITY;
+              const float ta = va ? fmaf(__uint_as_float(v[ii * kUnit + 2 * k2]), sc, -base) : -INFINITY;
+              const float tb = vb ? fmaf(__uint_as_float(v[ii * kUnit + 2 * k2 + 1]), sc, -base) : -INFINITY;
               tmax = fmaxf(tmax, fmaxf(ta, tb));
               pk[k2] = pack_bf16x2(ex2_approx(ta), ex2_approx(tb));
             }
