@@ -49,13 +49,14 @@ constexpr int kCH = 4;       // superblocks per chunk (one handshake between MMA
 constexpr int kCT = kCH * kUnit;  // token slots per chunk
 constexpr int kWin = 2048;   // block ids per union window
 constexpr int kWinWords = 16;     // occupancy bits for up to 512 windows
-constexpr int kNS = 3;       // K/V chunk stages
+constexpr int kNS = 4;       // K/V chunk stages
 constexpr int kSmWarps = 8;  // softmax warps: two per TMEM lane quadrant
 constexpr int kThreads = (2 + kSmWarps) * 32;
 constexpr int kM = 128;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kRiskLog2 = 60.f;  // a row whose scores exceed its reference by more than this (log2)
-                                   // is recomputed with its exact maximum
+constexpr float kRiskSum = 1.152921504606846976e18f;  // 2^60: a row whose sum of P (scaled by its
+                                                     // reference maximum) exceeds this, or is not
+                                                     // finite, is recomputed with its exact maximum
 
 template <int D>
 struct AtcCfg {
@@ -252,7 +253,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   const float m_ref = is_sm ? fmaxf(sh->ref_part[0][r], sh->ref_part[1][r]) : -INFINITY;
   float m_use = m_ref, m_exact = -INFINITY;
-  bool risky = false;  // this row's scores exceed m_use by more than kRiskLog2
+  bool risky = false;  // this row's P sum exceeds kRiskSum (some exponent is near the fp32 range)
+  bool o_ok = false;   // this thread saw the last main pass's MMAs complete
+  int o_phase = 0, o_commits = 0;
 
   const int spb = kUnit >> lb;  // blocks per superblock
   long kc = 0;                  // chunks streamed (producer & MMA ring position)
@@ -455,16 +458,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // masked slots get -inf, whose exp2 is an exact 0; the row sums come from the MMA
             uint32_t pk[8];
-            float tmax = -INFINITY;
 #pragma unroll
             for (int k2 = 0; k2 < 8; ++k2) {
               const bool va = (vmask >> (2 * k2)) & 1u, vb = (vmask >> (2 * k2 + 1)) & 1u;
               const float ta = va ? fmaf(__uint_as_float(v[ii * kUnit + 2 * k2]), sc, -base) : -INFINITY;
               const float tb = vb ? fmaf(__uint_as_float(v[ii * kUnit + 2 * k2 + 1]), sc, -base) : -INFINITY;
-              tmax = fmaxf(tmax, fmaxf(ta, tb));
               pk[k2] = pack_bf16x2(ex2_approx(ta), ex2_approx(tb));
             }
-            if (tmax > kRiskLog2) risky = true;
             uint8_t* prow = sP + pb * C::kP + i * C::kPsb + (r >> 3) * 256 + (r & 7) * 16;
             *reinterpret_cast<uint4*>(prow) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             *reinterpret_cast<uint4*>(prow + 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
@@ -483,6 +483,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < spb; ++i) wmask[(usb[e] * spb + i) - w0] = 0u;
       __syncthreads();
     }
+    if (main_pass) {
+      // all of this pass's MMAs have completed once o_done arrives (at once if none was issued);
+      // after the first pass the row sums tell which rows need their exact maximum
+      if (warp == 1 && lane == 0) {
+        tc::mma_commit(&sh->o_done);
+        ++o_commits;
+      }
+      if (is_sm) {
+        o_ok = warp_wait(&sh->o_done, (uint32_t)o_phase, &sh->abort_flag);
+        if (!o_ok) {
+          if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
+          sh->abort_flag = 1;
+        } else if (pass == 0) {
+          tc::fence_after_sync();
+          uint32_t lv[16];
+          tc::tmem_ld16(tmem_l + lane_base, lv);
+          risky = !(__uint_as_float(lv[0]) <= kRiskSum);
+        }
+      }
+      o_phase ^= 1;
+    }
     if (pass == 0) {
       rerun = __syncthreads_or(is_sm && risky) != 0;
     } else if (pass == 1) {
@@ -493,11 +514,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // ---- epilogue ----
-  // o_done arrives once every MMA this thread issued has completed (at once if none was issued)
-  if (warp == 1 && lane == 0) tc::mma_commit(&sh->o_done);
   if (is_sm) {
-    bool ok = warp_wait(&sh->o_done, 0, &sh->abort_flag);
-    if (ok) {
+    if (o_ok) {
       tc::fence_after_sync();
       uint32_t lv[16];
       tc::tmem_ld16(tmem_l + lane_base, lv);
@@ -527,9 +545,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-    } else if (lane == 0 && !sh->abort_flag) {
-      report(a.status, SGQA_ERR_TIMEOUT);
-      sh->abort_flag = 1;
     }
   }
 
@@ -542,9 +557,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_wait(&sh->kv_full[k2 % kNS], (uint32_t)((k2 / kNS) & 1), &no_abort);
     }
   }
-  if (warp == 1 && lane == 0) {
+  if (warp == 1 && lane == 0 && o_commits > 0) {  // every MMA issued must finish before TMEM is freed
     volatile int no_abort = 0;
-    tc::mbar_wait(&sh->o_done, 0, &no_abort);
+    tc::mbar_wait(&sh->o_done, (uint32_t)((o_commits - 1) & 1), &no_abort);
   }
   tc::fence_before_sync();
   __syncthreads();

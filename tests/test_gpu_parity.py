@@ -16,6 +16,7 @@ torch = pytest.importorskip("torch")
 
 import oracle
 import block_sparse_long_kbar_b200 as sg
+import sgqa_inputs as sgi
 from sgqa_inputs import CONFIGS, DECODE_NEW, Config, gen_device, gen_rows
 from tests._helpers import (NAMES, all_rows, assert_outputs_close, compare_selection, device_inputs, host_inputs,
                             output_errors, sample_rows, shape_of, to_dev, to_host)
@@ -110,6 +111,53 @@ def test_attend_with_oracle_selection(small_cases, name):
     ref = oracle.attend(dm, rows, h["q"].reshape(len(rows), -1), h["k"], h["v"], h["gate"].reshape(len(rows), -1),
                         sel_o)
     assert_outputs_close(to_host(out), ref.reshape(shape_of(cfg, "q")), name)
+
+
+def test_attend_rows_far_above_their_reference_max(small_cases):
+    """Rows whose scores exceed their own block's maximum by far more than the fp32 exponent range
+    allows to keep unscaled: the keys of block 0 are scaled by 64 and every row selects block 0,
+    so the tile is streamed again with exact maxima for those rows (the kernel's fallback).
+    Such rows attend almost to one token, so their outputs are as large as single values of v;
+    v is scaled by 1/4 so that the bf16 rounding of the output alone (half an ulp, 2^-6 at
+    |y| >= 4) stays well inside the max-abs bound."""
+    cfg, h, d, dm, kbar64, rows, sel_o, s_m = small_cases("ragged_g4")
+    k = h["k"].copy()
+    kf = sgi.bf16_bits_to_f64(k[:, :cfg.B]) * 64.0  # exact: a power of two
+    k[:, :cfg.B] = sgi.f64_to_bf16_bits(kf)
+    v = sgi.f64_to_bf16_bits(sgi.bf16_bits_to_f64(h["v"]) * 0.25)
+    sel = sel_o.reshape(-1, cfg.Kb).copy()
+    for i in range(sel.shape[0]):
+        t = int(rows[i // cfg.G][1])
+        c = t // cfg.B
+        s = [int(j) for j in sel[i] if j >= 0]
+        if 0 not in s:
+            if len(s) >= cfg.Kb:
+                s.remove(next(j for j in s if j != c))
+            s = sorted(s + [0])
+        sel[i] = s + [-1] * (cfg.Kb - len(s))
+    sel = sel.reshape(sel_o.shape)
+    # the case is really exercised: some row's block-0 score is far above its own block's
+    qf = sgi.bf16_bits_to_f64(h["q"].reshape(len(rows), cfg.Hq, cfg.d))
+    kk = sgi.bf16_bits_to_f64(k.reshape(cfg.batch, cfg.T, cfg.G, cfg.d))
+    sc = np.log2(np.e) / np.sqrt(cfg.d)
+    gap = 0.0
+    for i in range(100, len(rows), 997):
+        b, t = int(rows[i][0]), int(rows[i][1])
+        c = t // cfg.B
+        for hq in range(0, cfg.Hq, 5):
+            g = hq // cfg.R
+            s0 = kk[b, :cfg.B, g] @ qf[i, hq]
+            so = kk[b, c * cfg.B:t + 1, g] @ qf[i, hq]
+            gap = max(gap, (s0.max() - so.max()) * sc)
+    assert gap > 80, gap
+    dims = sg.sgqa_dims.of(cfg)
+    ws = _ws(dims)
+    out = torch.full(shape_of(cfg, "q"), float("nan"), dtype=torch.bfloat16, device="cuda")
+    sg.sgqa_attend(dims, d["q"], to_dev(k, shape_of(cfg, "k")), to_dev(v, shape_of(cfg, "v")), d["gate"],
+                   torch.from_numpy(sel.reshape(cfg.batch, cfg.T, cfg.G, cfg.Kb)).cuda(), out, ws)
+    _status_ok(ws)
+    ref = oracle.attend(dm, rows, h["q"].reshape(len(rows), -1), k, v, h["gate"].reshape(len(rows), -1), sel)
+    assert_outputs_close(to_host(out), ref.reshape(shape_of(cfg, "q")), "far above reference")
 
 
 @pytest.mark.parametrize("name", list(SMALL))
