@@ -50,6 +50,7 @@ constexpr int kCT = kCH * kUnit;  // token slots per chunk
 constexpr int kWin = 2048;   // block ids per union window
 constexpr int kWinWords = 16;     // occupancy bits for up to 512 windows
 constexpr int kNS = 4;       // K/V chunk stages
+constexpr int kPB = 2;       // P buffers in shared memory
 constexpr int kSmWarps = 8;  // softmax warps: two per TMEM lane quadrant
 constexpr int kThreads = (2 + kSmWarps) * 32;
 constexpr int kM = 128;
@@ -68,11 +69,11 @@ struct AtcCfg {
   static constexpr int kPsb = kM * kUnit * 2;           // P of one superblock: 128 x 16 bf16
   static constexpr int kP = kCH * kPsb;                 // P of one chunk
   static constexpr int kOnes = 16 * 128;                // 16 x 64 bf16 ones: B operand of the row-sum MMA
-  static constexpr int kSmem = 1024 + kQ + kNS * kStage + 2 * kP + kOnes + 2 * kWin * 4 + 4096;
+  static constexpr int kSmem = 1024 + kQ + kNS * kStage + kPB * kP + kOnes + 2 * kWin * 4 + 4096;
 };
 
 struct AtcShared {
-  uint64_t kv_full[kNS], kv_empty[kNS], s_full[2], s_empty[2], p_full[2], p_empty[2], o_done;
+  uint64_t kv_full[kNS], kv_empty[kNS], s_full[2], s_empty[2], p_full[kPB], p_empty[kPB], o_done;
   float ref_part[2][kM];  // per-row reference maxima from the own block (two halves of its tokens)
   float max_part[2][kM];  // per-row exact maxima by superblock parity (fallback pass)
   uint32_t wbits[kWinWords];
@@ -135,8 +136,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_align<1024>(smem_raw);
   uint8_t* sQ = smem;
   uint8_t* sKV = sQ + C::kQ;                             // [stage][K|V][half][64 tokens][128 B]
-  uint8_t* sP = sKV + kNS * C::kStage;                   // [2][superblock][16 groups][2][8 rows][16 B]
-  uint8_t* sOnes = sP + 2 * C::kP;                       // [16 rows][128 B] of bf16 1.0
+  uint8_t* sP = sKV + kNS * C::kStage;                   // [kPB][superblock][16 groups][2][8 rows][16 B]
+  uint8_t* sOnes = sP + kPB * C::kP;                     // [16 rows][128 B] of bf16 1.0
   uint32_t* wmask = reinterpret_cast<uint32_t*>(sOnes + C::kOnes);
   int32_t* usb = reinterpret_cast<int32_t*>(wmask + kWin);
   AtcShared* sh = reinterpret_cast<AtcShared*>(usb + kWin);
@@ -154,6 +155,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&sh->s_full[i], 1);
       tc::mbar_init(&sh->s_empty[i], kSmWarps);
+    }
+    for (int i = 0; i < kPB; ++i) {
       tc::mbar_init(&sh->p_full[i], kSmWarps);
       tc::mbar_init(&sh->p_empty[i], 1);
     }
@@ -359,8 +362,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
           long pend_stage = -1;  // ring position of the chunk whose P V is still to issue
           auto issue_pv = [&](long stage_of) -> bool {
-            const int pb = (int)(pcnt & 1);
-            if (!tc::mbar_wait(&sh->p_full[pb], (uint32_t)((pcnt >> 1) & 1), &sh->abort_flag)) return false;
+            const int pb = (int)(pcnt % kPB);
+            if (!tc::mbar_wait(&sh->p_full[pb], (uint32_t)((pcnt / kPB) & 1), &sh->abort_flag)) return false;
             tc::fence_after_sync();
             const int st = (int)(stage_of % kNS);
             const uint8_t* vbase = sKV + st * C::kStage + C::kKc;
@@ -427,9 +430,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::fence_before_sync();
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(&sh->s_empty[sb]);
-          const int pb = (int)(pcnt & 1);
-          if (main_pass && pcnt >= 2 &&
-              !warp_wait(&sh->p_empty[pb], (uint32_t)(((pcnt >> 1) - 1) & 1), &sh->abort_flag)) {
+          const int pb = (int)(pcnt % kPB);
+          if (main_pass && pcnt >= kPB &&
+              !warp_wait(&sh->p_empty[pb], (uint32_t)(((pcnt / kPB) - 1) & 1), &sh->abort_flag)) {
             if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
             sh->abort_flag = 1;
             break;
@@ -440,30 +443,47 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int i = shalf * (kCH / 2) + ii;
             const int e = ch * kCH + i;
             const int sbid = e < nu ? usb[e] : -1;
-            uint32_t vmask = 0;  // bit k: token sbid * 16 + k is valid for this row
-            if (sbid >= 0 && t_r >= 0) {
-              const int u0 = sbid * kUnit;
-              for (int blk = 0; blk < spb; ++blk) {
-                const int j = (u0 >> lb) + blk;
-                if ((wmask[j - w0] >> q_r) & 1u) vmask |= ((1u << (1 << lb)) - 1u) << (blk << lb);
-              }
-              const int lim = t_r - u0;
-              if (lim < 15) vmask &= lim < 0 ? 0u : ((2u << lim) - 1u);
-            }
-            if (!main_pass) {
-#pragma unroll
-              for (int k2 = 0; k2 < kUnit; ++k2)
-                if ((vmask >> k2) & 1u) m_exact = fmaxf(m_exact, __uint_as_float(v[ii * kUnit + k2]));
-              continue;
-            }
-            // masked slots get -inf, whose exp2 is an exact 0; the row sums come from the MMA
+            const int u0 = sbid * kUnit;
+            const bool live = sbid >= 0 && t_r >= 0;
             uint32_t pk[8];
+            if (main_pass && lb >= 3 && live && u0 + (kUnit - 1) <= t_r) {
+              // blocks of 8 or 16 tokens wholly before the row's token: the selection bit of each
+              // half superblock becomes the additive term of the exponent (-inf when unselected,
+              // whose exp2 is an exact 0); no per-token mask
+              const int jb = (u0 >> lb) - w0;
+              const float bias0 = ((wmask[jb] >> q_r) & 1u) ? -base : -INFINITY;
+              const float bias1 = ((wmask[jb + spb - 1] >> q_r) & 1u) ? -base : -INFINITY;
 #pragma unroll
-            for (int k2 = 0; k2 < 8; ++k2) {
-              const bool va = (vmask >> (2 * k2)) & 1u, vb = (vmask >> (2 * k2 + 1)) & 1u;
-              const float ta = va ? fmaf(__uint_as_float(v[ii * kUnit + 2 * k2]), sc, -base) : -INFINITY;
-              const float tb = vb ? fmaf(__uint_as_float(v[ii * kUnit + 2 * k2 + 1]), sc, -base) : -INFINITY;
-              pk[k2] = pack_bf16x2(ex2_approx(ta), ex2_approx(tb));
+              for (int k2 = 0; k2 < 8; ++k2) {
+                const float bias = k2 < 4 ? bias0 : bias1;
+                const float ta = fmaf(__uint_as_float(v[ii * kUnit + 2 * k2]), sc, bias);
+                const float tb = fmaf(__uint_as_float(v[ii * kUnit + 2 * k2 + 1]), sc, bias);
+                pk[k2] = pack_bf16x2(ex2_approx(ta), ex2_approx(tb));
+              }
+            } else {
+              uint32_t vmask = 0;  // bit k: token sbid * 16 + k is valid for this row
+              if (live) {
+                for (int blk = 0; blk < spb; ++blk) {
+                  const int j = (u0 >> lb) + blk;
+                  if ((wmask[j - w0] >> q_r) & 1u) vmask |= ((1u << (1 << lb)) - 1u) << (blk << lb);
+                }
+                const int lim = t_r - u0;
+                if (lim < 15) vmask &= lim < 0 ? 0u : ((2u << lim) - 1u);
+              }
+              if (!main_pass) {
+#pragma unroll
+                for (int k2 = 0; k2 < kUnit; ++k2)
+                  if ((vmask >> k2) & 1u) m_exact = fmaxf(m_exact, __uint_as_float(v[ii * kUnit + k2]));
+                continue;
+              }
+              // masked slots get -inf, whose exp2 is an exact 0; the row sums come from the MMA
+#pragma unroll
+              for (int k2 = 0; k2 < 8; ++k2) {
+                const bool va = (vmask >> (2 * k2)) & 1u, vb = (vmask >> (2 * k2 + 1)) & 1u;
+                const float ta = va ? fmaf(__uint_as_float(v[ii * kUnit + 2 * k2]), sc, -base) : -INFINITY;
+                const float tb = vb ? fmaf(__uint_as_float(v[ii * kUnit + 2 * k2 + 1]), sc, -base) : -INFINITY;
+                pk[k2] = pack_bf16x2(ex2_approx(ta), ex2_approx(tb));
+              }
             }
             uint8_t* prow = sP + pb * C::kP + i * C::kPsb + (r >> 3) * 256 + (r & 7) * 16;
             *reinterpret_cast<uint4*>(prow) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
