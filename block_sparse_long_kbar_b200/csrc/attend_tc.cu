@@ -557,8 +557,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 4; ++i) {
               const float o0 = inv > 0.f ? __uint_as_float(o[c8 * 8 + 2 * i]) * inv : 0.f;
               const float o1 = inv > 0.f ? __uint_as_float(o[c8 * 8 + 2 * i + 1]) * inv : 0.f;
-              const float y0 = o0 * (1.f / (1.f + expf(-bf16_lo(gw[i]))));
-              const float y1 = o1 * (1.f / (1.f + expf(-bf16_hi(gw[i]))));
+              const float y0 = o0 * sigmoid_fast(bf16_lo(gw[i]));
+              const float y1 = o1 * sigmoid_fast(bf16_hi(gw[i]));
               ov[i] = pack_bf16x2(y0, y1);
             }
             *reinterpret_cast<uint4*>(a.out + off) = make_uint4(ov[0], ov[1], ov[2], ov[3]);

@@ -36,6 +36,12 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// Gate of the Gated-GQA epilogue, sigmoid(x) = 1 / (1 + 2^(-x log2 e)), from the hardware
+// exp2 approximation and a fast divide; both errors are far below the bf16 rounding of the
+// output it multiplies. Saturates to 0 (2^.. = inf) and 1 (2^.. = 0) at the ends.
+__device__ __forceinline__ float sigmoid_fast(float x) {
+  return __fdividef(1.f, 1.f + ex2_approx(-1.4426950408889634f * x));
+}
 
 // Order-preserving map of an fp32 score to uint32 (larger score -> larger key). -0 is first
 // folded into +0 so that equal scores give equal keys.
