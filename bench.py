@@ -36,6 +36,18 @@ CLOCK_FIELDS = ["pci.bus_id", "clocks.sm", "clocks.max.sm", "power.draw", "clock
                 "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
 
 
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the current kernels,
+# from the ncu captures summarised in profiles/select_tc_attend_tc_32k.md: the attend kernel moved
+# 2.284 GB on the 32K workload (65536 query tokens), exactly its compulsory bytes, which are all
+# per query token; the 128K entry is that capture scaled by the 131072 query tokens of a launch.
+# An entry must be dropped (None) when its kernel changes.
+NCU_TRAFFIC = {
+    ("attend", "32k"): 2.2838e9,
+    ("attend", "128k"): 2.2838e9 * 131072 / 65536,
+    ("select", "32k"): 0.5201e9,
+}
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -280,7 +292,7 @@ def run_ours(args, world, rank):
     roof = dict(stage_roof[dominant])
     roof.pop("ms")
     roof["kernel"] = dominant
-    roof["traffic"] = None
+    roof["traffic"] = NCU_TRAFFIC.get((dominant, cfg.name))
     roof["peak_source"] = peaks["source"]
 
     # end to end through the C ABI with host buffers: H2D of the step's inputs, D2H of its output
