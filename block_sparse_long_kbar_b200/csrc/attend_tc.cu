@@ -11,18 +11,18 @@
 //   * Q tile: 128 rows x d bf16 in shared memory (K-major, 128B swizzle), loaded once.
 //   * The union of the tile's selections is built window by window over block ids (a shared
 //     bitmap of 32-bit query masks per block) and consumed as 16-token superblocks aligned on
-//     block ids, four per chunk. Each chunk's K and V rows of the group arrive by 3-D TMA boxes
+//     block ids, two per chunk. Each chunk's K and V rows of the group arrive by 3-D TMA boxes
 //     (16 tokens x 64 dims, 128B swizzle) into a 3-stage ring; a missing superblock of the last
 //     chunk is loaded from out of bounds, which fills zeros.
-//   * S[128 x 64] = Q K^T per chunk: tcgen05.mma (kind::f16, M=128, N=64) into TMEM, double
+//   * S[128 x 32] = Q K^T per chunk: tcgen05.mma (kind::f16, M=128, N=32) into TMEM, double
 //     buffered.
-//   * Softmax: two threads per row (TMEM lane), each taking the chunk's superblocks of one block-id
-//     parity; masks from the bitmap (the query selected the block, token <= query position).
+//   * Softmax: two threads per row (TMEM lane), each taking one of the chunk's two superblocks;
+//     masks from the bitmap (the query selected the block, token <= query position).
 //     Every row is scaled by a reference maximum computed up front on the CUDA cores from its
 //     own block (always selected), so there is a single streaming pass and no rescaling of O:
 //     P = exp2((S - m_ref) log2(e) / sqrt(d)), rounded to bf16 into shared memory. A row whose
-//     exponents exceed 2^60 anywhere is flagged, and if any row is, the tile streams the union
-//     again for exact maxima and then repeats the main pass (flagged rows with their exact
+//     sum of P exceeds 2^60 or is not finite is flagged, and if any row is, the tile streams the
+//     union again for exact maxima and then repeats the main pass (flagged rows with their exact
 //     maximum, the others with exactly the same arithmetic as before).
 //   * O[128 x d] += P V with tcgen05.mma (V as an MN-major operand) in TMEM, and the row sums
 //     l[128] += P 1 by one more MMA against a tile of ones, so l adds exactly the bf16 P that O
@@ -31,7 +31,8 @@
 //     the same whatever rows share its tile (bitwise causal, chunk-invariant).
 //   * Epilogue: O / l times sigmoid(gate_logits), bf16.
 // Warp roles: warp 0 issues TMA, warp 1 allocates TMEM and issues MMAs, warps 2-9 run the
-// softmax and the epilogue; all ten build the union. Every wait is bounded by %globaltimer: on
+// softmax and the epilogue; all ten build the union. Two tiles are resident per SM (shared memory
+// and TMEM are sized for it), so one tile's union, setup and epilogue overlap the other's chunks. Every wait is bounded by %globaltimer: on
 // expiry the kernel records SGQA_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and
 // returns.
 #include <cmath>
@@ -45,14 +46,16 @@ namespace sgqa {
 namespace {
 
 constexpr int kUnit = 16;    // tokens per superblock
-constexpr int kCH = 4;       // superblocks per chunk (one handshake between MMA and softmax)
+constexpr int kCH = 2;       // superblocks per chunk (one handshake between MMA and softmax)
 constexpr int kCT = kCH * kUnit;  // token slots per chunk
-constexpr int kWin = 2048;   // block ids per union window
+constexpr int kWin = 1024;   // block ids per union window
 constexpr int kWinWords = 16;     // occupancy bits for up to 512 windows
-constexpr int kNS = 4;       // K/V chunk stages
+constexpr int kNS = 3;       // K/V chunk stages
 constexpr int kPB = 2;       // P buffers in shared memory
 constexpr int kSmWarps = 8;  // softmax warps: two per TMEM lane quadrant
 constexpr int kThreads = (2 + kSmWarps) * 32;
+constexpr int kCtasPerSm = 2;  // two tiles resident per SM: one's union, setup and epilogue overlap
+                               // the other's chunk loop
 constexpr int kM = 128;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRiskSum = 1.152921504606846976e18f;  // 2^60: a row whose sum of P (scaled by its
@@ -63,13 +66,17 @@ template <int D>
 struct AtcCfg {
   static constexpr int kHalves = D / 64;
   static constexpr int kQ = kM * D * 2;                 // [half][128 rows][128 B]
-  static constexpr int kHalfRows = kCT * 128;           // one 64-dim half of a chunk: [64 tokens][128 B]
+  static constexpr int kHalfRows = kCT * 128;           // one 64-dim half of a chunk: [kCT tokens][128 B]
   static constexpr int kKc = kHalves * kHalfRows;       // K (or V) of one chunk: [half][64][128 B]
   static constexpr int kStage = 2 * kKc;                // K then V
   static constexpr int kPsb = kM * kUnit * 2;           // P of one superblock: 128 x 16 bf16
   static constexpr int kP = kCH * kPsb;                 // P of one chunk
   static constexpr int kOnes = 16 * 128;                // 16 x 64 bf16 ones: B operand of the row-sum MMA
   static constexpr int kSmem = 1024 + kQ + kNS * kStage + kPB * kP + kOnes + 2 * kWin * 4 + 4096;
+  static_assert(kCtasPerSm * (kSmem + 1024) <= 233472, "shared memory for the resident tiles");
+  static constexpr int kSCols = 2 * kCT;                // TMEM: S buffers, then O (D), then l (16)
+  static constexpr int kTmemCols = kSCols + D + 16 <= 256 ? 256 : 512;
+  static_assert(kCtasPerSm * kTmemCols <= 512, "TMEM for the resident tiles");
 };
 
 struct AtcShared {
@@ -127,7 +134,7 @@ __device__ __forceinline__ void for_each_selected(const int32_t* row, int Kb, in
 }
 
 template <int D, int R>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
     attend_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
                      AttendArgs a, const uint32_t* __restrict__ perm, int n_per_seg, int tiles_per_seg, int lb) {
   using C = AtcCfg<D>;
@@ -135,7 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_align<1024>(smem_raw);
   uint8_t* sQ = smem;
-  uint8_t* sKV = sQ + C::kQ;                             // [stage][K|V][half][64 tokens][128 B]
+  uint8_t* sKV = sQ + C::kQ;                             // [stage][K|V][half][kCT tokens][128 B]
   uint8_t* sP = sKV + kNS * C::kStage;                   // [kPB][superblock][16 groups][2][8 rows][16 B]
   uint8_t* sOnes = sP + kPB * C::kP;                     // [16 rows][128 B] of bf16 1.0
   uint32_t* wmask = reinterpret_cast<uint32_t*>(sOnes + C::kOnes);
@@ -176,7 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     sh->t[tid] = t;
     if (t >= 0) atomicMax(&sh->maxc, t / B);
   }
-  if (warp == 1) tc::tmem_alloc(&sh->tmem, 512);
+  if (warp == 1) tc::tmem_alloc(&sh->tmem, C::kTmemCols);
 
   // Q tile: row r = query r / R, head r % R; 16-byte chunk c of half h at
   // h * 16 KB + r * 128 + ((c ^ (r & 7)) * 16) (the 128B-swizzled K-major layout).
@@ -211,8 +218,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = sh->tmem;
-  const uint32_t tmem_o = tmem + 128;  // O: columns 128 .. 128 + D - 1; S buffers: columns 0 .. 127
-  const uint32_t tmem_l = tmem + 256;  // row sums of P: columns 256 .. 271 (all equal)
+  const uint32_t tmem_o = tmem + C::kSCols;  // O: D columns after the two S buffers
+  const uint32_t tmem_l = tmem_o + D;        // row sums of P: 16 columns (all equal)
 
   // softmax role state (warps 2..9): TMEM lane quadrant warp % 4; `shalf` also picks the
   // half of every chunk (superblocks 2 shalf, 2 shalf + 1) and the own-block tokens this thread
@@ -426,7 +433,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::fence_after_sync();
           constexpr int kHalfCT = kCT / 2;
           uint32_t v[kHalfCT];
-          tc::tmem_ld32(tmem + lane_base + (uint32_t)(sb * kCT + shalf * kHalfCT), v);
+          static_assert(kHalfCT == 16, "one superblock of S per softmax thread and chunk");
+          tc::tmem_ld16(tmem + lane_base + (uint32_t)(sb * kCT + shalf * kHalfCT), v);
           tc::fence_before_sync();
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(&sh->s_empty[sb]);
@@ -585,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, 512);
+    tc::tmem_dealloc(tmem, C::kTmemCols);
   }
 }
 

@@ -123,6 +123,11 @@ __device__ __forceinline__ void red_shared_add(uint32_t addr, uint32_t val) {
   asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(addr), "r"(val) : "memory");
 }
 
+__device__ __forceinline__ void st_shared_u32_if(uint32_t addr, uint32_t v, uint32_t pred) {
+  asm volatile("{ .reg .pred p; setp.ne.u32 p, %2, 0; @p st.shared.u32 [%0], %1; }" ::"r"(addr), "r"(v), "r"(pred)
+               : "memory");
+}
+
 // Histogram pass: count, in the row's 256 bins, the next 8 key bits (at `shift`) of the keys
 // whose resolved bits (mask) equal prefix. kFull: all 64 candidates exist (else only q < lim).
 template <bool kFull, bool kFirst>
@@ -509,16 +514,22 @@ __global__ void __launch_bounds__(kThreads, 1)
               emit_chunk<true>(v, lim, thr, blo, bw, tie_lim, col_lim, my_hist, j0, pos, eqn, tb);
             else if (lim > 0)
               emit_chunk<false>(v, lim, thr, blo, bw, tie_lim, col_lim, my_hist, j0, pos, eqn, tb);
-            // stage the taken indices in order (warp-uniform trip count: no divergent loop), then
+            // stage the taken indices in order, each at the position the population count of
+            // the taken bits below it gives (predicated stores, no loop over set bits), then
             // write out the rows that have 64 staged
+            const uint32_t ring_base = smem_u32(ring);
 #pragma unroll
             for (int w = 0; w < 2; ++w) {
-              uint32_t bits = tb[w];
-              const int n_it = (int)__reduce_max_sync(0xFFFFFFFFu, (unsigned)__popc(bits));
-              for (int it = 0; it < n_it; ++it) {
-                const int q = __ffs(bits) - 1;
-                bits &= bits - 1u;
-                if (q >= 0 && pos < m) ring[pos++ & 127] = (uint32_t)(j0 + 32 * w + q);
+              const uint32_t bits = tb[w];
+              if (__any_sync(0xFFFFFFFFu, bits != 0u)) {
+                const int base = pos;
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                  const int ps = base + __popc(bits & ((1u << q) - 1u));
+                  st_shared_u32_if(ring_base + ((uint32_t)(ps & 127) << 2), (uint32_t)(j0 + 32 * w + q),
+                                   (((bits >> q) & 1u) != 0u && ps < m) ? 1u : 0u);
+                }
+                pos = min(m, base + __popc(bits));
               }
             }
             flush_rows(hist, quad, lane, out, pos, flushed, 64);
