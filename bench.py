@@ -332,7 +332,8 @@ def run_ours(args, world, rank):
                                f"seed {cfg.seed}",
                    "global_batch": world * cfg.batch, "seq_len": cfg.T, "parallelism": f"dp{world} (one sequence per GPU)",
                    "l2": "inputs larger than L2 (q+gate+out 3.2 GB per step), no flush"},
-        "gpu_launches": 3 * args.steps,
+        # per step: compress, select, the plan (signature + 3 radix passes of 3 kernels), attend
+        "gpu_launches": 13 * args.steps,
         "e2e": {"value": tokens_step / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "roofline": roof,
@@ -353,6 +354,8 @@ def run_ours(args, world, rank):
     torch.cuda.empty_cache()
     if not args.no_decode:
         result["decode"] = run_decode(args, world, s)
+    if not args.no_swa:
+        result["swa"] = run_swa(args, world, s)
     if cpu_in is not None:
         result["cpu_baseline"] = cpu_baseline(cfg, *cpu_in)
     return result
@@ -416,6 +419,59 @@ def run_decode(args, world, s):
     return res
 
 
+SWA_WINDOW = 4096  # the pages give no window size for Gated SWA; this one matches the sparse budget
+
+
+def run_swa(args, world, s):
+    """Gated SWA (the efficient layer that alternates 3:1 with Sparse GQA) on the 128K prefill
+    inputs: keys t - window < u <= t, through sgqa_gated_swa, inputs resident in HBM."""
+    import torch
+    import block_sparse_long_kbar_b200 as sg
+    from sgqa_inputs import gen_device
+    base = CONFIGS["128k"]
+    cfg = base.replace(k=((SWA_WINDOW + 2 * base.B - 1) // base.B) * base.B)  # selection capacity
+    dims = sg.sgqa_dims.of(cfg)
+    dev = {}
+    for n in ("q", "k", "v", "gate"):
+        dev[n] = torch.empty(cfg.shape(n), dtype=torch.bfloat16, device="cuda")
+        gen_device(cfg, n, dev[n])
+    out = torch.empty(cfg.shape("q"), dtype=torch.bfloat16, device="cuda")
+    sel = torch.empty((cfg.batch, cfg.T, cfg.G, cfg.Kb), dtype=torch.int32, device="cuda")
+    ws = sg.alloc_workspace(sg.sgqa_workspace_size(dims))
+    sg.sgqa_reset_device_status(ws)
+    torch.cuda.synchronize()
+
+    def step():
+        sg.sgqa_gated_swa(dims, SWA_WINDOW, dev["q"], dev["k"], dev["v"], dev["gate"], out, ws, sel_out=sel, stream=s)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(args.steps):
+        step()
+    e1.record(s)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    assert sg.sgqa_get_device_status(ws) == 0
+    visits = cfg.batch * cfg.G * sum(min(t + 1, SWA_WINDOW) for t in range(cfg.T))  # (query, group, key)
+    flops = visits * cfg.R * 4 * cfg.d
+    peak = load_peaks()["bf16_tflops_sustained"]
+    res = {"metric": "Gated SWA prefill tokens/s at 128K (window 4096)",
+           "value": world * cfg.batch * cfg.T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+           "steps": args.steps,
+           "workload": f"gated swa 128k: batch {cfg.batch} per GPU, T={cfg.T}, Hq={cfg.Hq}, G={cfg.G}, d={cfg.d}, "
+                       f"B={cfg.B}, window {SWA_WINDOW}, seed {cfg.seed} (the 128K prefill inputs)",
+           "roofline": {"bound": "tensor", "achieved": flops / (ms / 1e3) / 1e12, "peak": peak, "unit": "TFLOP/s",
+                        "frac": flops / (ms / 1e3) / 1e12 / peak},
+           "gpu_launches_per_step": 12}  # window selection, plan (10), attend
+    del dev, out, sel, ws
+    torch.cuda.empty_cache()
+    return res
+
+
 CPU_STRIDE = 64
 
 
@@ -472,6 +528,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="128k", choices=["tiny", "32k", "128k", "64k_b8", "64k_b1"])
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-swa", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

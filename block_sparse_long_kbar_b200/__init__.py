@@ -26,7 +26,7 @@ STATUS_NAMES = {0: "SGQA_OK", 1: "SGQA_ERR_INVALID_ARG", 2: "SGQA_ERR_UNSUPPORTE
 # every symbol include/sgqa.h declares
 EXPORTS = ["sgqa_status_string", "sgqa_version", "sgqa_workspace_size", "sgqa_decode_workspace_size",
            "sgqa_reset_device_status", "sgqa_get_device_status", "sgqa_compress_keys", "sgqa_select",
-           "sgqa_attend", "sgqa_forward", "sgqa_decode", "sgqa_decode_noalloc"]
+           "sgqa_attend", "sgqa_forward", "sgqa_decode", "sgqa_decode_noalloc", "sgqa_gated_swa"]
 
 
 class SgqaError(RuntimeError):
@@ -73,8 +73,9 @@ def load_library():
     L.sgqa_forward.argtypes = [D, P, P, P, P, P, P, P, P, P, S, P]
     L.sgqa_decode.argtypes = [D, I, I] + [P] * 13 + [S, P]
     L.sgqa_decode_noalloc.argtypes = [D, I, I] + [P] * 12 + [P]
+    L.sgqa_gated_swa.argtypes = [D, I, P, P, P, P, P, P, P, S, P]
     for n in ("sgqa_reset_device_status", "sgqa_get_device_status", "sgqa_compress_keys", "sgqa_select",
-              "sgqa_attend", "sgqa_forward", "sgqa_decode", "sgqa_decode_noalloc"):
+              "sgqa_attend", "sgqa_forward", "sgqa_decode", "sgqa_decode_noalloc", "sgqa_gated_swa"):
         getattr(L, n).restype = I
     _lib = L
     return L
@@ -156,6 +157,12 @@ def sgqa_attend(dims, q, k, v, gate, sel, out, ws, stream=None):
     _check("sgqa_attend", load_library().sgqa_attend(
         ctypes.byref(dims), _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _ptr(gate, "gate"), _ptr(sel, "sel"),
         _ptr(out, "out"), _ptr(ws, "ws"), ws.numel(), _stream(stream)))
+
+
+def sgqa_gated_swa(dims, window, q, k, v, gate, out, ws, sel_out=None, stream=None):
+    _check("sgqa_gated_swa", load_library().sgqa_gated_swa(
+        ctypes.byref(dims), int(window), _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _ptr(gate, "gate"),
+        _ptr(out, "out"), _ptr(sel_out, "sel_out"), _ptr(ws, "ws"), ws.numel(), _stream(stream)))
 
 
 def sgqa_forward(dims, q, k, v, q_idx, k_idx, gate, out, ws, sel_out=None, stream=None):

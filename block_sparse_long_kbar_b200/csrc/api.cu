@@ -237,6 +237,36 @@ int sgqa_forward(const sgqa_dims* dims, const uint16_t* q, const uint16_t* k, co
   return SGQA_OK;
 }
 
+int sgqa_gated_swa(const sgqa_dims* dims, int window, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                   const uint16_t* gate, uint16_t* out, int32_t* sel_out, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (window < dims->B || (long)dims->k < (long)window + dims->B) return SGQA_ERR_INVALID_ARG;
+  if (!attend_tc_supported(dims->Hq, dims->G, dims->B, dims->d)) return SGQA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gate) || !aligned16(out) ||
+      (sel_out && !aligned16(sel_out)))
+    return SGQA_ERR_INVALID_ARG;
+  const PrefillWs w = prefill_layout(dims, ws);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < w.bytes) return SGQA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  AttendArgs aa = prefill_attend_args(dims, q, k, v, gate, out, w.status);
+  aa.window = window;
+  const int Kb = dims->k / dims->B;
+  const int chunk = sel_out ? dims->T : (dims->T < kSelChunkT ? dims->T : kSelChunkT);
+  for (int t0 = 0; t0 < dims->T; t0 += chunk) {
+    const int t1 = t0 + chunk < dims->T ? t0 + chunk : dims->T;
+    aa.sel = sel_out ? sel_out : w.sel;
+    aa.sel_T = sel_out ? dims->T : chunk;
+    aa.sel_t0 = sel_out ? 0 : t0;
+    aa.t_begin = t0; aa.t_end = t1;
+    if (launch_window_select(const_cast<int32_t*>(aa.sel), aa.sel_T, aa.sel_t0, dims->batch, dims->G, Kb, dims->B,
+                             window, t0, t1, s) != cudaSuccess)
+      return SGQA_ERR_CUDA;
+    if (launch_prefill_attend(aa, w.plan, s) != cudaSuccess) return SGQA_ERR_CUDA;
+  }
+  return SGQA_OK;
+}
+
 int sgqa_decode(const sgqa_dims* dims, int cache_len, int n_new, uint16_t* k_cache, uint16_t* v_cache,
                 uint16_t* kidx_cache, float* kbar_cache, const uint16_t* q_new, const uint16_t* k_new,
                 const uint16_t* v_new, const uint16_t* qidx_new, const uint16_t* kidx_new, const uint16_t* gate_new,

@@ -230,6 +230,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   const int r = quad * 32 + lane;
   const int q_r = r / R, h_r = r % R;
   const int t_r = is_sm ? sh->t[q_r] : -1;
+  // lowest key position the row may attend to (Gated SWA); -1 (below every key) without a window,
+  // so that lo_r - u0 cannot overflow
+  const int lo_r = (a.window > 0 && t_r >= 0) ? t_r - a.window + 1 : -1;
   const float sc = kLog2e / sqrtf((float)D);
   const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
 
@@ -454,8 +457,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             const int u0 = sbid * kUnit;
             const bool live = sbid >= 0 && t_r >= 0;
             uint32_t pk[8];
-            if (main_pass && lb >= 3 && live && u0 + (kUnit - 1) <= t_r) {
-              // blocks of 8 or 16 tokens wholly before the row's token: the selection bit of each
+            if (main_pass && lb >= 3 && live && u0 + (kUnit - 1) <= t_r && u0 >= lo_r) {
+              // blocks of 8 or 16 tokens wholly before the row's token (and inside its window, if
+              // any): the selection bit of each
               // half superblock becomes the additive term of the exponent (-inf when unselected,
               // whose exp2 is an exact 0); no per-token mask
               const int jb = (u0 >> lb) - w0;
@@ -477,6 +481,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 }
                 const int lim = t_r - u0;
                 if (lim < 15) vmask &= lim < 0 ? 0u : ((2u << lim) - 1u);
+                const int below = lo_r - u0;  // tokens of this superblock before the window
+                if (below > 0) vmask &= below >= kUnit ? 0u : ~((1u << below) - 1u);
               }
               if (!main_pass) {
 #pragma unroll

@@ -46,6 +46,7 @@ struct AttendArgs {
   int t_begin, t_end;
   int splits;
   int* status;
+  int window;  // > 0: only keys u > t - window count (Gated SWA); 0: no lower bound (tcgen05 path only)
 };
 cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s);
 cudaError_t launch_attend_merge(const AttendArgs& a, cudaStream_t s);
@@ -59,6 +60,10 @@ cudaError_t launch_plan(const int32_t* sel, int sel_T, int sel_t0, int batch, in
                         int t_end, void* ws, const uint32_t** perm_out, cudaStream_t s);
 // K3 tiled: tiles of consecutive rows of perm, union of their selections (requires ascending rows).
 bool attend_tiles_supported(int Hq, int G, int B);
+// Gated SWA: the selection of the blocks a window of `window` tokens ending at t overlaps
+// (ascending, -1 padded), rows [t_begin, t_end) into sel (row t at sel_T offset t - sel_t0).
+cudaError_t launch_window_select(int32_t* sel, int sel_T, int sel_t0, int batch, int G, int Kb, int B, int window,
+                                 int t_begin, int t_end, cudaStream_t s);
 cudaError_t launch_attend_tiles(const AttendArgs& a, const uint32_t* perm, cudaStream_t s);
 
 // K3 on tcgen05 (R in {4, 8, 16}): same contract as launch_attend_tiles.

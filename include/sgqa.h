@@ -139,6 +139,26 @@ int sgqa_decode(const sgqa_dims* dims, int cache_len, int n_new, uint16_t* k_cac
                 const uint16_t* kidx_new, const uint16_t* gate_new, uint16_t* out,
                 int32_t* sel_out, void* ws, size_t ws_bytes, void* stream);
 
+/* Gated SWA: the efficient attention layer that alternates 3:1 with the Sparse GQA layer
+ * (mo.ai.kr, "Step 5 Preview agentic work design", section "model structure and training
+ * stability"; ai.info, "StepFun illustrates the 92-block architecture of Step 5 Preview", section
+ * "Why StepFun chose 92 transformer blocks"). The pages name the layer but give no window size;
+ * it is the `window` argument here. For each (b, t) and head h of group g:
+ *     U = {u : t - window < u <= t};  o = softmax_U(q[b,t,h] . k[b,u,g] / sqrt(d)) v;
+ *     out[b,t,h,:] = o * sigmoid(gate_logits[b,t,h,:])                  (bf16 RNE)
+ * i.e. the steps (3) and (4) above with a sliding window of keys in place of the selection.
+ * q, k, v, gate, out as above; no index keys. The blocks the window overlaps are written as a
+ * selection (ascending block ids, -1 padded) to sel_out [batch, T, G, k/B] if not NULL, else into
+ * ws in chunks, and the tiled attention masks the tokens before the window.
+ *   - dims->k is the selection row capacity in tokens: it must hold every block a window can
+ *     overlap, so window >= B and dims->k >= window + B are required (else SGQA_ERR_INVALID_ARG).
+ *   - Runs on the tcgen05 attention only: Hq/G in {4, 8, 16}, d in {64, 128}, B <= 16 (else
+ *     SGQA_ERR_UNSUPPORTED).
+ *   - ws as for sgqa_attend (sgqa_workspace_size(dims)). */
+int sgqa_gated_swa(const sgqa_dims* dims, int window, const uint16_t* q, const uint16_t* k,
+                   const uint16_t* v, const uint16_t* gate, uint16_t* out, int32_t* sel_out,
+                   void* ws, size_t ws_bytes, void* stream);
+
 /* Size of the library-owned scratch array that sgqa_decode_noalloc uses (16 MiB). */
 #define SGQA_NOALLOC_SCRATCH_BYTES (16u << 20)
 

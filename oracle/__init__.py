@@ -9,7 +9,9 @@ section "model structure and training stability", and ai.info "StepFun illustrat
 architecture of Step 5 Preview", section "Sparse GQA aims at a 1 million token context"):
 block-mean index keys (B tokens per block), per-KV-group top-(k/B) block selection that always
 keeps the query's own block, causal softmax attention of every head of the group over the
-selected tokens scaled by 1/sqrt(d), and an elementwise sigmoid output gate.
+selected tokens scaled by 1/sqrt(d), and an elementwise sigmoid output gate. Also the Gated SWA
+layer that alternates 3:1 with it (same section): the gated attention over a sliding window of
+keys, the window size being a parameter (the pages give none).
 
 Parity pins: every function here is pinned by tests/test_oracle_pins.py (brute force on
 T <= 64, dense reduction against torch's SDPA in fp64, closed forms and invariants).
@@ -51,8 +53,9 @@ def load(path: str):
     L.oracle_attend.argtypes = [ctypes.POINTER(Dims), ctypes.c_int, P, P, P, P, P, P, P, ctypes.c_int]
     L.oracle_coverage.argtypes = [ctypes.POINTER(Dims), ctypes.c_int, P, P, P, P, ctypes.c_int, P,
                                   ctypes.c_int]
+    L.oracle_swa.argtypes = [ctypes.POINTER(Dims), ctypes.c_int, P, P, P, P, P, ctypes.c_int, P, ctypes.c_int]
     for f in (L.oracle_compress, L.oracle_scores, L.oracle_select, L.oracle_attend, L.oracle_coverage,
-              L.oracle_max_threads):
+              L.oracle_swa, L.oracle_max_threads):
         f.restype = ctypes.c_int
     return L
 
@@ -148,6 +151,21 @@ def attend(dm: Dims, rows_bt, q_rows, k, v, gate_rows, sel, n_threads: int = 0) 
                              _p(out), n_threads)
     if rc != 0:
         raise ValueError(f"oracle_attend: {rc}")
+    return out
+
+
+def swa(dm: Dims, rows_bt, q_rows, k, v, gate_rows, window: int, n_threads: int = 0) -> np.ndarray:
+    """Gated SWA: out [n, Hq, d] fp64 for query rows (b, t) over the keys t - window < u <= t."""
+    rows = _rows(rows_bt)
+    n = rows.shape[0]
+    q_rows, gate_rows, k, v = _u16(q_rows), _u16(gate_rows), _u16(k), _u16(v)
+    assert q_rows.size == n * dm.Hq * dm.d and gate_rows.size == q_rows.size
+    assert k.size == dm.batch * dm.T * dm.G * dm.d and v.size == k.size
+    out = np.zeros((n, dm.Hq, dm.d), dtype=np.float64)
+    rc = lib().oracle_swa(ctypes.byref(dm), n, _p(rows), _p(q_rows), _p(k), _p(v), _p(gate_rows), int(window),
+                          _p(out), n_threads)
+    if rc != 0:
+        raise ValueError(f"oracle_swa: {rc}")
     return out
 
 

@@ -209,6 +209,50 @@ int oracle_attend(const Dims* dm, int n_rows, const int32_t* rows_bt, const uint
   return bad ? -3 : 0;
 }
 
+// Gated SWA, the efficient layer that alternates 3:1 with the full-context layer (mo.ai.kr,
+// "Step 5 Preview agentic work design", section "model structure and training stability"): the
+// same gated softmax attention over the keys of a sliding window, U = {u : t - window < u <= t}.
+// The pages give no window size; it is a parameter. Shapes as for oracle_attend; out [n_rows,
+// Hq, d] fp64. Returns -1 for window < 1.
+int oracle_swa(const Dims* dm, int n_rows, const int32_t* rows_bt, const uint16_t* q, const uint16_t* k,
+               const uint16_t* v, const uint16_t* gate, int window, double* out, int n_threads) {
+  if (!dims_ok(dm) || window < 1) return -1;
+  set_threads(n_threads);
+  const int R = dm->Hq / dm->G, d = dm->d;
+  const double inv_sqrt_d = 1.0 / std::sqrt((double)d);
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long rh = 0; rh < (long)n_rows * dm->Hq; ++rh) {
+    const long row = rh / dm->Hq;
+    const int h = (int)(rh % dm->Hq), g = h / R;
+    const long b = rows_bt[2 * row];
+    const int t = rows_bt[2 * row + 1];
+    const int u_lo = std::max(0, t - window + 1);
+    const uint16_t* qv = q + rh * d;
+    std::vector<double> z(t - u_lo + 1);
+    double zmax = -INFINITY;
+    for (int u = u_lo; u <= t; ++u) {
+      const uint16_t* kv = k + ((b * dm->T + u) * dm->G + g) * d;
+      double dot = 0.0;
+      for (int e = 0; e < d; ++e) dot += bf16_to_f64(qv[e]) * bf16_to_f64(kv[e]);
+      z[u - u_lo] = dot * inv_sqrt_d;
+      zmax = std::max(zmax, z[u - u_lo]);
+    }
+    std::vector<double> o(d, 0.0);
+    double l = 0.0;
+    for (int u = u_lo; u <= t; ++u) {
+      const double p = std::exp(z[u - u_lo] - zmax);
+      l += p;
+      const uint16_t* vv = v + ((b * dm->T + u) * dm->G + g) * d;
+      for (int e = 0; e < d; ++e) o[e] += p * bf16_to_f64(vv[e]);
+    }
+    for (int e = 0; e < d; ++e) {
+      const double gl = bf16_to_f64(gate[rh * d + e]);
+      out[rh * d + e] = (o[e] / l) * (1.0 / (1.0 + std::exp(-gl)));
+    }
+  }
+  return 0;
+}
+
 // Token coverage of a selection (the ablation's quality metric): for each (row, head), the
 // fraction of the top-`ktop` tokens u <= t by exact q[t,h] . k[u,g] (ties to the lower u)
 // that lie in the selected token set U(t, g). cov: [n_rows, Hq].

@@ -106,6 +106,16 @@ def test_host_validation_codes(lib):
     assert lib.sgqa_decode(ctypes.byref(D(T=64)), 0, 0, *args, P(good), 1 << 30, None) == 1
     assert lib.sgqa_decode(ctypes.byref(D(T=64, G=16, Hq=16)), 0, 4, *args, P(good), 1 << 30, None) == 1
     assert lib.sgqa_decode(ctypes.byref(D(T=64)), 0, 4, *args, P(good), 1024, None) == 3
+    # Gated SWA: window below one block, selection capacity below window + B, heads per group
+    # outside the tcgen05 attention, workspace too small
+    swa = lambda dims, w, ws_bytes: lib.sgqa_gated_swa(ctypes.byref(dims), w, *[P(good)] * 5, None, P(good),
+                                                       ws_bytes, None)
+    ds = D(k=512)
+    ws_swa = sg.sgqa_workspace_size(ds)
+    assert swa(ds, ds.B - 1, ws_swa) == 1
+    assert swa(ds, ds.k - ds.B + 1, ws_swa) == 1
+    assert swa(D(k=512, Hq=8, G=8), 64, sg.sgqa_workspace_size(D(k=512, Hq=8, G=8))) == 2
+    assert swa(ds, 64, ws_swa - 1) == 3
     v = ctypes.c_int(0)
     assert lib.sgqa_get_device_status(None, 256, ctypes.byref(v)) == 1
     assert lib.sgqa_reset_device_status(None, 256, None) == 3
