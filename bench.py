@@ -38,13 +38,13 @@ CLOCK_FIELDS = ["pci.bus_id", "clocks.sm", "clocks.max.sm", "power.draw", "clock
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the current kernels,
 # from the ncu captures summarised in profiles/select_tc_attend_tc_32k.md: the attend kernel moved
-# 2.291 GB on the 32K workload (65536 query tokens), exactly its compulsory bytes, which are all
+# 2.293 GB on the 32K workload (65536 query tokens), exactly its compulsory bytes, which are all
 # per query token; the 128K entry is that capture scaled by the 131072 query tokens of a launch.
 # An entry must be dropped (None) when its kernel changes.
 NCU_TRAFFIC = {
-    ("attend", "32k"): 2.2912e9,
-    ("attend", "128k"): 2.2912e9 * 131072 / 65536,
-    ("select", "32k"): 0.5178e9,
+    ("attend", "32k"): 2.2932e9,
+    ("attend", "128k"): 2.2932e9 * 131072 / 65536,
+    ("select", "32k"): 0.5187e9,
 }
 
 
