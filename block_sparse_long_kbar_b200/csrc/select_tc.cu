@@ -15,15 +15,22 @@
 // fp32; splitting it into bf16 hi + lo planes keeps the product exact to ~2^-17 relative, and
 // q_idx is exactly bf16, so the contraction runs at the bf16 tensor rate.
 //
-// Warp roles: warp 4 issues TMA loads, warp 5 allocates TMEM and issues MMAs, warps 0-3 own one
-// row each per thread (TMEM lane = row). The epilogue performs an exact radix select of the
-// m-th largest order-preserving 32-bit score key per row: every pass re-streams the same score
-// tiles (recomputed, bit-identical) and fills the row's 256-bin shared histogram of the next 8
-// key bits among keys that still match the resolved prefix; once every row's threshold bucket
-// is resolved (or taken whole), a final pass streams the candidates in ascending j and emits
-// keys above the threshold plus the first ties at it, so ties go to the lower block index and
-// the output is ascending without a sort. The epilogue tells the producer and MMA warps at the
-// start of each pass whether another pass follows, so they run up to one pass ahead.
+// Warp roles: warp 8 issues TMA loads, warp 9 allocates TMEM and issues MMAs, warps 0-7 are the
+// epilogue, two per TMEM lane quadrant (TMEM lane = row). The epilogue performs an exact radix
+// select of the m-th largest order-preserving 32-bit score key per row: every pass re-streams the
+// same score tiles (recomputed, bit-identical); in a histogram pass the two threads of a row take
+// half of every tile's columns each and add 0 or 1 per key to the row's 256-bin shared histogram
+// of the next 8 key bits (1 for keys that still match the resolved prefix; branch-free). Once
+// every row's threshold bucket is resolved or taken whole, the emit pass streams the candidates
+// in ascending j: keys above the threshold are taken, bucket keys are taken in j order up to the
+// remaining count (so ties go to the lower block index and the output is ascending without a
+// sort). From the third pass on, if every unresolved row's bucket holds at most kCap keys, the
+// emit pass comes early: it also collects those keys with the number of keys taken before each,
+// resolves them exactly afterwards and places the chosen ones by moving blocks of the row. The
+// emit marks taken candidates in bit masks (ALU only), stages the indices in a 128-entry shared
+// ring per row at positions from population counts, and the warp writes each row out 64 indices
+// at a time as whole lines. The epilogue tells the producer and MMA warps at the start of each
+// pass whether another pass follows, so they run up to one pass ahead.
 //
 // Every wait is bounded (globaltimer): on timeout the kernel records SGQA_ERR_TIMEOUT, stops all
 // roles, waits (bounded) for its own copies and MMAs in flight, frees TMEM and returns.

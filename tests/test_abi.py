@@ -29,7 +29,8 @@ def declared_symbols():
 
 def test_header_declares_expected_api():
     syms = declared_symbols()
-    for name in ("sgqa_compress_keys", "sgqa_select", "sgqa_attend", "sgqa_forward", "sgqa_decode"):
+    for name in ("sgqa_compress_keys", "sgqa_select", "sgqa_attend", "sgqa_forward", "sgqa_decode",
+                 "sgqa_gated_swa"):
         assert name in syms
     assert sorted(sg.EXPORTS) == syms
 
