@@ -351,6 +351,13 @@ def test_full_size_prefill_sampled(name):
     print(f"{name}: near-tie rows {n_tie}; max-abs/mean-abs/rel-rms {err}")
 
 
+def test_largest_budget_sampled():
+    """The largest supported budget, k/B = 16384 blocks (B = 1, so up to 16383 picks per row):
+    selections far longer than a tile, nearly every candidate taken in the early rows."""
+    n_tie, err = _full_size_forward(Config("max_budget", 1, 17000, 8, 2, 64, 32, 1, 16384, 1000, 21), 40, 7)
+    print(f"max budget: near-tie rows {n_tie}; max-abs/mean-abs/rel-rms {err}")
+
+
 def test_full_size_decode_1m_sampled():
     cfg = CONFIGS["decode_1m"]
     errs = _decode_case(cfg, cfg.T, DECODE_NEW, [0, 31])
