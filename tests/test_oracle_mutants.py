@@ -4,7 +4,9 @@ oracle (on the CPU), rebuild it, and check that at least one pin in test_oracle_
 Each mutation is a mistake someone writing the Sparse GQA definition could make: a reversed
 tie rule, the own block not counted in the budget, a lost causal limit, the wrong softmax
 scale, a flipped gate sign, an off-by-one in the candidate range, a dropped term in the block
-mean, an interleaved head->group mapping, or the wrong group's index query.
+mean, an interleaved head->group mapping, or the wrong group's index query; and in the Gated
+SWA definition, a window one key too long or too short, unscaled scores, a missing gate or an
+interleaved head->group mapping (these are checked against the SWA pins).
 """
 import os
 import subprocess
@@ -42,9 +44,34 @@ PIN_CALLS = [
 ]
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
+# Gated SWA: a window one key too long or too short, no softmax scale, no gate, the wrong group
+SWA_MUTANTS = {
+    "swa_window_one_longer": ("const int u_lo = std::max(0, t - window + 1);",
+                              "const int u_lo = std::max(0, t - window);"),
+    "swa_window_one_shorter": ("const int u_lo = std::max(0, t - window + 1);",
+                               "const int u_lo = std::max(0, t - window + 2);"),
+    "swa_unscaled_scores": ("z[u - u_lo] = dot * inv_sqrt_d;", "z[u - u_lo] = dot;"),
+    "swa_no_gate": ("out[rh * d + e] = (o[e] / l) * (1.0 / (1.0 + std::exp(-gl)));", "out[rh * d + e] = (o[e] / l);"),
+    "swa_interleaved_heads": ("const int h = (int)(rh % dm->Hq), g = h / R;\n    const long b = rows_bt[2 * row];\n    const int t = rows_bt[2 * row + 1];\n    const int u_lo",
+                              "const int h = (int)(rh % dm->Hq), g = h % dm->G;\n    const long b = rows_bt[2 * row];\n    const int t = rows_bt[2 * row + 1];\n    const int u_lo"),
+}
+
+
+def _swa_pin_calls():
+    import tests.test_oracle_swa_pins as swa
+    return [
+        lambda: swa.test_swa_brute_force(None, 40, 8, 13),
+        lambda: swa.test_swa_brute_force(None, 33, 1, 5),
+        lambda: swa.test_swa_full_window_is_dense_causal(None, 70, 8, 2, 16),
+        lambda: swa.test_swa_block_aligned_window_equals_block_selection(None),
+        lambda: swa.test_swa_locality(None),
+    ]
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS) + sorted(SWA_MUTANTS))
 def test_pins_catch_mutant(tmp_path, name):
-    old, new = MUTANTS[name]
+    old, new = MUTANTS[name] if name in MUTANTS else SWA_MUTANTS[name]
+    calls = PIN_CALLS if name in MUTANTS else _swa_pin_calls()
     src = open(oracle.SRC).read()
     assert src.count(old) >= 1, f"mutation anchor not found: {name}"
     mutated = src.replace(old, new)
@@ -57,7 +84,7 @@ def test_pins_catch_mutant(tmp_path, name):
     oracle._lib = oracle.load(str(so))
     caught = []
     try:
-        for call in PIN_CALLS:
+        for call in calls:
             try:
                 call()
             except (AssertionError, ValueError) as e:
