@@ -21,6 +21,8 @@ int check_dims(const sgqa_dims* d) {
       d->k <= 0)
     return SGQA_ERR_INVALID_ARG;
   if (d->T >= (1 << 28) || d->batch > 65535) return SGQA_ERR_UNSUPPORTED;
+  // row indices of q, gate, out and q_idx (and TMA coordinates) are 32-bit
+  if ((long)d->batch * d->T * (d->Hq > d->G ? d->Hq : d->G) >= (1L << 31)) return SGQA_ERR_UNSUPPORTED;
   if (d->d != 64 && d->d != 128) return SGQA_ERR_UNSUPPORTED;
   if (d->d_idx != 32 && d->d_idx != 64) return SGQA_ERR_UNSUPPORTED;
   if (d->B != 1 && d->B != 2 && d->B != 4 && d->B != 8 && d->B != 16) return SGQA_ERR_UNSUPPORTED;

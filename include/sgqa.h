@@ -36,7 +36,7 @@
  *     synchronising the stream.
  *   - Supported shapes (else SGQA_ERR_UNSUPPORTED): d in {64, 128}; d_idx in {32, 64};
  *     B in {1, 2, 4, 8, 16}; k % B == 0; Hq % G == 0 with 1 <= Hq/G <= 16; 128 % G == 0;
- *     1 <= T < 2^28. A trailing partial block is never a candidate.
+ *     1 <= T < 2^28; batch * T * Hq < 2^31. A trailing partial block is never a candidate.
  *   - Results are deterministic: the same inputs give the same bits, run after run.
  */
 #ifndef SGQA_H

@@ -93,6 +93,7 @@ def test_host_validation_codes(lib):
     need = sg.sgqa_workspace_size(d)
     assert _call_forward(lib, D(d=96), good, good, need) == 2          # unsupported
     assert _call_forward(lib, D(T=0), good, good, need) == 1           # invalid
+    assert _call_forward(lib, D(batch=64, T=(1 << 27) - 8, Hq=32, G=4), good, good, need) == 2  # 2^31 rows
     assert _call_forward(lib, d, good + 8, good, need) == 1            # misaligned tensor
     assert _call_forward(lib, d, 0, good, need) == 1                   # null tensor
     assert _call_forward(lib, d, good, good, need - 1) == 3            # workspace too small
