@@ -33,6 +33,7 @@ SMALL = {
     "t9": Config("t9", 3, 9, 8, 2, 64, 32, 8, 16, 4, 12),
     "t1": Config("t1", 2, 1, 4, 4, 128, 64, 8, 64, 4, 13),
     "r3_rowkernel": Config("r3_rowkernel", 1, 1200, 12, 4, 64, 32, 8, 256, 150, 19),
+    "g4_r2": Config("g4_r2", 1, 1300, 8, 4, 64, 32, 8, 256, 150, 23),
 }
 
 
