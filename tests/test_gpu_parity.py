@@ -17,7 +17,7 @@ torch = pytest.importorskip("torch")
 import oracle
 import block_sparse_long_kbar_b200 as sg
 import sgqa_inputs as sgi
-from sgqa_inputs import CONFIGS, DECODE_NEW, Config, gen_device, gen_rows
+from sgqa_inputs import CONFIGS, DECODE_NEW, Config, gen_device, gen_full, gen_rows
 from tests._helpers import (NAMES, all_rows, assert_outputs_close, compare_selection, device_inputs, host_inputs,
                             output_errors, sample_rows, shape_of, to_dev, to_host)
 
@@ -195,6 +195,32 @@ def test_forward_chunked_selection_is_identical():
     sg.sgqa_forward(dims, d["q"], d["k"], d["v"], d["q_idx"], d["k_idx"], d["gate"], out2, ws)
     _status_ok(ws)
     assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+
+
+def test_exact_ties_go_to_lower_blocks():
+    """All index keys equal, so every candidate block has exactly the same score: the selection
+    must be the lowest m = min(k/B - 1, c) blocks plus the own block (ties to the lower index)."""
+    cfg = Config("ties", 2, 1500, 8, 2, 64, 32, 8, 256, 100, 24)
+    dims = sg.sgqa_dims.of(cfg)
+    one = gen_rows(cfg, "k_idx", 0, np.array([5]))[0]
+    k_idx = np.broadcast_to(one, (cfg.batch, cfg.T, cfg.d_idx)).copy()
+    q_idx = to_dev(gen_full(cfg, "q_idx").reshape(shape_of(cfg, "q_idx")), shape_of(cfg, "q_idx"))
+    kbar = torch.empty((cfg.batch, cfg.T // cfg.B, cfg.d_idx), device="cuda")
+    sg.sgqa_compress_keys(dims, to_dev(k_idx, shape_of(cfg, "k_idx")), kbar, None)
+    ws = _ws(dims)
+    sel = torch.full((cfg.batch, cfg.T, cfg.G, cfg.Kb), -7, dtype=torch.int32, device="cuda")
+    sg.sgqa_select(dims, q_idx, kbar, sel, ws)
+    _status_ok(ws)
+    got = sel.cpu().numpy()
+    want = np.full((cfg.T, cfg.Kb), -1, dtype=np.int32)
+    for t in range(cfg.T):
+        c = t // cfg.B
+        m = min(cfg.Kb - 1, c)
+        want[t, :m] = np.arange(m)
+        want[t, m] = c
+    for b in range(cfg.batch):
+        for g in range(cfg.G):
+            np.testing.assert_array_equal(got[b, :, g], want)
 
 
 def test_causality_on_gpu():
