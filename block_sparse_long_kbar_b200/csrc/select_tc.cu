@@ -100,7 +100,7 @@ __device__ __forceinline__ int epi_vote_any(SelShared* sh, int slot, bool v) {
   return __shfl_sync(0xFFFFFFFFu, res, 0);
 }
 
-// Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast to the warp.
+// Warp-uniform bounded wait: lane 0 polls, the outcome is broadcast to the warp.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   int ok = 1;
   if ((threadIdx.x & 31) == 0) ok = tc::mbar_wait(bar, parity, abort) ? 1 : 0;

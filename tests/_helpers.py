@@ -8,7 +8,7 @@ import oracle
 from sgqa_inputs import Config, gen_device, gen_full, bf16_bits_to_f64
 
 NAMES = ("q", "k", "v", "gate", "q_idx", "k_idx")
-# the benchmark spec tolerances for bf16 inputs, outputs computed with the oracle's selection replayed
+# output tolerances for bf16 inputs, outputs computed with the oracle's selection replayed
 MAX_ABS = 1e-2
 MEAN_ABS = 1e-3
 NEAR_TIE_REL = 1e-4
