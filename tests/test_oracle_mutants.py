@@ -6,7 +6,10 @@ tie rule, the own block not counted in the budget, a lost causal limit, the wron
 scale, a flipped gate sign, an off-by-one in the candidate range, a dropped term in the block
 mean, an interleaved head->group mapping, or the wrong group's index query; and in the Gated
 SWA definition, a window one key too long or too short, unscaled scores, a missing gate or an
-interleaved head->group mapping (these are checked against the SWA pins).
+interleaved head->group mapping (these are checked against the SWA pins); and in the token
+coverage of the ablation, a reversed ranking, an interleaved head->group mapping, ties sent to
+the higher token, a top set one token short, and the query's own token left out (these are
+checked against the coverage pins).
 """
 import os
 import subprocess
@@ -57,6 +60,36 @@ SWA_MUTANTS = {
 }
 
 
+# Token coverage: each mutation touches only oracle_coverage (its anchors occur nowhere else)
+COVERAGE_MUTANTS = {
+    "coverage_ascending_rank": (
+        "if (n < t + 1) std::nth_element(z.begin(), z.begin() + n, z.end(), ranks_before);",
+        "if (n < t + 1) std::nth_element(z.begin(), z.begin() + n, z.end(),\n"
+        "        [](const Cand& a, const Cand& b) { return a.s < b.s || (a.s == b.s && a.j < b.j); });"),
+    "coverage_interleaved_heads": (
+        "const int h = (int)(rh % dm->Hq), g = h / R;\n    const long b = rows_bt[2 * row];\n"
+        "    const int t = rows_bt[2 * row + 1];\n    std::vector<char> in_sel",
+        "const int h = (int)(rh % dm->Hq), g = h % dm->G;\n    const long b = rows_bt[2 * row];\n"
+        "    const int t = rows_bt[2 * row + 1];\n    std::vector<char> in_sel"),
+    "coverage_ties_to_higher_token": (
+        "if (n < t + 1) std::nth_element(z.begin(), z.begin() + n, z.end(), ranks_before);",
+        "if (n < t + 1) std::nth_element(z.begin(), z.begin() + n, z.end(),\n"
+        "        [](const Cand& a, const Cand& b) { return a.s > b.s || (a.s == b.s && a.j > b.j); });"),
+    "coverage_top_set_one_short": ("const int n = std::min(ktop, t + 1);", "const int n = std::min(ktop, t);"),
+    "coverage_own_token_left_out": ("std::vector<Cand> z(t + 1);\n    for (int u = 0; u <= t; ++u) {",
+                                    "std::vector<Cand> z(t + 1);\n    for (int u = 0; u < t; ++u) {"),
+}
+
+
+def _coverage_pin_calls():
+    return [
+        lambda: pins.test_coverage_brute_force(None, False),
+        lambda: pins.test_coverage_brute_force(None, True),
+        lambda: pins.test_coverage_all_scores_tied_takes_lowest_tokens(None),
+        lambda: pins.test_coverage_closed_forms(None),
+    ]
+
+
 def _swa_pin_calls():
     import tests.test_oracle_swa_pins as swa
     return [
@@ -68,12 +101,18 @@ def _swa_pin_calls():
     ]
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS) + sorted(SWA_MUTANTS))
+ALL_MUTANTS = {**MUTANTS, **SWA_MUTANTS, **COVERAGE_MUTANTS}
+
+
+@pytest.mark.parametrize("name", sorted(ALL_MUTANTS))
 def test_pins_catch_mutant(tmp_path, name):
-    old, new = MUTANTS[name] if name in MUTANTS else SWA_MUTANTS[name]
-    calls = PIN_CALLS if name in MUTANTS else _swa_pin_calls()
+    old, new = ALL_MUTANTS[name]
+    calls = (PIN_CALLS if name in MUTANTS else _swa_pin_calls() if name in SWA_MUTANTS
+             else _coverage_pin_calls())
     src = open(oracle.SRC).read()
     assert src.count(old) >= 1, f"mutation anchor not found: {name}"
+    if name in COVERAGE_MUTANTS:
+        assert src.count(old) == 1, f"coverage mutation anchor not unique: {name}"
     mutated = src.replace(old, new)
     cpp = tmp_path / "mut.cpp"
     so = tmp_path / "libmut.so"

@@ -310,3 +310,78 @@ def test_coverage_closed_forms(oracle_lib):
     cov2 = oracle.coverage(dm, rows, qr, x["k"], only_own, ktop=1000)
     want = np.array([((t % 4) + 1) / (t + 1) for t in rows[:, 1]])
     np.testing.assert_allclose(cov2[:, 0], want, rtol=1e-15)
+
+
+def _coverage_brute_force(cfg, q, k, rows, sel, ktop):
+    """Token coverage written out directly: every (row, head) sorts all tokens u <= t by
+    (exact score desc, u asc) with a Python sort, keeps the first min(ktop, t + 1), and counts
+    those whose block the row's group selected. Scores are sums of exact products taken with
+    math.fsum (correctly rounded), so they do not depend on a summation order."""
+    T, G, Hq, d, B = cfg.T, cfg.G, cfg.Hq, cfg.d, cfg.B
+    R, Kb = Hq // G, cfg.k // cfg.B
+    qf = _f(q).reshape(len(rows), Hq, d)
+    kf = _f(k).reshape(cfg.batch, T, G, d)
+    cov = np.zeros((len(rows), Hq))
+    for i, (b, t) in enumerate(rows):
+        for h in range(Hq):
+            g = h // R
+            S = {int(j) for j in sel[i, g] if j >= 0}
+            order = sorted(range(t + 1), key=lambda u: (-math.fsum(qf[i, h] * kf[b, u, g]), u))
+            top = order[:min(ktop, t + 1)]
+            cov[i, h] = sum(1 for u in top if u // B in S) / len(top)
+    return cov
+
+
+def _random_selection(cfg, rows, seed):
+    """A valid selection per (row, group) that is neither empty nor everything: the own block plus
+    a seeded random subset of the complete past blocks, at most k/B - 1 of them, ascending."""
+    rng = np.random.default_rng(seed)
+    Kb = cfg.k // cfg.B
+    sel = np.full((len(rows), cfg.G, Kb), -1, dtype=np.int32)
+    for i, (_, t) in enumerate(rows):
+        c = t // cfg.B
+        for g in range(cfg.G):
+            past = [j for j in range(c) if rng.random() < 0.5][:Kb - 1]
+            S = sorted(past + [c])
+            sel[i, g, :len(S)] = S
+    return sel
+
+
+@pytest.mark.parametrize("integer_valued", [False, True])
+def test_coverage_brute_force(oracle_lib, integer_valued):
+    """oracle_coverage against the brute force with ktop < t + 1 (the top set really has to be
+    chosen), two groups of two heads (so h // R and h % G differ), and a selection that covers
+    about half of every row. The integer-valued case has scores in [-72, 72] with many exact
+    ties at the ktop boundary, which only the (score desc, u asc) rule orders correctly."""
+    cfg, x = _rand_case(56, 4, 16, Hq=4, G=2, d=8, d_idx=4, seed=31)
+    q, k = x["q"], x["k"]
+    if integer_valued:
+        rng = np.random.default_rng(5)
+        q = f64_to_bf16_bits(rng.integers(-3, 4, size=q.shape).astype(np.float64))
+        k = f64_to_bf16_bits(rng.integers(-3, 4, size=k.shape).astype(np.float64))
+    rows = np.array([[0, t] for t in range(cfg.T)], dtype=np.int32)
+    sel = _random_selection(cfg, rows, seed=3)
+    dm = oracle.dims_of(cfg)
+    qr = np.ascontiguousarray(q.reshape(cfg.T, -1))
+    for ktop in (1, 5, 12):
+        got = oracle.coverage(dm, rows, qr, k, sel, ktop=ktop)
+        want = _coverage_brute_force(cfg, q, k, rows, sel, ktop)
+        np.testing.assert_array_equal(got, want)
+        assert 0.0 < got[ktop + 8:].mean() < 1.0
+
+
+def test_coverage_all_scores_tied_takes_lowest_tokens(oracle_lib):
+    """Every key equal, so every score ties: the top-ktop set is the ktop lowest tokens u < ktop
+    (ties to the lower index), and coverage is the closed form |{u < ktop : u // B in S}| / ktop."""
+    cfg, x = _rand_case(48, 4, 16, Hq=4, G=2, d=8, d_idx=4, seed=32)
+    k = np.broadcast_to(x["k"][:, :1], x["k"].shape).copy()
+    rows = np.array([[0, t] for t in range(cfg.T)], dtype=np.int32)
+    sel = _random_selection(cfg, rows, seed=4)
+    dm = oracle.dims_of(cfg)
+    ktop = 9
+    cov = oracle.coverage(dm, rows, np.ascontiguousarray(x["q"].reshape(cfg.T, -1)), k, sel, ktop=ktop)
+    for i, (_, t) in enumerate(rows):
+        n = min(ktop, t + 1)
+        for h in range(cfg.Hq):
+            S = {int(j) for j in sel[i, h // cfg.R] if j >= 0}
+            assert cov[i, h] == sum(1 for u in range(n) if u // cfg.B in S) / n
