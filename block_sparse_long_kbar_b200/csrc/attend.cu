@@ -63,11 +63,21 @@ __global__ void __launch_bounds__(kWarps * 32) attend_kernel(AttendArgs a) {
   if (tid == 0) s_nsel = 0;
   __syncthreads();
   int last = -1;
+  // the format: strictly ascending block ids in [0, c_own], then -1 padding. An entry out of
+  // range, not above the entry before it, or after the padding began is reported and skipped
+  // (each thread compares with the previous entry as stored, so no ordering between threads)
   for (int i = tid; i < a.Kb; i += kWarps * 32) {
     int j = __ldg(srow + i);
     if (j > c_own || j < -1) {
       report(a.status, SGQA_ERR_DEVICE_CHECK);
       j = -1;
+    }
+    if (j >= 0 && i > 0) {
+      const int p = __ldg(srow + i - 1);
+      if (p < 0 || p > c_own || j <= p) {
+        report(a.status, SGQA_ERR_DEVICE_CHECK);
+        j = -1;
+      }
     }
     s_sel[i] = j;
     if (j >= 0) last = i;

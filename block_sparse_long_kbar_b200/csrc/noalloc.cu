@@ -13,7 +13,9 @@
 // variable). The first call on each device therefore asks the runtime for the array's device
 // address with cudaGetSymbolAddress, with that device current, checks the result and caches it
 // per device; later calls reuse the cached address. Because the first call on a device does
-// that set-up, make it before any stream capture.
+// that set-up, make it before any stream capture. The cached address is only valid for the
+// context it was taken in: a device reset (cudaDeviceReset, or resetting the primary context)
+// unloads the module and frees the array, so calls after such a reset are not supported.
 //
 // Every call uses the same array and the array keeps the last call's contents. The call zeroes
 // the status word itself (asynchronously, on the caller's stream) and every other scratch byte

@@ -130,9 +130,13 @@ int sgqa_forward(const sgqa_dims* dims, const uint16_t* q, const uint16_t* k, co
  * [batch, n_new, G, d], qidx_new [batch, n_new, G, d_idx], kidx_new [batch, n_new, d_idx].
  * The step writes the new k, v, k_idx rows at positions [cache_len, cache_len + n_new), adds
  * kbar for the blocks they complete, and writes out [batch, n_new, Hq, d] (and, if not NULL,
- * sel_out [batch, n_new, G, k/B]) exactly as sgqa_forward would give for the last n_new rows of
- * the concatenated sequence. Requires cache_len + n_new <= T. Repeating a step at the same
- * cache_len rewrites the same rows, so it is idempotent. */
+ * sel_out [batch, n_new, G, k/B]) for the last n_new rows of the concatenated sequence: the same
+ * definition sgqa_forward computes for those rows, with the same selection rule, but not the same
+ * arithmetic. Decode scores the candidates on its own kernels, so where two candidate scores
+ * agree to within the rounding of the fp32 scores (a near-tie at the k/B-th place) decode and
+ * forward may keep different blocks; elsewhere the selections are identical and the outputs agree
+ * within the bf16 rounding. Requires cache_len + n_new <= T. Repeating a step at the same
+ * cache_len rewrites the same rows and gives the same bits, so it is idempotent. */
 int sgqa_decode(const sgqa_dims* dims, int cache_len, int n_new, uint16_t* k_cache,
                 uint16_t* v_cache, uint16_t* kidx_cache, float* kbar_cache, const uint16_t* q_new,
                 const uint16_t* k_new, const uint16_t* v_new, const uint16_t* qidx_new,
@@ -172,7 +176,10 @@ int sgqa_gated_swa(const sgqa_dims* dims, int window, const uint16_t* q, const u
  *     SGQA_NOALLOC_SCRATCH_BYTES (e.g. 32 sequences at a 1M-token cache need more; use sgqa_decode),
  *     SGQA_ERR_INVALID_ARG / SGQA_ERR_UNSUPPORTED as sgqa_decode does.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
- *     that device current) and caches it; make that first call before any stream capture.
+ *     that device current) and caches it; make that first call before any stream capture. The
+ *     cached address belongs to the device's current context: resetting the device
+ *     (cudaDeviceReset, or a reset of its primary context) while the library stays loaded
+ *     invalidates it, and calling this entry point after such a reset is not supported.
  *   - Each call zeroes the status word (on `stream`) before its kernels; the device status is not
  *     readable through this entry point (use sgqa_decode with a workspace when it is needed).
  *   - All calls share the array and it keeps the last call's contents: calls that overlap on the

@@ -263,6 +263,49 @@ def test_invalid_selection_is_reported_not_faulted():
     assert torch.isfinite(out.float()).all()
 
 
+def test_duplicate_selection_entry_is_reported_on_the_row_kernel(small_cases):
+    """R = 3 runs on the per-row attention kernel. A selection row that names a block twice breaks
+    the format (strictly ascending ids): the device check flags it (status 6) and skips the
+    repeated entry instead of weighting that block twice; every other row is unchanged."""
+    cfg, h, d, dm, kbar64, rows, sel_o, s_m = small_cases("r3_rowkernel")
+    assert cfg.Hq // cfg.G == 3
+    dims = sg.sgqa_dims.of(cfg)
+    sel_ok = torch.from_numpy(sel_o.reshape(cfg.batch, cfg.T, cfg.G, cfg.Kb)).cuda()
+    t_bad, g_bad = 777, 1
+    row = sel_o.reshape(cfg.batch, cfg.T, cfg.G, cfg.Kb)[0, t_bad, g_bad].copy()
+    n = int((row >= 0).sum())
+    assert n >= 3
+    dup = row.copy()
+    dup[1] = dup[0]  # block dup[0] named twice; the block that was second is dropped
+    sel_dup = sel_ok.clone()
+    sel_dup[0, t_bad, g_bad] = torch.from_numpy(dup).cuda()
+    outs = []
+    for s_, want in ((sel_ok, 0), (sel_dup, 6)):
+        ws = _ws(dims)
+        out = torch.full(shape_of(cfg, "q"), float("nan"), dtype=torch.bfloat16, device="cuda")
+        sg.sgqa_attend(dims, d["q"], d["k"], d["v"], d["gate"], s_, out, ws)
+        torch.cuda.synchronize()
+        assert sg.sgqa_get_device_status(ws) == want
+        outs.append(out)
+    a, b = outs[0].view(torch.int16), outs[1].view(torch.int16)
+    R = cfg.Hq // cfg.G
+    heads = slice(g_bad * R, (g_bad + 1) * R)
+    other = torch.ones(a.shape[:3], dtype=torch.bool, device="cuda")
+    other[0, t_bad, heads] = False
+    assert torch.equal(a[other], b[other])
+    # the flagged row attends to its selection without the repeated entry
+    kept = np.array([j for i, j in enumerate(dup) if j >= 0 and i != 1], dtype=np.int32)
+    sel_kept = np.full((1, cfg.G, cfg.Kb), -1, dtype=np.int32)
+    sel_kept[0] = sel_o.reshape(cfg.batch, cfg.T, cfg.G, cfg.Kb)[0, t_bad]
+    sel_kept[0, g_bad] = -1
+    sel_kept[0, g_bad, :len(kept)] = kept
+    r1 = np.array([[0, t_bad]], dtype=np.int32)
+    ref = oracle.attend(dm, r1, h["q"][0, t_bad].reshape(1, -1), h["k"], h["v"], h["gate"][0, t_bad].reshape(1, -1),
+                        sel_kept)
+    assert_outputs_close(to_host(outs[1][0, t_bad]), ref.reshape(cfg.Hq, cfg.d), "duplicate entry skipped")
+    assert torch.isfinite(outs[1].float()).all()
+
+
 def test_device_generator_matches_host_generator():
     cfg = CONFIGS["128k"]
     for name in NAMES:
@@ -337,6 +380,62 @@ def test_decode_small_matches_oracle():
 def test_decode_n1_and_b1():
     _decode_case(Config("dec_b1", 2, 3000, 8, 2, 64, 32, 1, 64, 300, 17), 2500, 3, [1])
     _decode_case(Config("dec_n1", 2, 3000, 8, 2, 64, 32, 8, 128, 300, 18), 2999, 1, [0])
+
+
+def test_decode_selection_matches_forward():
+    """Decode and forward compute the same definition on different kernels: on the same
+    sequence, decode's selection for the new rows equals forward's for those rows except at
+    near-ties (both are also checked against the oracle), and the outputs agree within the
+    parity bounds."""
+    cfg = Config("dec_fwd", 2, 6000, 32, 4, 128, 64, 8, 512, 500, 25)
+    cache_len, n_new = 5996, 4
+    Tn = cache_len + n_new
+    T_cap = Tn
+    # forward over the concatenated sequence
+    fcfg = cfg.replace(T=Tn)
+    fdims = sg.sgqa_dims.of(fcfg)
+    d = device_inputs(fcfg)
+    ws = _ws(fdims)
+    fout = torch.empty(shape_of(fcfg, "q"), dtype=torch.bfloat16, device="cuda")
+    fsel = torch.empty((fcfg.batch, Tn, cfg.G, cfg.Kb), dtype=torch.int32, device="cuda")
+    sg.sgqa_forward(fdims, d["q"], d["k"], d["v"], d["q_idx"], d["k_idx"], d["gate"], fout, ws, sel_out=fsel)
+    _status_ok(ws)
+    # decode of the last n_new rows after a cache of cache_len
+    dims = sg.sgqa_dims(cfg.batch, T_cap, cfg.Hq, cfg.G, cfg.d, cfg.d_idx, cfg.B, cfg.k)
+    caches = {n: torch.zeros(shape_of(cfg, n, T=T_cap), dtype=torch.bfloat16, device="cuda") for n in ("k", "v", "k_idx")}
+    for n in caches:
+        caches[n][:, :cache_len] = d[n][:, :cache_len]
+    kbar = torch.zeros((cfg.batch, T_cap // cfg.B, cfg.d_idx), device="cuda")
+    sg.sgqa_compress_keys(dims, caches["k_idx"], kbar, None)
+    new = {n: d[n][:, cache_len:].contiguous() for n in NAMES}
+    dws = sg.alloc_workspace(sg.sgqa_decode_workspace_size(dims, n_new))
+    sg.sgqa_reset_device_status(dws)
+    dout = torch.empty((cfg.batch, n_new, cfg.Hq, cfg.d), dtype=torch.bfloat16, device="cuda")
+    dsel = torch.empty((cfg.batch, n_new, cfg.G, cfg.Kb), dtype=torch.int32, device="cuda")
+    sg.sgqa_decode(dims, cache_len, n_new, caches["k"], caches["v"], caches["k_idx"], kbar, new["q"], new["k"],
+                   new["v"], new["q_idx"], new["k_idx"], new["gate"], dout, dws, sel_out=dsel)
+    _status_ok(dws)
+    dm = oracle.dims(1, Tn, cfg.Hq, cfg.G, cfg.d, cfg.d_idx, cfg.B, cfg.k)
+    differ = 0
+    for b in range(cfg.batch):
+        kbar64 = oracle.compress(dm, to_host(d["k_idx"][b:b + 1]))
+        rows = np.array([[0, t] for t in range(cache_len, Tn)], dtype=np.int32)
+        qi = to_host(new["q_idx"][b]).reshape(n_new, -1)
+        sel_o, s_m, _ = oracle.select(dm, kbar64, rows, qi)
+        ds = dsel[b].cpu().numpy()
+        fs = fsel[b, cache_len:].cpu().numpy()
+        compare_selection(dm, kbar64, rows, qi, ds, sel_o, s_m)
+        compare_selection(dm, kbar64, rows, qi, fs, sel_o, s_m)
+        differ += int((ds != fs).any(axis=2).sum())
+        ref = oracle.attend(dm, rows, to_host(new["q"][b]).reshape(n_new, -1), to_host(d["k"][b:b + 1]),
+                            to_host(d["v"][b:b + 1]), to_host(new["gate"][b]).reshape(n_new, -1), ds)
+        assert_outputs_close(to_host(dout[b]), ref.reshape(n_new, cfg.Hq, cfg.d), "decode")
+        same = (ds == fs).all(axis=2).all(axis=1)
+        if same.any():
+            sm = torch.from_numpy(same).cuda()
+            assert_outputs_close(to_host(dout[b][sm]), sgi.bf16_bits_to_f64(to_host(fout[b, cache_len:][sm])),
+                                 "decode vs forward")
+    print(f"decode vs forward: {differ} of {cfg.batch * n_new * cfg.G} rows differ (near-ties)")
 
 
 # ---- full-size workloads, sampled rows, the benchmark's launch configuration ----------------

@@ -40,11 +40,11 @@ def test_decode_noalloc_matches_decode_on_two_calls():
         new[n] = torch.empty((cfg.batch, n_new) + cfg.shape(n)[2:], dtype=torch.bfloat16, device="cuda")
         gen_device(cfg, n, new[n], t0=cache_len, n_t=n_new, dst_t0=0)
 
-    def run(fn, **kw):
+    def run(fn, with_sel=True, **kw):
         out = torch.full((cfg.batch, n_new, cfg.Hq, cfg.d), float("nan"), dtype=torch.bfloat16, device="cuda")
         sel = torch.full((cfg.batch, n_new, cfg.G, cfg.Kb), -7, dtype=torch.int32, device="cuda")
         fn(dims, cache_len, n_new, caches["k"], caches["v"], caches["k_idx"], kbar, new["q"], new["k"], new["v"],
-           new["q_idx"], new["k_idx"], new["gate"], out, sel_out=sel, **kw)
+           new["q_idx"], new["k_idx"], new["gate"], out, sel_out=sel if with_sel else None, **kw)
         torch.cuda.synchronize()
         return out, sel
 
@@ -53,10 +53,14 @@ def test_decode_noalloc_matches_decode_on_two_calls():
     ref_out, ref_sel = run(sg.sgqa_decode, ws=ws)
     assert sg.sgqa_get_device_status(ws) == 0
     ref = bf16_bits_to_f64(to_host(ref_out))
-    for _ in range(2):
-        out, sel = run(sg.sgqa_decode_noalloc)
-        assert torch.equal(sel, ref_sel)
+    # two calls in a row, the second without sel_out (the selection then lives in the scratch
+    # array); both run the same kernels on the same inputs as sgqa_decode, so the bits agree too
+    for with_sel in (True, False):
+        out, sel = run(sg.sgqa_decode_noalloc, with_sel=with_sel)
+        if with_sel:
+            assert torch.equal(sel, ref_sel)
         assert_outputs_close(to_host(out), ref, "sgqa_decode_noalloc vs sgqa_decode")
+        assert torch.equal(out.view(torch.int16), ref_out.view(torch.int16))
 
 
 def test_decode_noalloc_rejects_sizes_beyond_its_scratch():
