@@ -471,10 +471,19 @@ def _full_size_forward(cfg, n_rows, seed):
     return n_tie, err
 
 
+# near-tie (row, group) pairs allowed in a sample: the 32K workload's topic spans (128 blocks)
+# put the 511th place inside a cluster of similar scores in about a tenth of its rows
+NEAR_TIE_FRACTION = {"32k": 0.25, "128k": 0.05, "64k_b8": 0.15, "64k_b1": 0.15}
+
+
 @pytest.mark.parametrize("name", ["32k", "128k", "64k_b8", "64k_b1"])
 def test_full_size_prefill_sampled(name):
-    n_tie, err = _full_size_forward(CONFIGS[name], 48, 100)
-    print(f"{name}: near-tie rows {n_tie}; max-abs/mean-abs/rel-rms {err}")
+    cfg = CONFIGS[name]
+    n_rows = 2048
+    n_tie, err = _full_size_forward(cfg, n_rows, 100)
+    print(f"{name}: near-tie (row, group) pairs {n_tie} of {n_rows * cfg.G}; max-abs/mean-abs/rel-rms {err}")
+    assert n_tie <= NEAR_TIE_FRACTION[name] * n_rows * cfg.G
+    assert err[2] < 1e-2, f"rel-rms {err[2]}"
 
 
 def test_largest_budget_sampled():
@@ -486,5 +495,5 @@ def test_largest_budget_sampled():
 
 def test_full_size_decode_1m_sampled():
     cfg = CONFIGS["decode_1m"]
-    errs = _decode_case(cfg, cfg.T, DECODE_NEW, [0, 31])
+    errs = _decode_case(cfg, cfg.T, DECODE_NEW, [0, 5, 9, 14, 18, 23, 27, 31])
     print(f"decode 1M: {errs}")
