@@ -11,7 +11,9 @@ block-mean index keys (B tokens per block), per-KV-group top-(k/B) block selecti
 keeps the query's own block, causal softmax attention of every head of the group over the
 selected tokens scaled by 1/sqrt(d), and an elementwise sigmoid output gate. Also the Gated SWA
 layer that alternates 3:1 with it (same section): the gated attention over a sliding window of
-keys, the window size being a parameter (the pages give none).
+keys, the window size being a parameter (the pages give none). And the FP8 storage of the KV
+cache (section "long-horizon RL and run cost"): e4m3 values with a power-of-two scale per
+(token, group) row; decode over an FP8 cache is attention over the dequantized values.
 
 Parity pins: every function here is pinned by tests/test_oracle_pins.py (brute force on
 T <= 64, dense reduction against torch's SDPA in fp64, closed forms and invariants).
@@ -54,8 +56,10 @@ def load(path: str):
     L.oracle_coverage.argtypes = [ctypes.POINTER(Dims), ctypes.c_int, P, P, P, P, ctypes.c_int, P,
                                   ctypes.c_int]
     L.oracle_swa.argtypes = [ctypes.POINTER(Dims), ctypes.c_int, P, P, P, P, P, ctypes.c_int, P, ctypes.c_int]
+    L.oracle_quantize_fp8.argtypes = [ctypes.c_int, ctypes.c_int, P, P, P]
+    L.oracle_dequantize_fp8.argtypes = [ctypes.c_int, ctypes.c_int, P, P, P]
     for f in (L.oracle_compress, L.oracle_scores, L.oracle_select, L.oracle_attend, L.oracle_coverage,
-              L.oracle_swa, L.oracle_max_threads):
+              L.oracle_swa, L.oracle_max_threads, L.oracle_quantize_fp8, L.oracle_dequantize_fp8):
         f.restype = ctypes.c_int
     return L
 
@@ -181,6 +185,32 @@ def coverage(dm: Dims, rows_bt, q_rows, k, sel, ktop: int = 2048, n_threads: int
     if rc != 0:
         raise ValueError(f"oracle_coverage: {rc}")
     return cov
+
+
+def quantize_fp8(x) -> tuple:
+    """FP8 KV storage of bf16 rows x [..., d]: (codes uint8 [..., d] e4m3, scale fp64 [...]),
+    one power-of-two scale per row (the smallest with max |x| <= 448 * scale)."""
+    x = _u16(x)
+    d = x.shape[-1]
+    n = x.size // d
+    q = np.zeros(x.shape, dtype=np.uint8)
+    sc = np.zeros(x.shape[:-1], dtype=np.float64)
+    rc = lib().oracle_quantize_fp8(n, d, _p(x), _p(q), _p(sc))
+    if rc != 0:
+        raise ValueError(f"oracle_quantize_fp8: {rc}")
+    return q, sc
+
+
+def dequantize_fp8(q, scale) -> np.ndarray:
+    """fp64 values of FP8 rows: e4m3 value * row scale."""
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    scale = np.ascontiguousarray(scale, dtype=np.float64)
+    d = q.shape[-1]
+    out = np.zeros(q.shape, dtype=np.float64)
+    rc = lib().oracle_dequantize_fp8(q.size // d, d, _p(q), _p(scale), _p(out))
+    if rc != 0:
+        raise ValueError(f"oracle_dequantize_fp8: {rc}")
+    return out
 
 
 def forward(dm: Dims, q, k, v, q_idx, k_idx, gate, rows_bt=None, n_threads: int = 0):

@@ -287,4 +287,75 @@ int oracle_coverage(const Dims* dm, int n_rows, const int32_t* rows_bt, const ui
   return 0;
 }
 
+
+// FP8 KV cache (mo.ai.kr, "Step 5 Preview agentic work design", section "long-horizon RL and run
+// cost": the KV cache is trained for FP8 storage). The pages give no format details; the reading
+// taken: every (token, group) row of K or V (d values) is stored as FP8 E4M3 values (1 sign, 4
+// exponent bits with bias 7, 3 mantissa bits; largest finite value 448 = 1.75 * 2^8; subnormals
+// in steps of 2^-9) with one power-of-two scale s = 2^e per row, e the smallest integer with
+// max_i |x_i| <= 448 * 2^e (e = 0 for an all-zero row). Each value is x_i / s (exact) rounded to
+// the nearest E4M3 value, ties to the even mantissa. The dequantized value q_i * s has at most 4
+// significant bits, so it is exact in bf16: attention then runs on those values.
+//
+// e4m3 code of a finite |y| <= 448 (sign separately): the representable magnitudes are k * 2^-9
+// (k = 0..7, subnormal) and (8 + m) * 2^(E-3) (E = -6..8, m = 0..7, except E = 8, m = 7 ... 448 is
+// E = 8, m = 6; the all-ones code is NaN). Rounding: quantum 2^(E-3) for the binade of |y|
+// (E = -6 below 2^-6), n = |y| / quantum exact, round half to even.
+static uint8_t e4m3_encode(double y) {
+  const uint8_t sign = std::signbit(y) ? 0x80 : 0x00;
+  const double a = std::fabs(y);
+  if (a == 0.0) return sign;
+  int E = (int)std::floor(std::log2(a));
+  // guard the floor(log2) against rounding at exact powers of two
+  while (std::ldexp(1.0, E) > a) --E;
+  while (std::ldexp(1.0, E + 1) <= a) ++E;
+  if (E < -6) E = -6;
+  const double quantum = std::ldexp(1.0, E - 3);
+  const double n = a / quantum;                 // exact: a has a short significand here
+  double r = std::floor(n);
+  const double frac = n - r;
+  if (frac > 0.5 || (frac == 0.5 && std::fmod(r, 2.0) != 0.0)) r += 1.0;
+  const double v = r * quantum;                 // the rounded magnitude
+  if (v == 0.0) return sign;
+  if (v < std::ldexp(1.0, -6)) return (uint8_t)(sign | (uint8_t)(v / std::ldexp(1.0, -9)));  // subnormal
+  int Ev = (int)std::floor(std::log2(v));
+  while (std::ldexp(1.0, Ev) > v) --Ev;
+  while (std::ldexp(1.0, Ev + 1) <= v) ++Ev;
+  const int m = (int)(v / std::ldexp(1.0, Ev - 3)) - 8;
+  return (uint8_t)(sign | (uint8_t)((Ev + 7) << 3) | (uint8_t)m);
+}
+
+static double e4m3_decode(uint8_t c) {
+  const int e = (c >> 3) & 15, m = c & 7;
+  const double mag = e == 0 ? m * std::ldexp(1.0, -9) : (8 + m) * std::ldexp(1.0, e - 7 - 3);
+  return (c & 0x80) ? -mag : mag;
+}
+
+// Quantize n_rows rows of d bf16 values: q [n_rows, d] e4m3 codes, scale [n_rows] (powers of 2).
+int oracle_quantize_fp8(int n_rows, int d, const uint16_t* x, uint8_t* q, double* scale) {
+  if (n_rows < 0 || d <= 0) return -1;
+  for (long r = 0; r < n_rows; ++r) {
+    double amax = 0.0;
+    for (int i = 0; i < d; ++i) amax = std::max(amax, std::fabs(bf16_to_f64(x[r * d + i])));
+    int e = 0;
+    if (amax > 0.0) {
+      // smallest e with amax <= 448 * 2^e
+      e = (int)std::ceil(std::log2(amax / 448.0));
+      while (amax > 448.0 * std::ldexp(1.0, e)) ++e;
+      while (amax <= 448.0 * std::ldexp(1.0, e - 1)) --e;
+    }
+    scale[r] = std::ldexp(1.0, e);
+    for (int i = 0; i < d; ++i) q[r * d + i] = e4m3_encode(bf16_to_f64(x[r * d + i]) / scale[r]);
+  }
+  return 0;
+}
+
+// Dequantize: out [n_rows, d] fp64 = e4m3 value * scale.
+int oracle_dequantize_fp8(int n_rows, int d, const uint8_t* q, const double* scale, double* out) {
+  if (n_rows < 0 || d <= 0) return -1;
+  for (long r = 0; r < n_rows; ++r)
+    for (int i = 0; i < d; ++i) out[r * d + i] = e4m3_decode(q[r * d + i]) * scale[r];
+  return 0;
+}
+
 }  // extern "C"

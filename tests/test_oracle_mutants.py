@@ -9,7 +9,9 @@ SWA definition, a window one key too long or too short, unscaled scores, a missi
 interleaved head->group mapping (these are checked against the SWA pins); and in the token
 coverage of the ablation, a reversed ranking, an interleaved head->group mapping, ties sent to
 the higher token, a top set one token short, and the query's own token left out (these are
-checked against the coverage pins).
+checked against the coverage pins); and in the FP8 KV storage, ties rounded away from even, a
+scale one power of two off either way, the subnormal range cut at the wrong binade, and a dropped
+sign (checked against the FP8 pins).
 """
 import os
 import subprocess
@@ -81,6 +83,30 @@ COVERAGE_MUTANTS = {
 }
 
 
+# FP8 KV storage: rounding ties away from even, a scale one power too small or too large, the
+# subnormal range cut at the wrong binade, a dropped sign
+FP8_MUTANTS = {
+    "fp8_ties_away_from_even": ("if (frac > 0.5 || (frac == 0.5 && std::fmod(r, 2.0) != 0.0)) r += 1.0;",
+                                "if (frac >= 0.5) r += 1.0;"),
+    "fp8_scale_one_too_small": ("while (amax <= 448.0 * std::ldexp(1.0, e - 1)) --e;",
+                                "while (amax <= 448.0 * std::ldexp(1.0, e - 1)) --e;\n      --e;"),
+    "fp8_scale_one_too_large": ("while (amax <= 448.0 * std::ldexp(1.0, e - 1)) --e;",
+                                "while (amax <= 448.0 * std::ldexp(1.0, e - 1)) --e;\n      ++e;"),
+    "fp8_subnormal_binade": ("if (E < -6) E = -6;", "if (E < -7) E = -7;"),
+    "fp8_sign_dropped": ("return (c & 0x80) ? -mag : mag;", "return mag;"),
+}
+
+
+def _fp8_pin_calls():
+    import tests.test_oracle_fp8_pins as fp8
+    return [
+        lambda: fp8.test_fp8_codes_match_torch_e4m3_cast(None),
+        lambda: fp8.test_fp8_scale_is_the_smallest_power_of_two(None),
+        lambda: fp8.test_fp8_closed_forms(None),
+        lambda: fp8.test_fp8_error_bound_and_bf16_exactness(None),
+    ]
+
+
 def _coverage_pin_calls():
     return [
         lambda: pins.test_coverage_brute_force(None, False),
@@ -101,18 +127,18 @@ def _swa_pin_calls():
     ]
 
 
-ALL_MUTANTS = {**MUTANTS, **SWA_MUTANTS, **COVERAGE_MUTANTS}
+ALL_MUTANTS = {**MUTANTS, **SWA_MUTANTS, **COVERAGE_MUTANTS, **FP8_MUTANTS}
 
 
 @pytest.mark.parametrize("name", sorted(ALL_MUTANTS))
 def test_pins_catch_mutant(tmp_path, name):
     old, new = ALL_MUTANTS[name]
     calls = (PIN_CALLS if name in MUTANTS else _swa_pin_calls() if name in SWA_MUTANTS
-             else _coverage_pin_calls())
+             else _coverage_pin_calls() if name in COVERAGE_MUTANTS else _fp8_pin_calls())
     src = open(oracle.SRC).read()
     assert src.count(old) >= 1, f"mutation anchor not found: {name}"
-    if name in COVERAGE_MUTANTS:
-        assert src.count(old) == 1, f"coverage mutation anchor not unique: {name}"
+    if name in COVERAGE_MUTANTS or name in FP8_MUTANTS:
+        assert src.count(old) == 1, f"mutation anchor not unique: {name}"
     mutated = src.replace(old, new)
     cpp = tmp_path / "mut.cpp"
     so = tmp_path / "libmut.so"
