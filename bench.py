@@ -392,6 +392,9 @@ def run_ours(args, world, rank):
     torch.cuda.empty_cache()
     if not args.no_decode:
         result["decode"] = run_decode(args, world, s)
+        result["decode_fp8"] = run_decode_fp8(args, world, s)
+    if not args.no_ablation and world == 1:
+        result["ablation"] = run_ablation(args, world, s)
     if not args.no_swa:
         result["swa"] = run_swa(args, world, s)
     if cpu_in is not None:
@@ -443,7 +446,7 @@ def run_decode(args, world, s):
     assert sg.sgqa_get_device_status(ws) == 0
     toks = world * cfg.batch * n_new
     kbar_bytes = cfg.batch * (cache_len // cfg.B) * cfg.d_idx * 4
-    visits = cfg.batch * cfg.G * sum((cfg.Kb - 1) * cfg.B + i + 1 for i in range(n_new))
+    visits = decode_visits(cfg, n_new, cache_len)
     gather = visits * 2 * cfg.d * 2
     res = {"metric": "decode query tokens/s at 1M context (32 seqs x 4 new tokens)", "value": toks / (ms / 1e3),
            "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
@@ -451,9 +454,176 @@ def run_decode(args, world, s):
                        f"G={cfg.G}, d={cfg.d}, d_idx={cfg.d_idx}, B={cfg.B}, k={cfg.k}, span {cfg.span}, seed {cfg.seed}",
            "algorithmic_bytes": kbar_bytes + gather,
            "hbm_frac": (kbar_bytes + gather) / (ms / 1e3) / 1e9 / load_peaks()["hbm_gbs"],
-           "gpu_launches_per_step": 7}
+           "gpu_launches_per_step": 7}  # append x3, scores, select, union, attend
     del caches, kbar, new, out, ws
     torch.cuda.empty_cache()
+    return res
+
+
+def decode_visits(cfg, n_new, cache_len):
+    """(query, group, token) visits of one decode step: every new token attends its k/B - 1 picked
+    blocks (B tokens each) plus the tokens of its own block up to itself."""
+    return cfg.batch * cfg.G * sum((cfg.Kb - 1) * cfg.B + (cache_len + i) % cfg.B + 1 for i in range(n_new))
+
+
+def run_decode_fp8(args, world, s):
+    """The same decode step over FP8 K/V caches (e4m3 codes + a power-of-two scale per (token,
+    group) row, through sgqa_decode_fp8): the gathered cache bytes halve."""
+    import torch
+    import block_sparse_long_kbar_b200 as sg
+    from sgqa_inputs import gen_device
+    cfg = CONFIGS["decode_1m"]
+    n_new = DECODE_NEW
+    cache_len = cfg.T
+    T_cap = cache_len + cfg.B
+    dims = sg.sgqa_dims(cfg.batch, T_cap, cfg.Hq, cfg.G, cfg.d, cfg.d_idx, cfg.B, cfg.k)
+    c8 = {n: torch.zeros(cfg.shape(n, T=T_cap), dtype=torch.uint8, device="cuda") for n in ("k", "v")}
+    csc = {n: torch.zeros((cfg.batch, T_cap, cfg.G), dtype=torch.float32, device="cuda") for n in ("k", "v")}
+    chunk = 65536
+    for t0 in range(0, cache_len, chunk):
+        n = min(chunk, cache_len - t0)
+        for name in ("k", "v"):
+            tmp = torch.empty((cfg.batch, n, cfg.G, cfg.d), dtype=torch.bfloat16, device="cuda")
+            gen_device(cfg, name, tmp, t0=t0, n_t=n, dst_t0=0)
+            sg.sgqa_quantize_kv_fp8(dims, t0, n, tmp, c8[name], csc[name])
+            del tmp
+    kidx = torch.zeros(cfg.shape("k_idx", T=T_cap), dtype=torch.bfloat16, device="cuda")
+    gen_device(cfg, "k_idx", kidx, t0=0, n_t=cache_len)
+    kbar = torch.zeros((cfg.batch, T_cap // cfg.B, cfg.d_idx), device="cuda")
+    sg.sgqa_compress_keys(dims, kidx, kbar, None)
+    new = {}
+    for n in ("q", "k", "v", "gate", "q_idx", "k_idx"):
+        new[n] = torch.empty((cfg.batch, n_new) + cfg.shape(n)[2:], dtype=torch.bfloat16, device="cuda")
+        gen_device(cfg, n, new[n], t0=cache_len, n_t=n_new, dst_t0=0)
+    out = torch.empty((cfg.batch, n_new, cfg.Hq, cfg.d), dtype=torch.bfloat16, device="cuda")
+    ws = sg.alloc_workspace(sg.sgqa_decode_workspace_size(dims, n_new))
+    sg.sgqa_reset_device_status(ws)
+    torch.cuda.synchronize()
+
+    def step():
+        sg.sgqa_decode_fp8(dims, cache_len, n_new, c8["k"], csc["k"], c8["v"], csc["v"], kidx, kbar, new["q"],
+                           new["k"], new["v"], new["q_idx"], new["k_idx"], new["gate"], out, ws, stream=s)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    steps = max(args.steps, 10)
+    e0.record(s)
+    for _ in range(steps):
+        step()
+    e1.record(s)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
+    assert sg.sgqa_get_device_status(ws) == 0
+    toks = world * cfg.batch * n_new
+    kbar_bytes = cfg.batch * (cache_len // cfg.B) * cfg.d_idx * 4
+    visits = decode_visits(cfg, n_new, cache_len)
+    gather = visits * 2 * (cfg.d + 4)  # codes + the row scale, K and V
+    res = {"metric": "decode query tokens/s at 1M context, FP8 (e4m3) K/V caches (32 seqs x 4 new tokens)",
+           "value": toks / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+           "workload": f"decode fp8: {cfg.batch} seqs x {n_new} new tokens after {cache_len} cached, Hq={cfg.Hq}, "
+                       f"G={cfg.G}, d={cfg.d}, d_idx={cfg.d_idx}, B={cfg.B}, k={cfg.k}, span {cfg.span}, "
+                       f"seed {cfg.seed}",
+           "algorithmic_bytes": kbar_bytes + gather,
+           "hbm_frac": (kbar_bytes + gather) / (ms / 1e3) / 1e9 / load_peaks()["hbm_gbs"],
+           "gpu_launches_per_step": 8}
+    del c8, csc, kidx, kbar, new, out, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+ABLATION_COV_STRIDE = 2048  # coverage rows: every 2048th query of the 64K sequence (all 32 heads)
+
+
+def run_ablation(args, world, s):
+    """The selection ablation on one 64K sequence (identical seeded inputs): B = 8, k = 4096 against
+    B = 1, k = 2048. Throughput and stage times of the whole layer for both; the scored-candidate
+    and attended-token ratios; and the token coverage per (query, head) of each GPU selection: the
+    fraction of the query's top-2048 tokens by exact q.k that the selection holds (computed by the
+    oracle's coverage function on sampled rows)."""
+    import torch
+    import block_sparse_long_kbar_b200 as sg
+    from sgqa_inputs import gen_device
+    import oracle
+    res = {}
+    dev = None
+    cov_rows = None
+    for name in ("64k_b8", "64k_b1"):
+        cfg = CONFIGS[name]
+        dims = sg.sgqa_dims.of(cfg)
+        if dev is None:  # the generator does not depend on B or k: one set of inputs serves both
+            dev = {}
+            for n in ("q", "k", "v", "gate", "q_idx", "k_idx"):
+                dev[n] = torch.empty(cfg.shape(n), dtype=torch.bfloat16, device="cuda")
+                gen_device(cfg, n, dev[n])
+        out = torch.empty(cfg.shape("q"), dtype=torch.bfloat16, device="cuda")
+        sel = torch.empty((cfg.batch, cfg.T, cfg.G, cfg.Kb), dtype=torch.int32, device="cuda")
+        kbar = torch.empty((cfg.batch, cfg.T // cfg.B, cfg.d_idx), dtype=torch.float32, device="cuda")
+        ws = sg.alloc_workspace(sg.sgqa_workspace_size(dims))
+        sg.sgqa_reset_device_status(ws)
+
+        def step():
+            sg.sgqa_forward(dims, dev["q"], dev["k"], dev["v"], dev["q_idx"], dev["k_idx"], dev["gate"], out, ws,
+                            sel_out=sel, stream=s)
+
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for _ in range(args.steps):
+            step()
+        e1.record(s)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        st = {"select": [], "attend": []}
+        for _ in range(args.steps):
+            sg.sgqa_compress_keys(dims, dev["k_idx"], kbar, ws, stream=s)
+            ev[0].record(s)
+            sg.sgqa_select(dims, dev["q_idx"], kbar, sel, ws, stream=s)
+            ev[1].record(s)
+            sg.sgqa_attend(dims, dev["q"], dev["k"], dev["v"], dev["gate"], sel, out, ws, stream=s)
+            ev[2].record(s)
+            torch.cuda.synchronize()
+            st["select"].append(ev[0].elapsed_time(ev[1]))
+            st["attend"].append(ev[1].elapsed_time(ev[2]))
+        assert sg.sgqa_get_device_status(ws) == 0
+        wc = work_counts(cfg)
+        entry = {"value": cfg.batch * cfg.T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+                 "select_ms": statistics.mean(st["select"]), "attend_ms": statistics.mean(st["attend"]),
+                 "scored_candidates": wc["scored"], "attended_visits": wc["visits"],
+                 "B": cfg.B, "k": cfg.k}
+        if not args.no_cpu_baseline:
+            if cov_rows is None:
+                ts = np.arange(ABLATION_COV_STRIDE - 1, cfg.T, ABLATION_COV_STRIDE, dtype=np.int32)
+                cov_rows = np.stack([np.zeros_like(ts), ts], axis=1)
+                ti = torch.from_numpy(ts.astype(np.int64)).cuda()
+                cov_q = to_host(dev["q"][0].index_select(0, ti)).reshape(len(ts), -1)
+                cov_k = to_host(dev["k"][:1])
+            ti = torch.from_numpy(cov_rows[:, 1].astype(np.int64)).cuda()
+            gsel = sel[0].index_select(0, ti).cpu().numpy()
+            dm = oracle.dims(1, cfg.T, cfg.Hq, cfg.G, cfg.d, cfg.d_idx, cfg.B, cfg.k)
+            cov = oracle.coverage(dm, cov_rows, cov_q, cov_k, gsel, ktop=2048)
+            late = cov_rows[:, 1] >= 4096
+            entry["coverage"] = {"mean": float(cov.mean()), "mean_t_ge_4096": float(cov[late].mean()),
+                                 "rows": int(len(cov_rows)), "heads": cfg.Hq,
+                                 "sample": f"every {ABLATION_COV_STRIDE}th query (t = {ABLATION_COV_STRIDE - 1} + "
+                                           f"{ABLATION_COV_STRIDE} i), all heads; top-2048 by exact q.k"}
+        res[name] = entry
+        del out, sel, kbar, ws
+        torch.cuda.empty_cache()
+    del dev
+    torch.cuda.empty_cache()
+    b8, b1 = res["64k_b8"], res["64k_b1"]
+    res["ratios"] = {"scored_b1_over_b8": b1["scored_candidates"] / b8["scored_candidates"],
+                     "attended_b8_over_b1": b8["attended_visits"] / b1["attended_visits"],
+                     "select_ms_b1_over_b8": b1["select_ms"] / b8["select_ms"],
+                     "throughput_b8_over_b1": b8["value"] / b1["value"]}
+    res["workload"] = ("selection ablation: batch 1, T=65536, Hq=32, G=4, d=128, d_idx=64, topic span 2048, seed 3; "
+                       "B=8/k=4096 vs B=1/k=2048 on identical inputs")
     return res
 
 
@@ -605,6 +775,7 @@ def main():
     ap.add_argument("--config", default="128k", choices=["tiny", "32k", "128k", "64k_b8", "64k_b1"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-swa", action="store_true")
+    ap.add_argument("--no-ablation", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -26,7 +26,8 @@ STATUS_NAMES = {0: "SGQA_OK", 1: "SGQA_ERR_INVALID_ARG", 2: "SGQA_ERR_UNSUPPORTE
 # every symbol include/sgqa.h declares
 EXPORTS = ["sgqa_status_string", "sgqa_version", "sgqa_workspace_size", "sgqa_decode_workspace_size",
            "sgqa_reset_device_status", "sgqa_get_device_status", "sgqa_compress_keys", "sgqa_select",
-           "sgqa_attend", "sgqa_forward", "sgqa_decode", "sgqa_decode_noalloc", "sgqa_gated_swa"]
+           "sgqa_attend", "sgqa_forward", "sgqa_decode", "sgqa_decode_noalloc", "sgqa_gated_swa",
+           "sgqa_quantize_kv_fp8", "sgqa_decode_fp8", "sgqa_test_stall_decode_cta"]
 
 
 class SgqaError(RuntimeError):
@@ -74,8 +75,12 @@ def load_library():
     L.sgqa_decode.argtypes = [D, I, I] + [P] * 13 + [S, P]
     L.sgqa_decode_noalloc.argtypes = [D, I, I] + [P] * 12 + [P]
     L.sgqa_gated_swa.argtypes = [D, I, P, P, P, P, P, P, P, S, P]
+    L.sgqa_quantize_kv_fp8.argtypes = [D, I, I, P, P, P, P]
+    L.sgqa_decode_fp8.argtypes = [D, I, I] + [P] * 15 + [S, P]
+    L.sgqa_test_stall_decode_cta.argtypes = [I]
     for n in ("sgqa_reset_device_status", "sgqa_get_device_status", "sgqa_compress_keys", "sgqa_select",
-              "sgqa_attend", "sgqa_forward", "sgqa_decode", "sgqa_decode_noalloc", "sgqa_gated_swa"):
+              "sgqa_attend", "sgqa_forward", "sgqa_decode", "sgqa_decode_noalloc", "sgqa_gated_swa",
+              "sgqa_quantize_kv_fp8", "sgqa_decode_fp8", "sgqa_test_stall_decode_cta"):
         getattr(L, n).restype = I
     _lib = L
     return L
@@ -179,6 +184,28 @@ def sgqa_decode(dims, cache_len, n_new, k_cache, v_cache, kidx_cache, kbar_cache
         _ptr(kidx_cache, "kidx_cache"), _ptr(kbar_cache, "kbar_cache"), _ptr(q_new, "q_new"), _ptr(k_new, "k_new"),
         _ptr(v_new, "v_new"), _ptr(qidx_new, "qidx_new"), _ptr(kidx_new, "kidx_new"), _ptr(gate_new, "gate_new"),
         _ptr(out, "out"), _ptr(sel_out, "sel_out"), _ptr(ws, "ws"), ws.numel(), _stream(stream)))
+
+
+def sgqa_quantize_kv_fp8(dims, t0, n_t, src, dst8, dst_scale, stream=None):
+    """FP8 (e4m3 + power-of-two row scale) storage of rows [t0, t0 + n_t) of a K or V cache."""
+    _check("sgqa_quantize_kv_fp8", load_library().sgqa_quantize_kv_fp8(
+        ctypes.byref(dims), int(t0), int(n_t), _ptr(src, "src"), _ptr(dst8, "dst8"), _ptr(dst_scale, "dst_scale"),
+        _stream(stream)))
+
+
+def sgqa_decode_fp8(dims, cache_len, n_new, k8_cache, k_scale, v8_cache, v_scale, kidx_cache, kbar_cache, q_new,
+                    k_new, v_new, qidx_new, kidx_new, gate_new, out, ws, sel_out=None, stream=None):
+    _check("sgqa_decode_fp8", load_library().sgqa_decode_fp8(
+        ctypes.byref(dims), int(cache_len), int(n_new), _ptr(k8_cache, "k8_cache"), _ptr(k_scale, "k_scale"),
+        _ptr(v8_cache, "v8_cache"), _ptr(v_scale, "v_scale"), _ptr(kidx_cache, "kidx_cache"),
+        _ptr(kbar_cache, "kbar_cache"), _ptr(q_new, "q_new"), _ptr(k_new, "k_new"), _ptr(v_new, "v_new"),
+        _ptr(qidx_new, "qidx_new"), _ptr(kidx_new, "kidx_new"), _ptr(gate_new, "gate_new"), _ptr(out, "out"),
+        _ptr(sel_out, "sel_out"), _ptr(ws, "ws"), ws.numel(), _stream(stream)))
+
+
+def sgqa_test_stall_decode_cta(cta: int):
+    """Failure-detection test hook: decode attention CTA `cta` issues no loads (-1: off)."""
+    _check("sgqa_test_stall_decode_cta", load_library().sgqa_test_stall_decode_cta(int(cta)))
 
 
 NOALLOC_SCRATCH_BYTES = 16 << 20

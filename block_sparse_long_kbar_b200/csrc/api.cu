@@ -12,6 +12,7 @@ using namespace sgqa;
 namespace {
 
 constexpr int kSelChunkT = 32768;  // query rows per selection chunk when sel stays in ws
+int g_test_stall_cta = -1;         // sgqa_test_stall_decode_cta (failure-detection tests only)
 
 bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -74,24 +75,55 @@ int decode_splits(long units) {
 struct DecodeWs {
   int* status;
   float* scores;
+  uint32_t* tmax;   // per row, the largest key of every 32 candidates (tcgen05 scoring path)
+  int tstride;
+  bool tc_scores;   // tcgen05 scoring and the bound-based select run (else the CUDA-core K4/K5)
   int32_t* sel;
-  float* part;
+  int32_t* ublk;    // union of the n_new selections per (sequence, group) (tcgen05 path)
+  uint32_t* umask;
+  int* ucount;
+  float* part;      // split-K partial records
+  int splits;
+  bool tc;          // the tcgen05 attention runs (else the per-row kernel)
   size_t bytes;
 };
 
 DecodeWs decode_layout(const sgqa_dims* d, int n_new, void* ws) {
   DecodeWs w{};
   const size_t nblk = (size_t)(d->T / d->B);
+  const int Kb = d->k / d->B;
   const long units = (long)d->batch * n_new * d->G;
+  const int ug = d->batch * d->G;
   uint8_t* base = static_cast<uint8_t*>(ws);
   size_t off = kStatusBytes;
   w.status = reinterpret_cast<int*>(base);
   w.scores = reinterpret_cast<float*>(base + off);
   off += align256((size_t)units * nblk * 4);
+  w.tc_scores = decode_scores_tc_supported(d->d_idx, n_new, d->G);
+  w.tstride = (int)((nblk + 31) / 32);
+  if (w.tc_scores) {
+    w.tmax = reinterpret_cast<uint32_t*>(base + off);
+    off += align256((size_t)units * w.tstride * 4);
+  }
   w.sel = reinterpret_cast<int32_t*>(base + off);
-  off += align256((size_t)units * (d->k / d->B) * 4);
-  w.part = reinterpret_cast<float*>(base + off);
-  off += align256(attend_part_bytes((int)units, decode_splits(units), d->Hq / d->G, d->d));
+  off += align256((size_t)units * Kb * 4);
+  w.tc = decode_attend_tc_supported(d->Hq, d->G, d->d, d->B, n_new, Kb);
+  if (w.tc) {
+    const size_t ucap = (size_t)n_new * Kb;
+    w.ublk = reinterpret_cast<int32_t*>(base + off);
+    off += align256((size_t)ug * ucap * 4);
+    w.umask = reinterpret_cast<uint32_t*>(base + off);
+    off += align256((size_t)ug * ucap * 4);
+    w.ucount = reinterpret_cast<int*>(base + off);
+    off += align256((size_t)ug * 4);
+    w.splits = decode_attend_splits(ug, n_new, Kb, d->B);
+    w.part = reinterpret_cast<float*>(base + off);
+    off += align256(decode_part_bytes(ug, w.splits));
+  } else {
+    w.splits = decode_splits(units);
+    w.part = reinterpret_cast<float*>(base + off);
+    off += align256(attend_part_bytes((int)units, w.splits, d->Hq / d->G, d->d));
+  }
   w.bytes = off;
   return w;
 }
@@ -269,31 +301,56 @@ int sgqa_gated_swa(const sgqa_dims* dims, int window, const uint16_t* q, const u
   return SGQA_OK;
 }
 
-int sgqa_decode(const sgqa_dims* dims, int cache_len, int n_new, uint16_t* k_cache, uint16_t* v_cache,
-                uint16_t* kidx_cache, float* kbar_cache, const uint16_t* q_new, const uint16_t* k_new,
-                const uint16_t* v_new, const uint16_t* qidx_new, const uint16_t* kidx_new, const uint16_t* gate_new,
-                uint16_t* out, int32_t* sel_out, void* ws, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// K/V caches of a decode step: bf16 (k, v) or fp8 (k8, v8 with row scales)
+struct KvCaches {
+  uint16_t* k;
+  uint16_t* v;
+  uint8_t* k8;
+  uint8_t* v8;
+  float* k_scale;
+  float* v_scale;
+};
+
+int decode_impl(const sgqa_dims* dims, int cache_len, int n_new, const KvCaches& kv, uint16_t* kidx_cache,
+                float* kbar_cache, const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new,
+                const uint16_t* qidx_new, const uint16_t* kidx_new, const uint16_t* gate_new, uint16_t* out,
+                int32_t* sel_out, void* ws, size_t ws_bytes, void* stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
   if (n_new <= 0 || cache_len < 0 || (long)cache_len + n_new > dims->T || n_new * dims->G > 32)
     return SGQA_ERR_INVALID_ARG;
-  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(kidx_cache) || !aligned16(kbar_cache) ||
-      !aligned16(q_new) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(qidx_new) || !aligned16(kidx_new) ||
-      !aligned16(gate_new) || !aligned16(out) || (sel_out && !aligned16(sel_out)))
+  const bool f8 = kv.k8 != nullptr;
+  if (f8 ? (!aligned16(kv.k8) || !aligned16(kv.v8) || !aligned16(kv.k_scale) || !aligned16(kv.v_scale))
+         : (!aligned16(kv.k) || !aligned16(kv.v)))
+    return SGQA_ERR_INVALID_ARG;
+  if (!aligned16(kidx_cache) || !aligned16(kbar_cache) || !aligned16(q_new) || !aligned16(k_new) ||
+      !aligned16(v_new) || !aligned16(qidx_new) || !aligned16(kidx_new) || !aligned16(gate_new) || !aligned16(out) ||
+      (sel_out && !aligned16(sel_out)))
     return SGQA_ERR_INVALID_ARG;
   const DecodeWs w = decode_layout(dims, n_new, ws);
+  if (f8 && !w.tc) return SGQA_ERR_UNSUPPORTED;
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < w.bytes) return SGQA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int T = dims->T, G = dims->G, d = dims->d, di = dims->d_idx, B = dims->B, Kb = dims->k / dims->B;
   const int nblk = T / B;
   cudaError_t e = cudaSuccess;
-  // 1. append the new rows
-  if ((e = launch_append(k_cache, k_new, dims->batch, (long)G * d, (long)T * G * d, (long)cache_len * G * d,
-                         (long)n_new * G * d, s)) != cudaSuccess)
-    return SGQA_ERR_CUDA;
-  if ((e = launch_append(v_cache, v_new, dims->batch, (long)G * d, (long)T * G * d, (long)cache_len * G * d,
-                         (long)n_new * G * d, s)) != cudaSuccess)
-    return SGQA_ERR_CUDA;
+  // 1. append the new rows (quantized for fp8 caches)
+  if (f8) {
+    if ((e = launch_quantize_fp8(k_new, kv.k8, kv.k_scale, dims->batch, n_new, G, T, cache_len, s)) != cudaSuccess ||
+        (e = launch_quantize_fp8(v_new, kv.v8, kv.v_scale, dims->batch, n_new, G, T, cache_len, s)) != cudaSuccess)
+      return SGQA_ERR_CUDA;
+  } else {
+    if ((e = launch_append(kv.k, k_new, dims->batch, (long)G * d, (long)T * G * d, (long)cache_len * G * d,
+                           (long)n_new * G * d, s)) != cudaSuccess)
+      return SGQA_ERR_CUDA;
+    if ((e = launch_append(kv.v, v_new, dims->batch, (long)G * d, (long)T * G * d, (long)cache_len * G * d,
+                           (long)n_new * G * d, s)) != cudaSuccess)
+      return SGQA_ERR_CUDA;
+  }
   if ((e = launch_append(kidx_cache, kidx_new, dims->batch, di, (long)T * di, (long)cache_len * di, (long)n_new * di,
                          s)) != cudaSuccess)
     return SGQA_ERR_CUDA;
@@ -303,23 +360,95 @@ int sgqa_decode(const sgqa_dims* dims, int cache_len, int n_new, uint16_t* k_cac
                      cudaSuccess)
     return SGQA_ERR_CUDA;
   // 3. indexer scores and selection
-  if ((e = launch_decode_scores(qidx_new, kbar_cache, w.scores, dims->batch, n_new, G, di, B, nblk, cache_len, s)) !=
-      cudaSuccess)
-    return SGQA_ERR_CUDA;
   int32_t* sel = sel_out ? sel_out : w.sel;
-  if ((e = launch_decode_select(w.scores, sel, dims->batch, n_new, G, B, Kb, nblk, cache_len, w.status, s)) !=
-      cudaSuccess)
-    return SGQA_ERR_CUDA;
-  // 4. split-K gated attention
+  if (w.tc_scores) {
+    DecodeScoreArgs sa{};
+    sa.qidx = qidx_new; sa.kbar = kbar_cache; sa.scores = w.scores; sa.tmax = w.tmax; sa.batch = dims->batch;
+    sa.n_new = n_new; sa.G = G; sa.B = B; sa.nblk = nblk; sa.tstride = w.tstride; sa.t0 = cache_len;
+    sa.cps = decode_scores_ctas(dims->batch, (cache_len + n_new - 1) / B); sa.status = w.status;
+    if ((e = launch_decode_scores_tc(sa, s)) != cudaSuccess) return SGQA_ERR_CUDA;
+    if ((e = launch_decode_select_bound(w.scores, w.tmax, sel, dims->batch, n_new, G, B, Kb, nblk, w.tstride,
+                                        cache_len, w.status, s)) != cudaSuccess)
+      return SGQA_ERR_CUDA;
+  } else {
+    if ((e = launch_decode_scores(qidx_new, kbar_cache, w.scores, dims->batch, n_new, G, di, B, nblk, cache_len,
+                                  s)) != cudaSuccess)
+      return SGQA_ERR_CUDA;
+    if ((e = launch_decode_select(w.scores, sel, dims->batch, n_new, G, B, Kb, nblk, cache_len, w.status, s)) !=
+        cudaSuccess)
+      return SGQA_ERR_CUDA;
+  }
+  // 4. gated attention over the selection
+  if (w.tc) {
+    if (launch_decode_union(sel, dims->batch, n_new, G, Kb, w.ublk, w.umask, w.ucount, n_new * Kb, s) != cudaSuccess)
+      return SGQA_ERR_CUDA;
+    DecodeAttendArgs da{};
+    da.q = q_new; da.gate = gate_new; da.out = out; da.k = kv.k; da.v = kv.v;
+    da.k8 = kv.k8; da.v8 = kv.v8; da.k_scale = kv.k_scale; da.v_scale = kv.v_scale;
+    da.ublk = w.ublk; da.umask = w.umask; da.ucount = w.ucount; da.ucap = n_new * Kb; da.part = w.part;
+    da.batch = dims->batch; da.n_new = n_new; da.t0 = cache_len; da.T_kv = T; da.Hq = dims->Hq; da.G = G; da.d = d;
+    da.B = B; da.splits = w.splits; da.status = w.status; da.stall_cta = g_test_stall_cta;
+    if (launch_decode_attend_tc(da, s) != cudaSuccess) return SGQA_ERR_CUDA;
+    return SGQA_OK;
+  }
   AttendArgs a{};
-  a.q = q_new; a.gate = gate_new; a.out = out; a.k = k_cache; a.v = v_cache; a.sel = sel; a.part = w.part;
+  a.q = q_new; a.gate = gate_new; a.out = out; a.k = kv.k; a.v = kv.v; a.sel = sel; a.part = w.part;
   a.batch = dims->batch; a.nQ = n_new; a.q_t0 = cache_len; a.T_kv = T; a.Hq = dims->Hq; a.G = G; a.d = d; a.B = B;
   a.Kb = Kb; a.sel_T = n_new; a.sel_t0 = cache_len; a.t_begin = cache_len; a.t_end = cache_len + n_new;
-  a.splits = decode_splits((long)dims->batch * n_new * G);
+  a.splits = w.splits;
   a.status = w.status;
   if ((e = launch_attend(a, s)) != cudaSuccess) return SGQA_ERR_CUDA;
   if ((e = launch_attend_merge(a, s)) != cudaSuccess) return SGQA_ERR_CUDA;
   return SGQA_OK;
+}
+
+
+}  // namespace
+
+extern "C" {
+
+int sgqa_decode(const sgqa_dims* dims, int cache_len, int n_new, uint16_t* k_cache, uint16_t* v_cache,
+                uint16_t* kidx_cache, float* kbar_cache, const uint16_t* q_new, const uint16_t* k_new,
+                const uint16_t* v_new, const uint16_t* qidx_new, const uint16_t* kidx_new, const uint16_t* gate_new,
+                uint16_t* out, int32_t* sel_out, void* ws, size_t ws_bytes, void* stream) {
+  KvCaches kv{};
+  kv.k = k_cache;
+  kv.v = v_cache;
+  return decode_impl(dims, cache_len, n_new, kv, kidx_cache, kbar_cache, q_new, k_new, v_new, qidx_new, kidx_new,
+                     gate_new, out, sel_out, ws, ws_bytes, stream);
+}
+
+int sgqa_decode_fp8(const sgqa_dims* dims, int cache_len, int n_new, uint8_t* k8_cache, float* k_scale,
+                    uint8_t* v8_cache, float* v_scale, uint16_t* kidx_cache, float* kbar_cache, const uint16_t* q_new,
+                    const uint16_t* k_new, const uint16_t* v_new, const uint16_t* qidx_new, const uint16_t* kidx_new,
+                    const uint16_t* gate_new, uint16_t* out, int32_t* sel_out, void* ws, size_t ws_bytes,
+                    void* stream) {
+  if (!k8_cache || !v8_cache || !k_scale || !v_scale) return SGQA_ERR_INVALID_ARG;
+  KvCaches kv{};
+  kv.k8 = k8_cache;
+  kv.v8 = v8_cache;
+  kv.k_scale = k_scale;
+  kv.v_scale = v_scale;
+  return decode_impl(dims, cache_len, n_new, kv, kidx_cache, kbar_cache, q_new, k_new, v_new, qidx_new, kidx_new,
+                     gate_new, out, sel_out, ws, ws_bytes, stream);
+}
+
+int sgqa_test_stall_decode_cta(int cta) {
+  if (cta < -1) return SGQA_ERR_INVALID_ARG;
+  g_test_stall_cta = cta;
+  return SGQA_OK;
+}
+
+int sgqa_quantize_kv_fp8(const sgqa_dims* dims, int t0, int n_t, const uint16_t* src, uint8_t* dst8, float* dst_scale,
+                         void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (dims->d != 128) return SGQA_ERR_UNSUPPORTED;
+  if (t0 < 0 || n_t < 0 || (long)t0 + n_t > dims->T) return SGQA_ERR_INVALID_ARG;
+  if (n_t == 0) return SGQA_OK;
+  if (!aligned16(src) || !aligned16(dst8) || !aligned16(dst_scale)) return SGQA_ERR_INVALID_ARG;
+  return cuda_status(launch_quantize_fp8(src, dst8, dst_scale, dims->batch, n_t, dims->G, dims->T, t0,
+                                         static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -91,9 +91,9 @@ struct AtcShared {
   int nu, maxc, all_windows;
 };
 
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, const int* gstatus) {
   int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = tc::mbar_wait(bar, parity, abort) ? 1 : 0;
+  if ((threadIdx.x & 31) == 0) ok = tc::mbar_wait(bar, parity, abort, gstatus) ? 1 : 0;
   return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
 }
 
@@ -154,6 +154,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   const int seg = blockIdx.x / tiles_per_seg, tile = blockIdx.x % tiles_per_seg;
   const int b = seg / G, g = seg % G;
 
+  // a timeout recorded by another CTA (this launch or an earlier one sharing the status word):
+  // do nothing (the decision is the CTA's, before any barrier or TMEM is set up)
+  if (__syncthreads_or(tid == 0 && tc::grid_timed_out(a.status))) return;
   if (tid == 0) {
     for (int i = 0; i < kNS; ++i) {
       tc::mbar_init(&sh->kv_full[i], 1);
@@ -346,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         if (lane == 0) {
           for (int ch = 0; ch < nch && !sh->abort_flag; ++ch, ++kc) {
             const int st = (int)(kc % kNS);
-            if (kc >= kNS && !tc::mbar_wait(&sh->kv_empty[st], (uint32_t)(((kc / kNS) - 1) & 1), &sh->abort_flag)) {
+            if (kc >= kNS && !tc::mbar_wait(&sh->kv_empty[st], (uint32_t)(((kc / kNS) - 1) & 1), &sh->abort_flag, a.status)) {
               if (!sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
               sh->abort_flag = 1;
               break;
@@ -373,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           long pend_stage = -1;  // ring position of the chunk whose P V is still to issue
           auto issue_pv = [&](long stage_of) -> bool {
             const int pb = (int)(pcnt % kPB);
-            if (!tc::mbar_wait(&sh->p_full[pb], (uint32_t)((pcnt / kPB) & 1), &sh->abort_flag)) return false;
+            if (!tc::mbar_wait(&sh->p_full[pb], (uint32_t)((pcnt / kPB) & 1), &sh->abort_flag, a.status)) return false;
             tc::fence_after_sync();
             const int st = (int)(stage_of % kNS);
             const uint8_t* vbase = sKV + st * C::kStage + C::kKc;
@@ -395,8 +398,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           for (int ch = 0; ch < nch && ok && !sh->abort_flag; ++ch, ++kc, ++scnt) {
             const int st = (int)(kc % kNS);
             const int sb = (int)(scnt & 1);
-            if (!tc::mbar_wait(&sh->kv_full[st], (uint32_t)((kc / kNS) & 1), &sh->abort_flag) ||
-                (scnt >= 2 && !tc::mbar_wait(&sh->s_empty[sb], (uint32_t)(((scnt >> 1) - 1) & 1), &sh->abort_flag))) {
+            if (!tc::mbar_wait(&sh->kv_full[st], (uint32_t)((kc / kNS) & 1), &sh->abort_flag, a.status) ||
+                (scnt >= 2 && !tc::mbar_wait(&sh->s_empty[sb], (uint32_t)(((scnt >> 1) - 1) & 1), &sh->abort_flag, a.status))) {
               ok = false;
               break;
             }
@@ -428,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         // does not enter the arithmetic: P is elementwise, the row sums come from the MMA) ----
         for (int ch = 0; ch < nch; ++ch, ++scnt) {
           const int sb = (int)(scnt & 1);
-          if (!warp_wait(&sh->s_full[sb], (uint32_t)((scnt >> 1) & 1), &sh->abort_flag)) {
+          if (!warp_wait(&sh->s_full[sb], (uint32_t)((scnt >> 1) & 1), &sh->abort_flag, a.status)) {
             if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
             sh->abort_flag = 1;
             break;
@@ -443,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           if (lane == 0) tc::mbar_arrive(&sh->s_empty[sb]);
           const int pb = (int)(pcnt % kPB);
           if (main_pass && pcnt >= kPB &&
-              !warp_wait(&sh->p_empty[pb], (uint32_t)(((pcnt / kPB) - 1) & 1), &sh->abort_flag)) {
+              !warp_wait(&sh->p_empty[pb], (uint32_t)(((pcnt / kPB) - 1) & 1), &sh->abort_flag, a.status)) {
             if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
             sh->abort_flag = 1;
             break;
@@ -525,7 +528,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         ++o_commits;
       }
       if (is_sm) {
-        o_ok = warp_wait(&sh->o_done, (uint32_t)o_phase, &sh->abort_flag);
+        o_ok = warp_wait(&sh->o_done, (uint32_t)o_phase, &sh->abort_flag, a.status);
         if (!o_ok) {
           if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
           sh->abort_flag = 1;

@@ -94,19 +94,16 @@ __device__ int block_exclusive_scan(int v, int* scratch, int* total) {
   return before;
 }
 
-__global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const float* __restrict__ scores,
-                                                                    int32_t* __restrict__ sel, int n_new, int G, int B,
-                                                                    int Kb, int nblk, int t0, int* status) {
+// Exact selection of one row over its scores in global memory: radix passes of 8 key bits
+// (256-bin shared histograms, early exit), then an ordered emit over per-thread contiguous
+// segments with block scans of the tie and pick counts, so the output is ascending and ties at the
+// threshold go to the lower block index. Called by all kSelThreads threads of the block.
+__device__ void select_row_radix(const float* __restrict__ row, int c, int m, int Kb, int32_t* __restrict__ out,
+                                 int* status) {
   __shared__ int hist[256];
   __shared__ int scratch[64];
   __shared__ uint32_t s_prefix, s_mask;
   __shared__ int s_rem, s_nb;
-  const int rows = n_new * G;
-  const int b = blockIdx.x / rows, r = blockIdx.x % rows;
-  const int t = t0 + r / G;
-  const int c = t / B;
-  const int m = min(Kb - 1, c);
-  const float* row = scores + ((long)b * rows + r) * nblk;
   if (threadIdx.x == 0) {
     s_prefix = 0; s_mask = 0; s_rem = m; s_nb = c;
     if (m == 0) { s_prefix = 0xFFFFFFFFu; s_mask = 0xFFFFFFFFu; }
@@ -145,7 +142,7 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const float*
   const int rem = s_rem;
   // ordered emit: contiguous segments, counts, scans, then writes
   const int seg = (c + kSelThreads - 1) / kSelThreads;
-  const int j_lo = min(c, threadIdx.x * seg), j_hi = min(c, j_lo + seg);
+  const int j_lo = min(c, (int)threadIdx.x * seg), j_hi = min(c, j_lo + seg);
   int n_gt = 0, n_eq = 0;
   for (int j = j_lo; j < j_hi; ++j) {
     const uint32_t key = score_key(__ldg(row + j)) & mask;
@@ -156,7 +153,6 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const float*
   const int eq_before = block_exclusive_scan(n_eq, scratch, &tot);
   const int eq_take = max(0, min(n_eq, rem - eq_before));
   const int pos0 = block_exclusive_scan(n_gt + eq_take, scratch, &tot);
-  int32_t* out = sel + ((long)b * rows + r) * Kb;
   int pos = pos0, eq_seen = 0;
   for (int j = j_lo; j < j_hi; ++j) {
     const uint32_t key = score_key(__ldg(row + j)) & mask;
@@ -169,6 +165,185 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const float*
     out[m] = c;
   }
   for (int i = m + 1 + threadIdx.x; i < Kb; i += kSelThreads) out[i] = -1;
+}
+
+__global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const float* __restrict__ scores,
+                                                                    int32_t* __restrict__ sel, int n_new, int G, int B,
+                                                                    int Kb, int nblk, int t0, int* status) {
+  const int rows = n_new * G;
+  const int b = blockIdx.x / rows, r = blockIdx.x % rows;
+  const int c = (t0 + r / G) / B;
+  select_row_radix(scores + ((long)b * rows + r) * nblk, c, min(Kb - 1, c), Kb,
+                   sel + ((long)b * rows + r) * Kb, status);
+}
+
+// ---- K5 with a threshold bound ------------------------------------------------------------------
+// The largest key of every 32 consecutive candidates (written by K4) gives m distinct candidates
+// whose keys are >= the m-th largest of those maxima, L: so the row's m-th largest key is >= L and
+// every candidate below L can be dropped. One stream over the row's scores collects the survivors
+// (key >= L) with their block ids in shared memory (warp-aggregated slots, any order); the exact
+// selection is then made among them: radix passes over the survivors' keys for the threshold key
+// K*, and among the candidates equal to K* the lowest block ids (radix passes over ~j); the chosen
+// ids are sorted (bitonic) and written ascending. A row with more than kCap survivors (flat or
+// adversarial scores) takes the full radix path over its scores instead.
+constexpr int kCap = 8192;
+
+// Warp-aggregated histogram increment of bin `bin` (lanes with want == false add nothing).
+__device__ __forceinline__ void hist_add(int* hist, uint32_t bin, bool want) {
+  const unsigned act = __ballot_sync(0xFFFFFFFFu, want);
+  if (!want) return;
+  const unsigned peers = __match_any_sync(act, bin);
+  if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+}
+
+// m-th largest (1-based, 1 <= m <= number of valid entries) of get(i) over valid(i), i < n; all
+// threads of the block call it. Returns the key; *rem_out = m - (number of valid keys above it).
+template <class Get, class Valid>
+__device__ uint32_t kth_largest(int n, int m, Get get, Valid valid, int* rem_out) {
+  __shared__ int hist[256];
+  __shared__ uint32_t s_prefix, s_mask;
+  __shared__ int s_rem;
+  if (threadIdx.x == 0) { s_prefix = 0; s_mask = 0; s_rem = m; }
+  __syncthreads();
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    const uint32_t prefix = s_prefix, mask = s_mask;
+    for (int i = threadIdx.x; i < 256; i += kSelThreads) hist[i] = 0;
+    __syncthreads();
+    const int n_pad = (n + 31) & ~31;
+    for (int i = threadIdx.x; i < n_pad; i += kSelThreads) {
+      bool want = false;
+      uint32_t key = 0;
+      if (i < n && valid(i)) {
+        key = get(i);
+        want = (key & mask) == prefix;
+      }
+      hist_add(hist, (key >> shift) & 255u, want);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int above = 0;
+      const int rem = s_rem;
+      for (int bin = 255; bin >= 0; --bin) {
+        const int h = hist[bin];
+        if (above + h >= rem) {
+          s_prefix = prefix | ((uint32_t)bin << shift);
+          s_mask = mask | (255u << shift);
+          s_rem = rem - above;
+          break;
+        }
+        above += h;
+      }
+    }
+    __syncthreads();
+  }
+  *rem_out = s_rem;
+  const uint32_t res = s_prefix;
+  __syncthreads();
+  return res;
+}
+
+__global__ void __launch_bounds__(kSelThreads) decode_select_bound_kernel(const float* __restrict__ scores,
+                                                                          const uint32_t* __restrict__ tmax,
+                                                                          int32_t* __restrict__ sel, int n_new, int G,
+                                                                          int B, int Kb, int nblk, int tstride, int t0,
+                                                                          int sort_n, int* status) {
+  extern __shared__ uint32_t sm[];
+  uint32_t* skey = sm;             // [kCap]
+  uint32_t* sj = sm + kCap;        // [kCap]
+  uint32_t* sorted = sm + 2 * kCap;  // [sort_n]
+  __shared__ int s_cnt, s_pick;
+  const int rows = n_new * G;
+  const int b = blockIdx.x / rows, r = blockIdx.x % rows;
+  const int c = (t0 + r / G) / B;
+  const int m = min(Kb - 1, c);
+  const float* row = scores + ((long)b * rows + r) * nblk;
+  int32_t* out = sel + ((long)b * rows + r) * Kb;
+  const int tid = threadIdx.x, lane = tid & 31;
+  if (m == c) {  // every candidate is taken
+    for (int i = tid; i < Kb; i += kSelThreads) out[i] = i <= c ? i : -1;
+    return;
+  }
+  if (m == 0) {  // a budget of one block: the own block alone
+    for (int i = tid; i < Kb; i += kSelThreads) out[i] = i == 0 ? c : -1;
+    return;
+  }
+  // 1. the bound L
+  const int n32 = (c + 31) / 32;
+  uint32_t L = 0;
+  int rem_dummy;
+  if (n32 >= m) {
+    const uint32_t* tm = tmax + ((long)b * rows + r) * tstride;
+    L = kth_largest(n32, m, [&](int i) { return __ldg(tm + i); }, [](int) { return true; }, &rem_dummy);
+  }
+  // 2. survivors
+  if (tid == 0) { s_cnt = 0; s_pick = 0; }
+  __syncthreads();
+  for (int base = 0; base < c; base += 4 * kSelThreads) {
+    float v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = base + u * kSelThreads + tid;
+      v[u] = j < c ? __ldg(row + j) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = base + u * kSelThreads + tid;
+      const uint32_t key = score_key(v[u]);
+      const bool keep = j < c && key >= L;
+      const unsigned bal = __ballot_sync(0xFFFFFFFFu, keep);
+      if (bal == 0u) continue;
+      int pos = 0;
+      if (lane == __ffs(bal) - 1) pos = atomicAdd(&s_cnt, __popc(bal));
+      pos = __shfl_sync(0xFFFFFFFFu, pos, __ffs(bal) - 1) + __popc(bal & ((1u << lane) - 1u));
+      if (keep && pos < kCap) {
+        skey[pos] = key;
+        sj[pos] = (uint32_t)j;
+      }
+    }
+  }
+  __syncthreads();
+  const int ns = s_cnt;
+  if (ns > kCap) {
+    select_row_radix(row, c, m, Kb, out, status);
+    return;
+  }
+  // 3. the threshold key among the survivors, then the lowest block ids among its ties
+  int rem = 0;
+  const uint32_t kstar = kth_largest(ns, m, [&](int i) { return skey[i]; }, [](int) { return true; }, &rem);
+  int rem2 = 0;
+  const uint32_t jstar_n = kth_largest(ns, rem, [&](int i) { return ~sj[i]; },
+                                       [&](int i) { return skey[i] == kstar; }, &rem2);
+  const uint32_t jstar = ~jstar_n;
+  // 4. the chosen ids, sorted ascending (bitonic, padded with 0xFFFFFFFF)
+  for (int i = tid; i < sort_n; i += kSelThreads) sorted[i] = 0xFFFFFFFFu;
+  __syncthreads();
+  for (int i = tid; i < ns; i += kSelThreads) {
+    const uint32_t key = skey[i];
+    if (key > kstar || (key == kstar && sj[i] <= jstar)) {
+      const int p = atomicAdd(&s_pick, 1);
+      if (p < sort_n) sorted[p] = sj[i];
+    }
+  }
+  __syncthreads();
+  for (int k = 2; k <= sort_n; k <<= 1) {
+    for (int jj = k >> 1; jj > 0; jj >>= 1) {
+      for (int i = tid; i < sort_n; i += kSelThreads) {
+        const int ixj = i ^ jj;
+        if (ixj > i) {
+          const uint32_t x = sorted[i], y = sorted[ixj];
+          const bool asc = (i & k) == 0;
+          if ((x > y) == asc) {
+            sorted[i] = y;
+            sorted[ixj] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  if (tid == 0 && s_pick != m) report(status, SGQA_ERR_DEVICE_CHECK);
+  for (int i = tid; i < Kb; i += kSelThreads) out[i] = i < m ? (int32_t)sorted[i] : i == m ? c : -1;
 }
 
 }  // namespace
@@ -192,6 +367,20 @@ cudaError_t launch_decode_scores(const uint16_t* qidx_new, const float* kbar, fl
   if (d_idx == 64) decode_scores_kernel<64><<<grid, 256, 0, s>>>(qidx_new, kbar, scores, n_new, G, B, nblk, t0);
   else if (d_idx == 32) decode_scores_kernel<32><<<grid, 256, 0, s>>>(qidx_new, kbar, scores, n_new, G, B, nblk, t0);
   else return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_select_bound(const float* scores, const uint32_t* tmax, int32_t* sel, int batch, int n_new,
+                                       int G, int B, int Kb, int nblk, int tstride, int t0, int* status,
+                                       cudaStream_t s) {
+  int sort_n = 1;
+  while (sort_n < Kb) sort_n <<= 1;
+  const size_t shmem = (size_t)(2 * kCap + sort_n) * 4;
+  cudaError_t e = cudaFuncSetAttribute(decode_select_bound_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)shmem);
+  if (e != cudaSuccess) return e;
+  decode_select_bound_kernel<<<(unsigned)(batch * n_new * G), kSelThreads, shmem, s>>>(
+      scores, tmax, sel, n_new, G, B, Kb, nblk, tstride, t0, sort_n, status);
   return cudaGetLastError();
 }
 

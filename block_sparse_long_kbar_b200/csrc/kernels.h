@@ -78,7 +78,61 @@ cudaError_t launch_append(uint16_t* dst, const uint16_t* src, int batch, long ro
 cudaError_t launch_decode_scores(const uint16_t* qidx_new, const float* kbar, float* scores, int batch,
                                  int n_new, int G, int d_idx, int B, int nblk, int t0, cudaStream_t s);
 // K5: exact top-m select over the score rows; sel [batch, n_new, G, Kb].
+// K4 on tcgen05 (d_idx = 64, n_new * G <= 32): scores as launch_decode_scores (row stride nblk,
+// candidates j < c_max written) plus tmax [batch, n_new * G, tstride]: the largest order-preserving
+// key of each 32 consecutive candidates j < t/B of the row (0 where there are none).
+struct DecodeScoreArgs {
+  const uint16_t* qidx;  // [batch, n_new, G, 64]
+  const float* kbar;     // [batch, nblk, 64]
+  float* scores;
+  uint32_t* tmax;
+  int batch, n_new, G, B, nblk, tstride, t0, cps;
+  int* status;
+};
+bool decode_scores_tc_supported(int d_idx, int n_new, int G);
+int decode_scores_ctas(int batch, int c_max);
+cudaError_t launch_decode_scores_tc(const DecodeScoreArgs& a, cudaStream_t s);
+// K5 with the bound from tmax (exact; falls back to the full radix select per row when needed).
+cudaError_t launch_decode_select_bound(const float* scores, const uint32_t* tmax, int32_t* sel, int batch, int n_new,
+                                       int G, int B, int Kb, int nblk, int tstride, int t0, int* status,
+                                       cudaStream_t s);
 cudaError_t launch_decode_select(const float* scores, int32_t* sel, int batch, int n_new, int G, int B, int Kb,
                                  int nblk, int t0, int* status, cudaStream_t s);
+
+// K6 for decode on tcgen05 (d = 128, B in {8, 16}, n_new * Hq/G <= 64, n_new * Kb <= kUnionMax):
+// per (sequence, group) the union of the n_new queries' selections (ascending block ids and the
+// mask of the queries that selected each), then gated attention over it, split over `splits` CTAs
+// per (sequence, group) with a fixed-order merge (part: decode_part_bytes).
+constexpr int kUnionMax = 4096;
+struct DecodeAttendArgs {
+  const uint16_t* q;     // [batch, n_new, Hq, d]
+  const uint16_t* gate;  // [batch, n_new, Hq, d]
+  uint16_t* out;         // [batch, n_new, Hq, d]
+  const uint16_t* k;     // caches [batch, T_kv, G, d] (bf16; unused for fp8 caches)
+  const uint16_t* v;
+  const uint8_t* k8;     // fp8 caches [batch, T_kv, G, d] e4m3 (NULL for bf16 caches)
+  const uint8_t* v8;
+  const float* k_scale;  // fp8 caches: [batch, T_kv, G] power-of-two row scales
+  const float* v_scale;
+  const int32_t* ublk;   // [batch * G][ucap]
+  const uint32_t* umask; // [batch * G][ucap]
+  const int* ucount;     // [batch * G]
+  int ucap;
+  float* part;
+  int batch, n_new, t0, T_kv, Hq, G, d, B, splits;
+  int* status;
+  int stall_cta;         // failure-detection test hook: this CTA issues no loads (-1: none)
+};
+bool decode_attend_tc_supported(int Hq, int G, int d, int B, int n_new, int Kb);
+int decode_attend_splits(int units, int n_new, int Kb, int B);
+size_t decode_part_bytes(int units, int splits);
+cudaError_t launch_decode_union(const int32_t* sel, int batch, int n_new, int G, int Kb, int32_t* ublk,
+                                uint32_t* umask, int* ucount, int ucap, cudaStream_t s);
+cudaError_t launch_decode_attend_tc(const DecodeAttendArgs& a, cudaStream_t s);
+
+// FP8 KV storage: rows (b, t, g) of src [batch, n_t, G, 128] bf16 -> dst8 [batch, T, G, 128] e4m3
+// codes and dscale [batch, T, G] power-of-two scales at positions t0 + t.
+cudaError_t launch_quantize_fp8(const uint16_t* src, uint8_t* dst8, float* dscale, int batch, int n_t, int G, int T,
+                                int t0, cudaStream_t s);
 
 }  // namespace sgqa

@@ -77,7 +77,7 @@ struct SelShared {
 // Bounded barrier + "any" vote among the epilogue warps (slot = a fresh index per use): every
 // epilogue warp adds its vote and waits (bounded, abort-aware) until all have voted. Returns 1/0,
 // or -1 on giving up.
-__device__ __forceinline__ int epi_vote_any(SelShared* sh, int slot, bool v) {
+__device__ __forceinline__ int epi_vote_any(SelShared* sh, int slot, bool v, const int* gstatus) {
   const int lane = threadIdx.x & 31;
   const unsigned any = __any_sync(0xFFFFFFFFu, v);
   int res = 0;
@@ -88,8 +88,9 @@ __device__ __forceinline__ int epi_vote_any(SelShared* sh, int slot, bool v) {
     const uint64_t t0 = tc::globaltimer();
     volatile int* cnt = &sh->vote_cnt[slot];
     res = 1;
-    while (*cnt < kEpiWarps) {
+    for (uint32_t it = 1; *cnt < kEpiWarps; ++it) {
       if (sh->abort_flag || tc::globaltimer() - t0 > tc::kWaitLimitNs) { res = -1; break; }
+      if ((it & 1023u) == 0u && tc::grid_timed_out(gstatus)) { sh->abort_flag = 1; res = -1; break; }
       __nanosleep(32);
     }
     if (res > 0) {
@@ -101,19 +102,23 @@ __device__ __forceinline__ int epi_vote_any(SelShared* sh, int slot, bool v) {
 }
 
 // Warp-uniform bounded wait: lane 0 polls, the outcome is broadcast to the warp.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, const int* gstatus) {
   int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = tc::mbar_wait(bar, parity, abort) ? 1 : 0;
+  if ((threadIdx.x & 31) == 0) ok = tc::mbar_wait(bar, parity, abort, gstatus) ? 1 : 0;
   return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
 }
 
 // Wait until the epilogue has announced pass p-1 (and with it whether pass p exists).
-__device__ __forceinline__ int pass_exists(SelShared* sh, int p) {
+__device__ __forceinline__ int pass_exists(SelShared* sh, int p, const int* gstatus) {
   if (p == 0) return 1;
   const uint64_t t0 = tc::globaltimer();
-  while (sh->signals < p) {
+  for (uint32_t it = 1; sh->signals < p; ++it) {
     if (sh->abort_flag) return 0;
     if (tc::globaltimer() - t0 > tc::kWaitLimitNs) return -1;
+    if ((it & 1023u) == 0u && tc::grid_timed_out(gstatus)) {
+      sh->abort_flag = 1;
+      return 0;
+    }
     __nanosleep(64);
   }
   __threadfence_block();
@@ -315,6 +320,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_nt = (n_cand + kN - 1) / kN;
   const int nblk = a.T / a.B;
 
+  // a timeout recorded by another CTA (this launch or an earlier one sharing the status word):
+  // do nothing (the decision is the CTA's, before any barrier or TMEM is set up)
+  if (__syncthreads_or(tid == 0 && tc::grid_timed_out(a.status))) return;
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       tc::mbar_init(&sh->full[s], 1);
@@ -347,13 +355,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       long k = 0;
       bool ok = true;
       for (int pass = 0; ok && pass < kMaxPasses; ++pass) {
-        const int ex = pass_exists(sh, pass);
+        const int ex = pass_exists(sh, pass, a.status);
         if (ex < 0) { report(a.status, SGQA_ERR_TIMEOUT); sh->abort_flag = 1; ok = false; break; }
         if (ex == 0) break;
         for (int i = 0; i < n_nt; ++i, ++k) {
           const int st = (int)(k % kStages);
           const uint32_t ph = (uint32_t)((k / kStages) & 1);
-          if (k >= kStages && !tc::mbar_wait(&sh->empty[st], ph ^ 1u, &sh->abort_flag)) {
+          if (k >= kStages && !tc::mbar_wait(&sh->empty[st], ph ^ 1u, &sh->abort_flag, a.status)) {
             if (!sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
             sh->abort_flag = 1;
             ok = false;
@@ -382,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- MMA issuer ----------------
     if (lane == 0 && n_nt > 0) {
       const uint32_t idesc = tc::idesc_bf16_f32(kRows, kN);
-      bool ok = tc::mbar_wait(&sh->a_full, 0, &sh->abort_flag);
+      bool ok = tc::mbar_wait(&sh->a_full, 0, &sh->abort_flag, a.status);
       if (!ok) {
         if (!sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
         sh->abort_flag = 1;
@@ -390,15 +398,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t da = tc::smem_desc_kmajor(sA, C::kRowBytes);
       long k = 0;
       for (int pass = 0; ok && pass < kMaxPasses; ++pass) {
-        const int ex = pass_exists(sh, pass);
+        const int ex = pass_exists(sh, pass, a.status);
         if (ex < 0) { report(a.status, SGQA_ERR_TIMEOUT); sh->abort_flag = 1; ok = false; break; }
         if (ex == 0) break;
         for (int i = 0; i < n_nt; ++i, ++k) {
           const int st = (int)(k % kStages);
           const uint32_t ph = (uint32_t)((k / kStages) & 1);
           const int buf = (int)(k & 1);
-          if (!tc::mbar_wait(&sh->full[st], ph, &sh->abort_flag) ||
-              (k >= 2 && !tc::mbar_wait(&sh->acc_empty[buf], (uint32_t)(((k >> 1) - 1) & 1), &sh->abort_flag))) {
+          if (!tc::mbar_wait(&sh->full[st], ph, &sh->abort_flag, a.status) ||
+              (k >= 2 && !tc::mbar_wait(&sh->acc_empty[buf], (uint32_t)(((k >> 1) - 1) & 1), &sh->abort_flag, a.status))) {
             if (!sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
             sh->abort_flag = 1;
             ok = false;
@@ -452,10 +460,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // zero the histograms for this pass, then a barrier+vote: is any row still unresolved?
       if (half == 0 && !done && pass < kMaxPasses - 1)
         for (int i = 0; i < 256; ++i) my_hist[i] = 0;
-      const int vote = epi_vote_any(sh, 4 * pass, !done);
+      const int vote = epi_vote_any(sh, 4 * pass, !done, a.status);
       // from the third pass on, if every unresolved row's threshold bucket is small, this pass is
       // the last: it also collects those buckets' keys, which are then resolved exactly
-      const int vote_big = (pass >= 2 && vote > 0) ? epi_vote_any(sh, 4 * pass + 3, !done && nb > kCap) : 1;
+      const int vote_big = (pass >= 2 && vote > 0) ? epi_vote_any(sh, 4 * pass + 3, !done && nb > kCap, a.status) : 1;
       if (vote < 0 || vote_big < 0) {
         if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
         sh->abort_flag = 1;
@@ -487,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int shift = 24 - 8 * pass;
       for (int i = 0; i < n_nt; ++i, ++k) {
         const int buf = (int)(k & 1);
-        if (!warp_wait(&sh->acc_full[buf], (uint32_t)((k >> 1) & 1), &sh->abort_flag)) {
+        if (!warp_wait(&sh->acc_full[buf], (uint32_t)((k >> 1) & 1), &sh->abort_flag, a.status)) {
           if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
           sh->abort_flag = 1;
           aborted = true;
@@ -595,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       // both halves' histogram updates are complete before either reads the histogram
-      if (epi_vote_any(sh, 4 * pass + 1, false) < 0) {
+      if (epi_vote_any(sh, 4 * pass + 1, false, a.status) < 0) {
         if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
         sh->abort_flag = 1;
         break;
@@ -616,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         done = (rem == nb) || (mask == 0xFFFFFFFFu);
       }
       // both halves have read the histogram before the next pass zeroes it
-      if (epi_vote_any(sh, 4 * pass + 2, false) < 0) {
+      if (epi_vote_any(sh, 4 * pass + 2, false, a.status) < 0) {
         if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
         sh->abort_flag = 1;
         break;

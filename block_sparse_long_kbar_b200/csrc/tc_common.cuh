@@ -55,14 +55,28 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
       : "memory");
   return ok != 0;
 }
-// Wait for the phase with this parity to complete, giving up after kWaitLimitNs or when another
-// role of the CTA has raised *abort. Returns false on giving up.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// True when the launch's status word (global memory) records a timeout: some CTA gave up a wait,
+// so every other CTA of the grid (and of later launches sharing the status word, until it is
+// reset) stops instead of waiting out its own limit.
+__device__ __forceinline__ bool grid_timed_out(const int* gstatus) {
+  return gstatus && *reinterpret_cast<const volatile int*>(gstatus) == SGQA_ERR_TIMEOUT;
+}
+
+// Wait for the phase with this parity to complete, giving up after kWaitLimitNs, when another
+// role of the CTA has raised *abort, or (polled every 256 rounds, about every quarter
+// millisecond) when the grid's status word records a timeout, which also raises *abort. Returns
+// false on giving up.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          const int* gstatus = nullptr) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
-  while (true) {
+  for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait_sleep(bar, parity, 1000u)) return true;
     if (*abort) return false;
+    if ((it & 255u) == 0u && grid_timed_out(gstatus)) {
+      *abort = 1;
+      return false;
+    }
     if (globaltimer() - t0 > kWaitLimitNs) return false;
   }
 }

@@ -33,7 +33,9 @@
  *   - The return value reports argument validation and launch errors only (sgqa_status).
  *     Errors found on the device (a selection naming a block outside [0, t/B], a bounded wait
  *     that ran out) are recorded in the status word; read it with sgqa_get_device_status after
- *     synchronising the stream.
+ *     synchronising the stream. Once it records SGQA_ERR_TIMEOUT, the tensor-core kernels of every
+ *     CTA and of later calls sharing that ws stop early and leave their outputs unwritten, until
+ *     sgqa_reset_device_status.
  *   - Supported shapes (else SGQA_ERR_UNSUPPORTED): d in {64, 128}; d_idx in {32, 64};
  *     B in {1, 2, 4, 8, 16}; k % B == 0; Hq % G == 0 with 1 <= Hq/G <= 16; 128 % G == 0;
  *     1 <= T < 2^28; batch * T * Hq < 2^31. A trailing partial block is never a candidate.
@@ -143,6 +145,32 @@ int sgqa_decode(const sgqa_dims* dims, int cache_len, int n_new, uint16_t* k_cac
                 const uint16_t* kidx_new, const uint16_t* gate_new, uint16_t* out,
                 int32_t* sel_out, void* ws, size_t ws_bytes, void* stream);
 
+/* FP8 storage of the KV cache (mo.ai.kr, "Step 5 Preview agentic work design", section
+ * "long-horizon RL and run cost": the KV cache is trained for FP8 storage; the format is not given
+ * there, this is the reading taken). Each (token, group) row of K or V is stored as d FP8 E4M3
+ * codes plus one power-of-two scale s = 2^e per row, e the smallest integer with
+ * max |x| <= 448 * s; a code is x / s rounded to the nearest E4M3 value (ties to even, 448 the
+ * largest magnitude). code * s has at most 4 significant bits, so it is exact in bf16.
+ * Quantizes rows [t0, t0 + n_t) of every sequence: src [batch, n_t, G, d] bf16 (the rows to
+ * store) -> dst8 [batch, T, G, d] uint8 codes and dst_scale [batch, T, G] fp32 at positions
+ * t0 .. t0 + n_t - 1 (dims->T = the caches' capacity). d must be 128 (else
+ * SGQA_ERR_UNSUPPORTED); t0 + n_t <= T (else SGQA_ERR_INVALID_ARG). No workspace. */
+int sgqa_quantize_kv_fp8(const sgqa_dims* dims, int t0, int n_t, const uint16_t* src, uint8_t* dst8,
+                         float* dst_scale, void* stream);
+
+/* sgqa_decode over FP8 K/V caches (format of sgqa_quantize_kv_fp8): k8_cache, v8_cache
+ * [batch, T, G, d] codes with k_scale, v_scale [batch, T, G]; the step quantizes the n_new new K and
+ * V rows into them (same rule), then computes the layer exactly as sgqa_decode would on caches
+ * holding the dequantized values (selection: the index keys are not quantized, so it is
+ * sgqa_decode's). Half the cache bytes of the bf16 step are gathered. Needs the tensor-core decode
+ * attention: d = 128, B in {8, 16}, n_new * Hq/G <= 64, n_new * k/B <= 4096 (else
+ * SGQA_ERR_UNSUPPORTED). Workspace: sgqa_decode_workspace_size. */
+int sgqa_decode_fp8(const sgqa_dims* dims, int cache_len, int n_new, uint8_t* k8_cache, float* k_scale,
+                    uint8_t* v8_cache, float* v_scale, uint16_t* kidx_cache, float* kbar_cache,
+                    const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new,
+                    const uint16_t* qidx_new, const uint16_t* kidx_new, const uint16_t* gate_new,
+                    uint16_t* out, int32_t* sel_out, void* ws, size_t ws_bytes, void* stream);
+
 /* Gated SWA: the efficient attention layer that alternates 3:1 with the Sparse GQA layer
  * (mo.ai.kr, "Step 5 Preview agentic work design", section "model structure and training
  * stability"; ai.info, "StepFun illustrates the 92-block architecture of Step 5 Preview", section
@@ -162,6 +190,15 @@ int sgqa_decode(const sgqa_dims* dims, int cache_len, int n_new, uint16_t* k_cac
 int sgqa_gated_swa(const sgqa_dims* dims, int window, const uint16_t* q, const uint16_t* k,
                    const uint16_t* v, const uint16_t* gate, uint16_t* out, int32_t* sel_out,
                    void* ws, size_t ws_bytes, void* stream);
+
+/* Failure-detection test hook (host-side setting, not for production use). While cta >= 0, the
+ * decode attention CTA with that grid index in later sgqa_decode / sgqa_decode_fp8 calls issues
+ * no loads, so its tensor-core issuer's wait for the first tile is never satisfied: the wait
+ * runs out after its bound (2 s), the kernel records SGQA_ERR_TIMEOUT in the status word and
+ * returns with nothing in flight, and every other CTA and later kernel that polls that status
+ * word stops early (until sgqa_reset_device_status). cta = -1 turns the hook off. Returns
+ * SGQA_ERR_INVALID_ARG for cta < -1. Not thread-safe: set it while no other host thread calls. */
+int sgqa_test_stall_decode_cta(int cta);
 
 /* Size of the library-owned scratch array that sgqa_decode_noalloc uses (16 MiB). */
 #define SGQA_NOALLOC_SCRATCH_BYTES (16u << 20)

@@ -382,6 +382,68 @@ def test_decode_n1_and_b1():
     _decode_case(Config("dec_n1", 2, 3000, 8, 2, 64, 32, 8, 128, 300, 18), 2999, 1, [0])
 
 
+@pytest.mark.parametrize("cfg,cache_len,n_new,seqs", [
+    (Config("dec_b16", 2, 4000, 32, 4, 128, 64, 16, 512, 500, 26), 3990, 4, [1]),      # blocks of 16
+    (Config("dec_r16", 2, 3000, 64, 4, 128, 64, 8, 256, 300, 27), 2996, 4, [0]),       # 64 query-head columns
+    (Config("dec_q1", 3, 3000, 32, 4, 128, 64, 8, 512, 300, 28), 2777, 1, [2]),        # one new token
+    (Config("dec_q3", 1, 3000, 16, 2, 128, 64, 8, 1024, 300, 29), 2600, 3, [0]),       # R = 8, G = 2, splits
+])
+def test_decode_tensor_core_shapes(cfg, cache_len, n_new, seqs):
+    _decode_case(cfg, cache_len, n_new, seqs)
+
+
+def test_decode_rows_far_above_their_reference_max():
+    """Decode rows whose scores exceed their own block's maximum far beyond the fp32 exponent range
+    (block 0's keys scaled by 64; every block is selected since k covers the whole cache): the
+    decode attention must stream its tiles again with exact maxima for those columns. v is scaled
+    by 1/4 so the bf16 rounding of the near-one-hot outputs stays inside the bound."""
+    cfg = Config("dec_risky", 2, 600, 32, 4, 128, 64, 8, 640, 100, 30)
+    cache_len, n_new = 596, 4
+    T_cap = 600
+    dims = sg.sgqa_dims(cfg.batch, T_cap, cfg.Hq, cfg.G, cfg.d, cfg.d_idx, cfg.B, cfg.k)
+    caches = {}
+    for n in ("k", "v", "k_idx"):
+        caches[n] = torch.zeros(shape_of(cfg, n, T=T_cap), dtype=torch.bfloat16, device="cuda")
+        gen_device(cfg, n, caches[n], t0=0, n_t=cache_len)
+    caches["k"][:, :cfg.B] *= 64.0
+    caches["v"] *= 0.25
+    kbar = torch.zeros((cfg.batch, T_cap // cfg.B, cfg.d_idx), device="cuda")
+    sg.sgqa_compress_keys(dims, caches["k_idx"], kbar, None)
+    new = {}
+    for n in NAMES:
+        new[n] = torch.empty((cfg.batch, n_new) + shape_of(cfg, n)[2:], dtype=torch.bfloat16, device="cuda")
+        gen_device(cfg, n, new[n], t0=cache_len, n_t=n_new, dst_t0=0)
+    new["v"] *= 0.25
+    ws = sg.alloc_workspace(sg.sgqa_decode_workspace_size(dims, n_new))
+    sg.sgqa_reset_device_status(ws)
+    out = torch.full((cfg.batch, n_new, cfg.Hq, cfg.d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    sel = torch.full((cfg.batch, n_new, cfg.G, cfg.Kb), -7, dtype=torch.int32, device="cuda")
+    sg.sgqa_decode(dims, cache_len, n_new, caches["k"], caches["v"], caches["k_idx"], kbar, new["q"], new["k"],
+                   new["v"], new["q_idx"], new["k_idx"], new["gate"], out, ws, sel_out=sel)
+    _status_ok(ws)
+    Tn = cache_len + n_new
+    dm = oracle.dims(1, Tn, cfg.Hq, cfg.G, cfg.d, cfg.d_idx, cfg.B, cfg.k)
+    sc = np.log2(np.e) / np.sqrt(cfg.d)
+    gap = 0.0
+    for b in range(cfg.batch):
+        kh, vh = to_host(caches["k"][b:b + 1, :Tn]), to_host(caches["v"][b:b + 1, :Tn])
+        gsel = sel[b].cpu().numpy()
+        assert (gsel[:, :, 0] == 0).all()  # every row selected block 0
+        rows = np.array([[0, cache_len + i] for i in range(n_new)], dtype=np.int32)
+        qh = to_host(new["q"][b]).reshape(n_new, -1)
+        kf = sgi.bf16_bits_to_f64(kh.reshape(Tn, cfg.G, cfg.d))
+        qf = sgi.bf16_bits_to_f64(qh.reshape(n_new, cfg.Hq, cfg.d))
+        for i in range(n_new):
+            t = cache_len + i
+            c = t // cfg.B
+            for h in range(cfg.Hq):
+                g = h // cfg.R
+                gap = max(gap, ((kf[:cfg.B, g] @ qf[i, h]).max() - (kf[c * cfg.B:t + 1, g] @ qf[i, h]).max()) * sc)
+        ref = oracle.attend(dm, rows, qh, kh, vh, to_host(new["gate"][b]).reshape(n_new, -1), gsel)
+        assert_outputs_close(to_host(out[b]), ref.reshape(n_new, cfg.Hq, cfg.d), f"risky decode seq {b}")
+    assert gap > 130, gap
+
+
 def test_decode_selection_matches_forward():
     """Decode and forward compute the same definition on different kernels: on the same
     sequence, decode's selection for the new rows equals forward's for those rows except at
