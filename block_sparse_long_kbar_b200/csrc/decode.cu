@@ -180,13 +180,17 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const float*
 // ---- K5 with a threshold bound ------------------------------------------------------------------
 // The largest key of every 32 consecutive candidates (written by K4) gives m distinct candidates
 // whose keys are >= the m-th largest of those maxima, L: so the row's m-th largest key is >= L and
-// every candidate below L can be dropped. One stream over the row's scores collects the survivors
-// (key >= L) with their block ids in shared memory (warp-aggregated slots, any order); the exact
-// selection is then made among them: radix passes over the survivors' keys for the threshold key
-// K*, and among the candidates equal to K* the lowest block ids (radix passes over ~j); the chosen
-// ids are sorted (bitonic) and written ascending. A row with more than kCap survivors (flat or
-// adversarial scores) takes the full radix path over its scores instead.
+// every candidate below L can be dropped. Index keys cluster by topic, so L alone can still leave
+// tens of thousands of candidates; one stream over the row's scores therefore histograms the top
+// 12 bits of every key >= L (4096 bins), which locates the bin holding the m-th largest key, and
+// a second stream collects the candidates at or above that bin (typically a few thousand) with
+// their block ids in shared memory. The exact selection is then made among them: radix passes
+// over their keys for the threshold key K*, and among the candidates equal to K* the lowest block
+// ids (radix passes over ~j); the chosen ids are sorted (bitonic) and written ascending. A row
+// whose threshold bin alone holds more than kCap candidates takes the full radix path instead.
 constexpr int kCap = 8192;
+constexpr int kHBits = 12;
+constexpr int kHBins = 1 << kHBits;
 
 // Warp-aggregated histogram increment of bin `bin` (lanes with want == false add nothing).
 __device__ __forceinline__ void hist_add(int* hist, uint32_t bin, bool want) {
@@ -221,18 +225,35 @@ __device__ uint32_t kth_largest(int n, int m, Get get, Valid valid, int* rem_out
       hist_add(hist, (key >> shift) & 255u, want);
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      int above = 0;
+    if (threadIdx.x < 32) {
+      // warp 0 locates the bin: lane l holds bins 255 - 8l .. 248 - 8l, counts above by a scan
+      const int ln = threadIdx.x;
       const int rem = s_rem;
-      for (int bin = 255; bin >= 0; --bin) {
-        const int h = hist[bin];
-        if (above + h >= rem) {
-          s_prefix = prefix | ((uint32_t)bin << shift);
-          s_mask = mask | (255u << shift);
-          s_rem = rem - above;
-          break;
+      __syncwarp();
+      int cnt[8], local = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        cnt[i] = hist[255 - 8 * ln - i];
+        local += cnt[i];
+      }
+      int x = local;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+        if (ln >= o) x += y;
+      }
+      int acc = x - local;  // keys in the bins above this lane's
+      if (acc < rem && acc + local >= rem) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (acc + cnt[i] >= rem) {
+            s_prefix = prefix | ((uint32_t)(255 - 8 * ln - i) << shift);
+            s_mask = mask | (255u << shift);
+            s_rem = rem - acc;
+            break;
+          }
+          acc += cnt[i];
         }
-        above += h;
       }
     }
     __syncthreads();
@@ -249,10 +270,12 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_bound_kernel(const 
                                                                           int B, int Kb, int nblk, int tstride, int t0,
                                                                           int sort_n, int* status) {
   extern __shared__ uint32_t sm[];
-  uint32_t* skey = sm;             // [kCap]
-  uint32_t* sj = sm + kCap;        // [kCap]
+  uint32_t* skey = sm;               // [kCap]
+  uint32_t* sj = sm + kCap;          // [kCap]
   uint32_t* sorted = sm + 2 * kCap;  // [sort_n]
-  __shared__ int s_cnt, s_pick;
+  int* hist = reinterpret_cast<int*>(sm);  // [kHBins], before the survivors are collected
+  __shared__ int s_cnt, s_pick, s_bin, s_total;
+  __shared__ int scratch[64];
   const int rows = n_new * G;
   const int b = blockIdx.x / rows, r = blockIdx.x % rows;
   const int c = (t0 + r / G) / B;
@@ -268,7 +291,7 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_bound_kernel(const 
     for (int i = tid; i < Kb; i += kSelThreads) out[i] = i == 0 ? c : -1;
     return;
   }
-  // 1. the bound L
+  // 1. the bound L from the maxima of 32 candidates
   const int n32 = (c + 31) / 32;
   uint32_t L = 0;
   int rem_dummy;
@@ -276,7 +299,8 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_bound_kernel(const 
     const uint32_t* tm = tmax + ((long)b * rows + r) * tstride;
     L = kth_largest(n32, m, [&](int i) { return __ldg(tm + i); }, [](int) { return true; }, &rem_dummy);
   }
-  // 2. survivors
+  // 2. histogram of the top 12 key bits of the keys >= L
+  for (int i = tid; i < kHBins; i += kSelThreads) hist[i] = 0;
   if (tid == 0) { s_cnt = 0; s_pick = 0; }
   __syncthreads();
   for (int base = 0; base < c; base += 4 * kSelThreads) {
@@ -290,7 +314,53 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_bound_kernel(const 
     for (int u = 0; u < 4; ++u) {
       const int j = base + u * kSelThreads + tid;
       const uint32_t key = score_key(v[u]);
-      const bool keep = j < c && key >= L;
+      hist_add(hist, key >> (32 - kHBits), j < c && key >= L);
+    }
+  }
+  __syncthreads();
+  // the bin of the m-th largest key: suffix sums over 8 bins per thread, scanned from the top
+  {
+    constexpr int kPer = kHBins / kSelThreads;
+    const int top = kHBins - 1 - kPer * tid;  // this thread's bins: top, top - 1, ..., top - kPer + 1
+    int local = 0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) local += hist[top - i];
+    int tot;
+    const int above = block_exclusive_scan(local, scratch, &tot);  // keys in all higher threads' bins
+    if (above < m && above + local >= m) {
+      int acc = above;
+      for (int i = 0; i < kPer; ++i) {
+        const int h = hist[top - i];
+        if (acc + h >= m) {
+          s_bin = top - i;
+          s_total = acc + h;  // keys at or above the threshold bin
+          break;
+        }
+        acc += h;
+      }
+    }
+  }
+  __syncthreads();
+  const int total = s_total;
+  if (total > kCap) {
+    select_row_radix(row, c, m, Kb, out, status);
+    return;
+  }
+  const uint32_t lo = (uint32_t)s_bin << (32 - kHBits);
+  __syncthreads();  // the histogram area is reused for the survivors below
+  // 3. the survivors (keys at or above the threshold bin), any order
+  for (int base = 0; base < c; base += 4 * kSelThreads) {
+    float v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = base + u * kSelThreads + tid;
+      v[u] = j < c ? __ldg(row + j) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = base + u * kSelThreads + tid;
+      const uint32_t key = score_key(v[u]);
+      const bool keep = j < c && key >= lo && key >= L;
       const unsigned bal = __ballot_sync(0xFFFFFFFFu, keep);
       if (bal == 0u) continue;
       int pos = 0;
@@ -304,18 +374,30 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_bound_kernel(const 
   }
   __syncthreads();
   const int ns = s_cnt;
-  if (ns > kCap) {
-    select_row_radix(row, c, m, Kb, out, status);
-    return;
-  }
-  // 3. the threshold key among the survivors, then the lowest block ids among its ties
+  if (ns != total) report(status, SGQA_ERR_DEVICE_CHECK);
+  // 4. the threshold key among the survivors, then the lowest block ids among its ties
   int rem = 0;
   const uint32_t kstar = kth_largest(ns, m, [&](int i) { return skey[i]; }, [](int) { return true; }, &rem);
-  int rem2 = 0;
-  const uint32_t jstar_n = kth_largest(ns, rem, [&](int i) { return ~sj[i]; },
-                                       [&](int i) { return skey[i] == kstar; }, &rem2);
-  const uint32_t jstar = ~jstar_n;
-  // 4. the chosen ids, sorted ascending (bitonic, padded with 0xFFFFFFFF)
+  // among the keys equal to K*, the rem lowest block ids (all of them when there are just rem)
+  if (tid == 0) s_pick = 0;
+  __syncthreads();
+  {
+    int eq = 0;
+    for (int i = tid; i < ns; i += kSelThreads) eq += skey[i] == kstar;
+    eq = __reduce_add_sync(0xFFFFFFFFu, eq);
+    if (lane == 0 && eq) atomicAdd(&s_pick, eq);
+  }
+  __syncthreads();
+  const int n_eq = s_pick;
+  __syncthreads();
+  if (tid == 0) s_pick = 0;
+  uint32_t jstar = 0xFFFFFFFFu;
+  if (n_eq > rem) {
+    int rem2 = 0;
+    jstar = ~kth_largest(ns, rem, [&](int i) { return ~sj[i]; }, [&](int i) { return skey[i] == kstar; }, &rem2);
+  }
+  __syncthreads();
+  // 5. the chosen ids, sorted ascending (bitonic, padded with 0xFFFFFFFF)
   for (int i = tid; i < sort_n; i += kSelThreads) sorted[i] = 0xFFFFFFFFu;
   __syncthreads();
   for (int i = tid; i < ns; i += kSelThreads) {

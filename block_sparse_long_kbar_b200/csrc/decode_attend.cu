@@ -44,7 +44,8 @@ namespace {
 constexpr int kTok = 128;                 // token slots per tile
 constexpr int kNQ = 64;                   // query-head columns
 constexpr int kD = 128;                   // head dim of this kernel
-constexpr int kNS = 2;                    // K/V tile stages
+constexpr int kNK = 3;                    // bf16 caches: K tile stages (free once S^T is issued)
+constexpr int kNV = 2;                    // bf16 caches: V tile stages (free once P V is issued)
 constexpr int kSmWarps = 4;
 constexpr int kThreads = (2 + kSmWarps) * 32;
 constexpr int kHalf = kTok * 128;         // one 64-dim half of a K or V tile: [128 tokens][128 B]
@@ -62,10 +63,10 @@ constexpr int kRow8 = kTok * 128;         // 8-bit K (or V) of one tile: [128 to
 constexpr int kThreads8 = (2 + kSmWarps + 4) * 32;  // fp8 caches: + 4 converter warps
 
 struct DecShared {
-  // bf16 caches: kv_full / kv_empty per K+V stage (TMA into the operand tiles). fp8 caches:
-  // st8_full / st8_empty per staging stage (TMA), k_full / k_empty and v_full / v_empty for the
-  // single K and V operand tiles (converter warps write them).
-  uint64_t kv_full[kNS], kv_empty[kNS], st8_full[kS8], st8_empty[kS8], k_full, k_empty, v_full, v_empty;
+  // bf16 caches: kf / ke per K stage and vf / ve per V stage (TMA into the operand tiles). fp8
+  // caches: st8_full / st8_empty per staging stage (TMA), k_full / k_empty and v_full / v_empty
+  // for the single K and V operand tiles (converter warps write them).
+  uint64_t kf[kNK], ke[kNK], vf[kNV], ve[kNV], st8_full[kS8], st8_empty[kS8], k_full, k_empty, v_full, v_empty;
   uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2], o_done;
   uint32_t tmem;
   volatile int abort_flag;
@@ -73,10 +74,11 @@ struct DecShared {
   float ref_part[2][kNQ];  // the own block's maxima, two halves of its tokens
   uint32_t maxkey[kNQ];    // exact maxima (order-preserving keys) for the fallback pass
 };
-// operand tiles (K and V) then, for fp8 caches, the staging ring
+// operand tiles (bf16: the K ring, then the V ring; fp8: one K and one V tile) then, for fp8
+// caches, the staging ring
 template <bool F8>
 struct DaCfg {
-  static constexpr int kOps = F8 ? kStage : kNS * kStage;
+  static constexpr int kOps = F8 ? kStage : (kNK + kNV) * kKV;
   static constexpr int kStaging = F8 ? kS8 * 2 * kRow8 : 0;
   static constexpr int kSmem = 1024 + kQ + kOps + kStaging + 2 * kP + kOnes + (int)sizeof(DecShared) + 64;
   static constexpr int kThr = F8 ? kThreads8 : kThreads;
@@ -141,9 +143,13 @@ __global__ void __launch_bounds__(DaCfg<F8>::kThr, 1)
   // do nothing (the decision is the CTA's, before any barrier or TMEM is set up)
   if (__syncthreads_or(tid == 0 && tc::grid_timed_out(a.status))) return;
   if (tid == 0) {
-    for (int i = 0; i < kNS; ++i) {
-      tc::mbar_init(&sh->kv_full[i], 1);
-      tc::mbar_init(&sh->kv_empty[i], 1);
+    for (int i = 0; i < kNK; ++i) {
+      tc::mbar_init(&sh->kf[i], 1);
+      tc::mbar_init(&sh->ke[i], 1);
+    }
+    for (int i = 0; i < kNV; ++i) {
+      tc::mbar_init(&sh->vf[i], 1);
+      tc::mbar_init(&sh->ve[i], 1);
     }
     for (int i = 0; i < kS8; ++i) {
       tc::mbar_init(&sh->st8_full[i], 1);
@@ -274,37 +280,73 @@ __global__ void __launch_bounds__(DaCfg<F8>::kThr, 1)
       // (a CTA named by the failure-detection test hook issues nothing: its issuer's first wait
       // then runs out, with no copy in flight)
       if (lane == 0 && (int)blockIdx.x != a.stall_cta) {
-        for (int i = tile0; i < tile1 && !sh->abort_flag; ++i, ++kc) {
-          const int nst = F8 ? kS8 : kNS;
-          const int st = (int)(kc % nst);
-          uint64_t* emp = F8 ? &sh->st8_empty[st] : &sh->kv_empty[st];
-          uint64_t* ful = F8 ? &sh->st8_full[st] : &sh->kv_full[st];
-          if (kc >= nst && !tc::mbar_wait(emp, (uint32_t)(((kc / nst) - 1) & 1), &sh->abort_flag, a.status)) {
-            if (!sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
-            sh->abort_flag = 1;
-            break;
+        // the tile's token coordinates, loaded together before any copy is issued
+        auto coords = [&](int i, int (&zs)[NB]) {
+#pragma unroll
+          for (int e = 0; e < NB; ++e) {
+            const int idx = i * NB + e;
+            zs[e] = idx < count ? b * a.T_kv + __ldg(ublk + idx) * B : 0x7FFFFFF0;
           }
-          if constexpr (F8) {
+        };
+        auto fail = [&]() {
+          if (!sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
+          sh->abort_flag = 1;
+        };
+        if constexpr (F8) {
+          for (int i = tile0; i < tile1 && !sh->abort_flag; ++i, ++kc) {
+            const int st = (int)(kc % kS8);
+            if (kc >= kS8 &&
+                !tc::mbar_wait(&sh->st8_empty[st], (uint32_t)(((kc / kS8) - 1) & 1), &sh->abort_flag, a.status)) {
+              fail();
+              break;
+            }
+            int zs[NB];
+            coords(i, zs);
+            uint64_t* ful = &sh->st8_full[st];
             uint8_t* dst = s8 + st * 2 * kRow8;
             tc::mbar_arrive_expect_tx(ful, main_pass ? 2 * kRow8 : kRow8);
-            for (int e = 0; e < NB; ++e) {
-              const int idx = i * NB + e;
-              const int z = idx < count ? b * a.T_kv + __ldg(ublk + idx) * B : 0x7FFFFFF0;
-              tc::tma_load_3d(dst + e * (B * 128), &map_k, ful, 0, g, z);
-              if (main_pass) tc::tma_load_3d(dst + kRow8 + e * (B * 128), &map_v, ful, 0, g, z);
-            }
-          } else {
-            uint8_t* dst = sKV + st * kStage;
-            tc::mbar_arrive_expect_tx(ful, main_pass ? kStage : kKV);
-            for (int e = 0; e < NB; ++e) {
-              const int idx = i * NB + e;
-              const int z = idx < count ? b * a.T_kv + __ldg(ublk + idx) * B : 0x7FFFFFF0;
 #pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                tc::tma_load_3d(dst + h * kHalf + e * (B * 128), &map_k, ful, h * 64, g, z);
-                if (main_pass) tc::tma_load_3d(dst + kKV + h * kHalf + e * (B * 128), &map_v, ful, h * 64, g, z);
-              }
+            for (int e = 0; e < NB; ++e) {
+              tc::tma_load_3d(dst + e * (B * 128), &map_k, ful, 0, g, zs[e]);
+              if (main_pass) tc::tma_load_3d(dst + kRow8 + e * (B * 128), &map_v, ful, 0, g, zs[e]);
             }
+          }
+        } else {
+          // K of tile i, then V of tile i - 1: a K stage frees as soon as its S^T is issued, so
+          // K runs up to three tiles ahead while V waits for the P V two tiles back
+          int zk[NB], zv[NB];
+          for (int i = tile0; i <= tile1 && !sh->abort_flag; ++i) {
+            if (i < tile1) {
+              const int st = (int)(kc % kNK);
+              if (kc >= kNK && !tc::mbar_wait(&sh->ke[st], (uint32_t)(((kc / kNK) - 1) & 1), &sh->abort_flag, a.status)) {
+                fail();
+                break;
+              }
+              coords(i, zk);
+              uint8_t* dst = sKV + st * kKV;
+              tc::mbar_arrive_expect_tx(&sh->kf[st], kKV);
+#pragma unroll
+              for (int e = 0; e < NB; ++e)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) tc::tma_load_3d(dst + h * kHalf + e * (B * 128), &map_k, &sh->kf[st], h * 64, g, zk[e]);
+              ++kc;
+            }
+            if (main_pass && i > tile0) {
+              const int st = (int)(vc % kNV);
+              if (vc >= kNV && !tc::mbar_wait(&sh->ve[st], (uint32_t)(((vc / kNV) - 1) & 1), &sh->abort_flag, a.status)) {
+                fail();
+                break;
+              }
+              uint8_t* dst = sKV + kNK * kKV + st * kKV;
+              tc::mbar_arrive_expect_tx(&sh->vf[st], kKV);
+#pragma unroll
+              for (int e = 0; e < NB; ++e)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) tc::tma_load_3d(dst + h * kHalf + e * (B * 128), &map_v, &sh->vf[st], h * 64, g, zv[e]);
+              ++vc;
+            }
+#pragma unroll
+            for (int e = 0; e < NB; ++e) zv[e] = zk[e];
           }
         }
       }
@@ -313,12 +355,14 @@ __global__ void __launch_bounds__(DaCfg<F8>::kThr, 1)
       if (lane == 0) {
         long pend = -1;
         bool first = true;
-        auto issue_pv = [&](long stage_of) -> bool {
+        auto issue_pv = [&](long) -> bool {
           const int pb = (int)(pcnt & 1);
           if (!tc::mbar_wait(&sh->p_full[pb], (uint32_t)((pcnt >> 1) & 1), &sh->abort_flag, a.status)) return false;
-          if (F8 && !tc::mbar_wait(&sh->v_full, (uint32_t)(vc & 1), &sh->abort_flag, a.status)) return false;
+          if (F8 ? !tc::mbar_wait(&sh->v_full, (uint32_t)(vc & 1), &sh->abort_flag, a.status)
+                 : !tc::mbar_wait(&sh->vf[vc % kNV], (uint32_t)((vc / kNV) & 1), &sh->abort_flag, a.status))
+            return false;
           tc::fence_after_sync();
-          const uint8_t* vbase = sKV + (F8 ? 0 : (stage_of % kNS) * kStage) + kKV;
+          const uint8_t* vbase = F8 ? sKV + kKV : sKV + kNK * kKV + (vc % kNV) * kKV;
           const uint8_t* pbase = sP + pb * kP;
 #pragma unroll
           for (int kk = 0; kk < kTok / 16; ++kk) {
@@ -329,29 +373,25 @@ __global__ void __launch_bounds__(DaCfg<F8>::kThr, 1)
             tc::mma_bf16_ss(tmem_l, d_ones, db, idesc_l, acc);
             first = false;
           }
-          if (F8) {
-            tc::mma_commit(&sh->v_empty);
-            ++vc;
-          } else {
-            tc::mma_commit(&sh->kv_empty[stage_of % kNS]);
-          }
+          tc::mma_commit(F8 ? &sh->v_empty : &sh->ve[vc % kNV]);
+          ++vc;
           tc::mma_commit(&sh->p_empty[pb]);
           ++pcnt;
           return true;
         };
         bool ok = true;
         for (int i = tile0; i < tile1 && ok && !sh->abort_flag; ++i, ++kc, ++scnt) {
-          const int st = F8 ? 0 : (int)(kc % kNS);
+          const int st = F8 ? 0 : (int)(kc % kNK);
           const int sb = (int)(scnt & 1);
-          uint64_t* kfull = F8 ? &sh->k_full : &sh->kv_full[st];
-          const uint32_t kpar = F8 ? (uint32_t)(kc & 1) : (uint32_t)((kc / kNS) & 1);
+          uint64_t* kfull = F8 ? &sh->k_full : &sh->kf[st];
+          const uint32_t kpar = F8 ? (uint32_t)(kc & 1) : (uint32_t)((kc / kNK) & 1);
           if (!tc::mbar_wait(kfull, kpar, &sh->abort_flag, a.status) ||
               (scnt >= 2 && !tc::mbar_wait(&sh->s_empty[sb], (uint32_t)(((scnt >> 1) - 1) & 1), &sh->abort_flag, a.status))) {
             ok = false;
             break;
           }
           tc::fence_after_sync();
-          const uint8_t* kst = sKV + st * kStage;
+          const uint8_t* kst = sKV + st * kKV;
 #pragma unroll
           for (int kk = 0; kk < kD / 16; ++kk) {
             const int h = kk >> 2, off = (kk & 3) * 32;
@@ -360,10 +400,8 @@ __global__ void __launch_bounds__(DaCfg<F8>::kThr, 1)
             tc::mma_bf16_ss(tmem + (uint32_t)(sb * kNQ), da, db, idesc_s, kk > 0 ? 1u : 0u);
           }
           tc::mma_commit(&sh->s_full[sb]);
-          if (F8) tc::mma_commit(&sh->k_empty);  // the K tile is free once S^T is computed
-          if (!main_pass) {
-            if (!F8) tc::mma_commit(&sh->kv_empty[st]);
-          } else {
+          tc::mma_commit(F8 ? &sh->k_empty : &sh->ke[st]);  // the K tile is free once S^T is computed
+          if (main_pass) {
             if (pend >= 0 && !issue_pv(pend)) { ok = false; break; }
             pend = kc;
           }
@@ -376,54 +414,84 @@ __global__ void __launch_bounds__(DaCfg<F8>::kThr, 1)
       }
     } else if (!is_sm) {
       // ---- fp8 converters: thread = token slot r; the staged 8-bit rows times their row
-      // scales into the bf16 K and V operand tiles (exact) ----
+      // scales into the bf16 K and V operand tiles (exact). K runs one tile ahead of V: K(i+1)
+      // needs only S^T(i) to be done with the K tile, V(i) needs P V(i-1), so the next S^T
+      // overlaps this tile's softmax. ----
       if constexpr (F8) {
         const int e = r / B;
-        for (int i = tile0; i < tile1; ++i, ++kc) {
-          const int st = (int)(kc % kS8);
-          if (!warp_wait(&sh->st8_full[st], (uint32_t)((kc / kS8) & 1), &sh->abort_flag, a.status)) {
-            if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
-            sh->abort_flag = 1;
-            break;
-          }
+        const long st_base = kc;  // staging uses before this pass
+        // (row of the cache, K scale, V scale) of a tile's token slot r
+        auto meta = [&](int i, long& srow, float& ks, float& vs) {
           const int idx = i * NB + e;
-          const long srow = idx < count ? ((long)b * a.T_kv + __ldg(ublk + idx) * B + (r % B)) * a.G + g : -1;
-          for (int part = 0; part < (main_pass ? 2 : 1); ++part) {
-            // K (part 0) is free once the previous S^T completed; V once the previous P V did
-            uint64_t* emp = part ? &sh->v_empty : &sh->k_empty;
-            const long uses = part ? vc : kc;
-            if (uses >= 1 && !warp_wait(emp, (uint32_t)((uses - 1) & 1), &sh->abort_flag, a.status)) {
-              if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
-              sh->abort_flag = 1;
-              break;
-            }
-            const float scale = srow >= 0 ? __ldg((part ? a.v_scale : a.k_scale) + srow) : 0.f;
-            const uint8_t* src = s8 + st * 2 * kRow8 + part * kRow8 + r * 128;
-            uint8_t* dst = sKV + part * kKV + r * 128;
+          srow = (i < tile1 && idx < count) ? ((long)b * a.T_kv + __ldg(ublk + idx) * B + (r % B)) * a.G + g : -1;
+          ks = srow >= 0 ? __ldg(a.k_scale + srow) : 0.f;
+          vs = (srow >= 0 && main_pass) ? __ldg(a.v_scale + srow) : 0.f;
+        };
+        auto convert = [&](int i, int part, float scale) -> bool {
+          const long use = st_base + (i - tile0);
+          const int st = (int)(use % kS8);
+          if (part == 0 &&
+              !warp_wait(&sh->st8_full[st], (uint32_t)((use / kS8) & 1), &sh->abort_flag, a.status))
+            return false;
+          uint64_t* emp = part ? &sh->v_empty : &sh->k_empty;
+          const long uses = part ? vc : kc;
+          if (uses >= 1 && !warp_wait(emp, (uint32_t)((uses - 1) & 1), &sh->abort_flag, a.status)) return false;
+          const uint8_t* src = s8 + st * 2 * kRow8 + part * kRow8 + r * 128;
+          uint8_t* dst = sKV + part * kKV + r * 128;
 #pragma unroll
-            for (int c8 = 0; c8 < 8; ++c8) {  // 16 codes = 16 dims = two 16-byte bf16 chunks
-              const uint4 w = *reinterpret_cast<const uint4*>(src + ((c8 ^ (r & 7)) * 16));
-              const uint2 x0 = e4m3x4_to_bf16(w.x, scale), x1 = e4m3x4_to_bf16(w.y, scale);
-              const uint2 x2 = e4m3x4_to_bf16(w.z, scale), x3 = e4m3x4_to_bf16(w.w, scale);
-              const int ca = 2 * c8, cb = 2 * c8 + 1;  // bf16 chunk index 0..15 over the 128 dims
-              *reinterpret_cast<uint4*>(dst + (ca >> 3) * kHalf + (((ca & 7) ^ (r & 7)) * 16)) =
-                  make_uint4(x0.x, x0.y, x1.x, x1.y);
-              *reinterpret_cast<uint4*>(dst + (cb >> 3) * kHalf + (((cb & 7) ^ (r & 7)) * 16)) =
-                  make_uint4(x2.x, x2.y, x3.x, x3.y);
-            }
-            tc::fence_proxy_async();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(part ? &sh->v_full : &sh->k_full);
-            if (part) ++vc;
+          for (int c8 = 0; c8 < 8; ++c8) {  // 16 codes = 16 dims = two 16-byte bf16 chunks
+            const uint4 w = *reinterpret_cast<const uint4*>(src + ((c8 ^ (r & 7)) * 16));
+            const uint2 x0 = e4m3x4_to_bf16(w.x, scale), x1 = e4m3x4_to_bf16(w.y, scale);
+            const uint2 x2 = e4m3x4_to_bf16(w.z, scale), x3 = e4m3x4_to_bf16(w.w, scale);
+            const int ca = 2 * c8, cb = 2 * c8 + 1;  // bf16 chunk index 0..15 over the 128 dims
+            *reinterpret_cast<uint4*>(dst + (ca >> 3) * kHalf + (((ca & 7) ^ (r & 7)) * 16)) =
+                make_uint4(x0.x, x0.y, x1.x, x1.y);
+            *reinterpret_cast<uint4*>(dst + (cb >> 3) * kHalf + (((cb & 7) ^ (r & 7)) * 16)) =
+                make_uint4(x2.x, x2.y, x3.x, x3.y);
           }
-          if (sh->abort_flag) break;
+          tc::fence_proxy_async();
           __syncwarp();
-          if (lane == 0) tc::mbar_arrive(&sh->st8_empty[st]);
+          if (lane == 0) tc::mbar_arrive(part ? &sh->v_full : &sh->k_full);
+          if (part) ++vc;
+          else ++kc;
+          return true;
+        };
+        long srow_c, srow_n;
+        float ks_c, vs_c, ks_n, vs_n;
+        meta(tile0, srow_c, ks_c, vs_c);
+        bool ok = tile0 >= tile1 || convert(tile0, 0, ks_c);
+        for (int i = tile0; ok && i < tile1; ++i) {
+          meta(i + 1, srow_n, ks_n, vs_n);  // in flight while this step waits and converts
+          if (i + 1 < tile1 && !convert(i + 1, 0, ks_n)) { ok = false; break; }
+          if (main_pass && !convert(i, 1, vs_c)) { ok = false; break; }
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&sh->st8_empty[(int)((st_base + (i - tile0)) % kS8)]);
+          srow_c = srow_n;
+          ks_c = ks_n;
+          vs_c = vs_n;
         }
+        if (!ok) {
+          if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
+          sh->abort_flag = 1;
+        }
+        kc = st_base + (tile1 - tile0);  // the staging ring position, as the producer counts it
       }
     } else {
       // ---- probabilities: thread = token slot r of the tile ----
+      // the union entry of this thread's token slot, one tile ahead
+      auto entry = [&](int i, uint32_t& qm, int& blk) {
+        const int idx = i * NB + r / B;
+        const bool in = i < tile1 && idx < count;
+        qm = in ? __ldg(umask + idx) : 0u;
+        blk = in ? __ldg(ublk + idx) : 0;
+      };
+      uint32_t qm_n;
+      int blk_n;
+      entry(tile0, qm_n, blk_n);
       for (int i = tile0; i < tile1; ++i, ++scnt) {
+        const uint32_t qm = qm_n;
+        const int blk = blk_n;
+        entry(i + 1, qm_n, blk_n);
         const int sb = (int)(scnt & 1);
         if (!warp_wait(&sh->s_full[sb], (uint32_t)((scnt >> 1) & 1), &sh->abort_flag, a.status)) {
           if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
@@ -437,11 +505,9 @@ __global__ void __launch_bounds__(DaCfg<F8>::kThr, 1)
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&sh->s_empty[sb]);
         // columns this token counts for: its block is in the query's selection and u <= t_q
-        const int idx = i * NB + r / B;
         uint64_t cm = 0;
-        if (idx < count) {
-          const uint32_t qm = __ldg(umask + idx);
-          const int u = __ldg(ublk + idx) * B + (r % B);
+        if (qm != 0u) {
+          const int u = blk * B + (r % B);
           for (int q = 0; q < a.n_new; ++q)
             if (((qm >> q) & 1u) && u <= a.t0 + q) cm |= ((R >= 64 ? ~0ull : ((1ull << R) - 1ull)) << (q * R));
         }
@@ -543,11 +609,16 @@ __global__ void __launch_bounds__(DaCfg<F8>::kThr, 1)
 
   // ---- drain and release ----
   if (warp == 0 && lane == 0) {
-    const int nst = F8 ? kS8 : kNS;
-    for (long k2 = kc - nst; k2 < kc; ++k2) {
-      if (k2 < 0) continue;
-      volatile int no_abort = 0;
-      tc::mbar_wait(F8 ? &sh->st8_full[k2 % nst] : &sh->kv_full[k2 % nst], (uint32_t)((k2 / nst) & 1), &no_abort);
+    // every copy issued lands before the CTA exits
+    volatile int no_abort = 0;
+    if constexpr (F8) {
+      for (long k2 = kc - kS8; k2 < kc; ++k2)
+        if (k2 >= 0) tc::mbar_wait(&sh->st8_full[k2 % kS8], (uint32_t)((k2 / kS8) & 1), &no_abort);
+    } else {
+      for (long k2 = kc - kNK; k2 < kc; ++k2)
+        if (k2 >= 0) tc::mbar_wait(&sh->kf[k2 % kNK], (uint32_t)((k2 / kNK) & 1), &no_abort);
+      for (long v2 = vc - kNV; v2 < vc; ++v2)
+        if (v2 >= 0) tc::mbar_wait(&sh->vf[v2 % kNV], (uint32_t)((v2 / kNV) & 1), &no_abort);
     }
   }
   if (warp == 1 && lane == 0 && o_commits > 0) {

@@ -14,9 +14,9 @@
 // at the bf16 tensor rate with fp32-accurate scores, hi products first, then lo, as in prefill.
 //
 // Pipeline (one CTA per (sequence, range of 128-candidate tiles)): warp 0 TMA-loads fp32 tiles
-// (32 KB) into a 4-stage ring; warps 2-5 convert a staged tile into the two bf16 operand planes
+// (32 KB) into a 4-stage ring; warps 2-9 convert a staged tile into the two bf16 operand planes
 // (128B-swizzled K-major, double-buffered); warp 1 allocates TMEM and issues the MMAs into two
-// accumulators; warps 6-9 (one per TMEM lane quadrant, a candidate per lane) write each row's fp32
+// accumulators; warps 10-13 (one per TMEM lane quadrant, a candidate per lane) write each row's fp32
 // scores for the candidates it has, and per row the largest order-preserving key of every 32
 // consecutive candidates (a lower bound on the row's selection threshold comes from these). Every
 // wait is bounded by %globaltimer: on expiry the kernel records SGQA_ERR_TIMEOUT, drains its
@@ -36,7 +36,8 @@ constexpr int kStg = 4;                    // fp32 staging stages
 constexpr int kStgBytes = kCand * kDI * 4; // 32 KB
 constexpr int kPlane = kCand * kDI * 2;    // one bf16 plane: 16 KB
 constexpr int kOp = 2 * kPlane;            // hi then lo
-constexpr int kThr = 10 * 32;
+constexpr int kConvWarps = 8;              // converter warps (2 .. 9); epilogue warps 10 .. 13
+constexpr int kThr = (2 + kConvWarps + 4) * 32;
 
 struct ScShared {
   uint64_t full[kStg], empty[kStg], op_full[2], op_empty[2], acc_full[2], acc_empty[2];
@@ -83,10 +84,10 @@ __global__ void __launch_bounds__(kThr, 1)
   if (tid == 0) {
     for (int s = 0; s < kStg; ++s) {
       tc::mbar_init(&sh->full[s], 1);
-      tc::mbar_init(&sh->empty[s], 4);
+      tc::mbar_init(&sh->empty[s], kConvWarps);
     }
     for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(&sh->op_full[s], 4);
+      tc::mbar_init(&sh->op_full[s], kConvWarps);
       tc::mbar_init(&sh->op_empty[s], 1);
       tc::mbar_init(&sh->acc_full[s], 1);
       tc::mbar_init(&sh->acc_empty[s], 4);
@@ -159,7 +160,7 @@ __global__ void __launch_bounds__(kThr, 1)
         tc::mbar_wait(&sh->acc_full[(k - 1) & 1], (uint32_t)(((k - 1) >> 1) & 1), &no_abort);
       }
     }
-  } else if (warp < 6) {
+  } else if (warp < 2 + kConvWarps) {
     // ---- converters: fp32 tile -> bf16 hi and lo planes (128B-swizzled K-major rows) ----
     const int ct = tid - 64;
     for (int k = 0; k < n; ++k) {
@@ -172,21 +173,18 @@ __global__ void __launch_bounds__(kThr, 1)
       }
       const float4* src = reinterpret_cast<const float4*>(sStg + st * kStgBytes);
       uint8_t* hi = sOp + op * kOp;
-#pragma unroll 4
-      for (int e = 0; e < kCand * kDI / 4 / 128; ++e) {
-        const int idx = ct + 128 * e;
+#pragma unroll
+      for (int e = 0; e < kCand * kDI / 4 / (32 * kConvWarps); ++e) {
+        const int idx = ct + 32 * kConvWarps * e;
         const int row = idx >> 4, c4 = idx & 15;
         const float4 f = src[idx];
-        const float x[4] = {f.x, f.y, f.z, f.w};
-        uint32_t h[4], l[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          h[i] = f32_to_bf16_rne(x[i]);
-          l[i] = f32_to_bf16_rne(x[i] - bf16_to_f32((uint16_t)h[i]));
-        }
+        // hi = bf16(x) two at a time; lo = bf16(x - hi), where x - hi is exact in fp32
+        const uint32_t h01 = pack_bf16x2(f.x, f.y), h23 = pack_bf16x2(f.z, f.w);
+        const uint32_t l01 = pack_bf16x2(f.x - bf16_lo(h01), f.y - bf16_hi(h01));
+        const uint32_t l23 = pack_bf16x2(f.z - bf16_lo(h23), f.w - bf16_hi(h23));
         const int off = row * 128 + (((c4 >> 1) ^ (row & 7)) * 16) + (c4 & 1) * 8;
-        *reinterpret_cast<uint2*>(hi + off) = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
-        *reinterpret_cast<uint2*>(hi + kPlane + off) = make_uint2(l[0] | (l[1] << 16), l[2] | (l[3] << 16));
+        *reinterpret_cast<uint2*>(hi + off) = make_uint2(h01, h23);
+        *reinterpret_cast<uint2*>(hi + kPlane + off) = make_uint2(l01, l23);
       }
       tc::fence_proxy_async();
       __syncwarp();
@@ -200,6 +198,12 @@ __global__ void __launch_bounds__(kThr, 1)
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
+    // per row: the own block (candidates are j < c_row), hoisted out of the tile loop
+    int c_row[NR];
+#pragma unroll
+    for (int rr = 0; rr < NR; ++rr) c_row[rr] = rr < rows ? (a.t0 + rr / a.G) / a.B : 0;
+    float* sbase = a.scores + (long)b * rows * a.nblk;
+    uint32_t* tbase = a.tmax + (long)b * rows * a.tstride;
     for (int k = 0; k < n; ++k) {
       const int acc = k & 1;
       if (!warp_wait(&sh->acc_full[acc], (uint32_t)((k >> 1) & 1), &sh->abort_flag, a.status)) {
@@ -217,16 +221,14 @@ __global__ void __launch_bounds__(kThr, 1)
       const int j = (i0 + k) * kCand + r;
       const int j_warp = j - lane;
       if (j_warp >= c_max) continue;  // warp-uniform
+      const bool in_range = j < c_max;
 #pragma unroll
       for (int rr = 0; rr < NR; ++rr) {
         if (rr >= rows) break;
         const float s = __uint_as_float(v[rr]);
-        const long row = (long)b * rows + rr;
-        if (j < c_max) a.scores[row * a.nblk + j] = s;
-        const int c_row = (a.t0 + rr / a.G) / a.B;
-        const uint32_t key = j < c_row ? score_key(s) : 0u;
-        const uint32_t wmax = __reduce_max_sync(0xFFFFFFFFu, key);
-        if (lane == 0) a.tmax[row * a.tstride + (j_warp >> 5)] = wmax;
+        if (in_range) sbase[rr * a.nblk + j] = s;
+        const uint32_t wmax = __reduce_max_sync(0xFFFFFFFFu, j < c_row[rr] ? score_key(s) : 0u);
+        if (lane == 0) tbase[rr * a.tstride + (j_warp >> 5)] = wmax;
       }
     }
   }

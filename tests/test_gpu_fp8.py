@@ -3,7 +3,7 @@
 * quantization: codes and row scales bit-exact against the oracle's quantizer (its e4m3
   rounding is pinned against torch's float8_e4m3fn cast in test_oracle_fp8_pins.py);
 * a decode step over FP8 caches: the caches it appends to equal the oracle's quantization of the
-  whole sequence, bit for bit; the selection equals sgqa_decode's on the bf16 caches (the index
+  sequence, bit for bit (on the new rows, every token the step attends to and a seeded sample); the selection equals sgqa_decode's on the bf16 caches (the index
   keys are not quantized); outputs match the oracle's attention over the dequantized values
   (exact in bf16) within max-abs 1e-2 / mean-abs 1e-3;
 * the 1M-context decode workload on sampled sequences.
@@ -100,22 +100,33 @@ def _fp8_decode_case(cfg, cache_len, n_new, check_seqs, compare_bf16=True):
     assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
     Tn = cache_len + n_new
     dm = oracle.dims(1, Tn, cfg.Hq, cfg.G, cfg.d, cfg.d_idx, cfg.B, cfg.k)
+    rng = np.random.default_rng(cfg.seed)
     errs = []
     for b in check_seqs:
-        t_all = np.arange(Tn)
-        kq, ks = oracle.quantize_fp8(gen_rows(cfg, "k", b, t_all).reshape(Tn, cfg.G, cfg.d))
-        vq, vs = oracle.quantize_fp8(gen_rows(cfg, "v", b, t_all).reshape(Tn, cfg.G, cfg.d))
-        np.testing.assert_array_equal(_u8(c8["k"][b, :Tn]), kq)
-        np.testing.assert_array_equal(_u8(c8["v"][b, :Tn]), vq)
-        np.testing.assert_array_equal(csc["k"][b, :Tn].cpu().numpy().astype(np.float64), ks)
-        np.testing.assert_array_equal(csc["v"][b, :Tn].cpu().numpy().astype(np.float64), vs)
-        kh = _dequant_bf16_bits(kq, ks).reshape(1, Tn, cfg.G, cfg.d)
-        vh = _dequant_bf16_bits(vq, vs).reshape(1, Tn, cfg.G, cfg.d)
+        gsel = sel[b].cpu().numpy()
+        # the tokens the step attends to (every group's selection), the new rows, and a sample
+        blocks = np.unique(gsel[gsel >= 0])
+        toks = (blocks[:, None] * cfg.B + np.arange(cfg.B)[None, :]).ravel()
+        toks = toks[toks < Tn]
+        sample = rng.integers(0, Tn, size=min(2048, Tn))
+        check = np.unique(np.concatenate([toks, np.arange(cache_len, Tn), sample]))
+        ti = torch.from_numpy(check.astype(np.int64)).cuda()
+        got = {n: (_u8(c8[n][b].index_select(0, ti)), csc[n][b].index_select(0, ti).cpu().numpy().astype(np.float64))
+               for n in ("k", "v")}
+        # the caches hold exactly the oracle's quantization of the sequence (checked rows)
+        for n in ("k", "v"):
+            q, sc_ = oracle.quantize_fp8(gen_rows(cfg, n, b, check).reshape(len(check), cfg.G, cfg.d))
+            np.testing.assert_array_equal(got[n][0], q)
+            np.testing.assert_array_equal(got[n][1], sc_)
+        # the oracle attends over the dequantized values (exact in bf16) of the tokens it needs
+        kh = np.zeros((1, Tn, cfg.G, cfg.d), dtype=np.uint16)
+        vh = np.zeros((1, Tn, cfg.G, cfg.d), dtype=np.uint16)
+        kh[0, check] = _dequant_bf16_bits(*got["k"])
+        vh[0, check] = _dequant_bf16_bits(*got["v"])
         kbar64 = oracle.compress(dm, to_host(kidx[b:b + 1, :Tn]))
         rows = np.array([[0, cache_len + i] for i in range(n_new)], dtype=np.int32)
         qi = to_host(new["q_idx"][b]).reshape(n_new, -1)
         sel_o, s_m, _ = oracle.select(dm, kbar64, rows, qi)
-        gsel = sel[b].cpu().numpy()
         compare_selection(dm, kbar64, rows, qi, gsel, sel_o, s_m)
         ref = oracle.attend(dm, rows, to_host(new["q"][b]).reshape(n_new, -1), kh, vh,
                             to_host(new["gate"][b]).reshape(n_new, -1), gsel)
