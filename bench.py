@@ -7,7 +7,9 @@ resident in HBM (q, gate and out alone are 3.2 GB, far above the 126 MB L2, so n
 needed between steps). Launch:
 
     python bench.py [--gpus 1] [--steps 5] [--warmup 3]
-    python -m torch.distributed.run --nproc-per-node N ... bench.py --gpus N ...   (one sequence per rank)
+    python -m torch.distributed.run --nproc-per-node N ... bench.py --gpus N ...
+        (N > 1: the 128K sequence split over the GPUs by query, K/V/k_idx all-gathered over NCCL;
+         decode: the 32 sequences split over the GPUs)
     python bench.py --impl reference ...   (the fp64 CPU oracle on a bounded sample, host cores)
 
 Rank 0 prints one JSON line.
@@ -402,11 +404,125 @@ def run_ours(args, world, rank):
     return result
 
 
+def run_sharded(args, world, rank):
+    """N > 1: one 128K sequence split over the GPUs by query (zig-zag ranges), K, V and k_idx
+    all-gathered over NCCL every step (each rank produces those of its own rows), then the layer
+    for the rank's rows (sgqa_forward_rows). Strong scaling: the whole job is one sequence."""
+    import torch
+    import block_sparse_long_kbar_b200 as sg
+    from block_sparse_long_kbar_b200.sharding import gather_sequence, prefill_rows, zigzag_ranges
+    from sgqa_inputs import gen_device
+    cfg = CONFIGS[args.config]
+    dims = sg.sgqa_dims.of(cfg)
+    s = torch.cuda.Stream()
+    ranges = zigzag_ranges(cfg.T, world, rank)
+    loc = {}
+    for n in ("q", "gate", "q_idx", "k", "v", "k_idx"):
+        loc[n] = []
+        for t0, t1 in ranges:
+            x = torch.empty(cfg.shape(n, T=t1 - t0), dtype=torch.bfloat16, device="cuda")
+            gen_device(cfg, n, x, t0=t0, n_t=t1 - t0, dst_t0=0)
+            loc[n].append(x)
+    outs = [torch.empty_like(x) for x in loc["q"]]
+    ws = sg.alloc_workspace(sg.sgqa_workspace_size(dims))
+    sg.sgqa_reset_device_status(ws)
+    torch.cuda.synchronize()
+
+    def gather():
+        return [gather_sequence(loc[n], world) for n in ("k", "v", "k_idx")]
+
+    def step():
+        k, v, k_idx = gather()
+        prefill_rows(dims, ranges, loc["q"], loc["gate"], loc["q_idx"], k, v, k_idx, outs, ws, stream=s)
+
+    with torch.cuda.stream(s):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    bus = getattr(torch.cuda.get_device_properties(torch.cuda.current_device()), "pci_bus_id", None)
+    sampler = ClockSampler(bus)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        e0.record(s)
+        for _ in range(args.steps):
+            step()
+        e1.record(s)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    assert sg.sgqa_get_device_status(ws) == 0
+    # the all-gather alone
+    with torch.cuda.stream(s):
+        e0.record(s)
+        for _ in range(args.steps):
+            gather()
+        e1.record(s)
+    torch.cuda.synchronize()
+    gather_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    # end to end: this rank's rows from pinned host buffers, the output back
+    host = {n: [torch.empty(x.shape, dtype=torch.bfloat16, pin_memory=True).copy_(x) for x in loc[n]] for n in loc}
+    out_h = [torch.empty(o.shape, dtype=torch.bfloat16, pin_memory=True) for o in outs]
+    h2d = sum(x.numel() * 2 for xs in host.values() for x in xs)
+    d2h = sum(o.numel() * 2 for o in outs)
+
+    def e2e_step():
+        for n in loc:
+            for dst, src in zip(loc[n], host[n]):
+                dst.copy_(src, non_blocking=True)
+        step()
+        for dst, src in zip(out_h, outs):
+            dst.copy_(src, non_blocking=True)
+
+    with torch.cuda.stream(s):
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0.record(s)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(s)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    wc = work_counts(cfg)
+    peaks = load_peaks()
+    per_gpu_flops = (wc["attn_flops"] + wc["index_flops"]) / world
+    result = {
+        "metric": METRIC, "value": cfg.batch * cfg.T / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded topic-structured generator)",
+        "config": {"workload": f"prefill {cfg.name}: batch {cfg.batch}, T={cfg.T}, Hq={cfg.Hq}, G={cfg.G}, "
+                               f"d={cfg.d}, d_idx={cfg.d_idx}, B={cfg.B}, k={cfg.k}, topic span {cfg.span}, "
+                               f"seed {cfg.seed}; queries split over {world} GPUs",
+                   "global_batch": cfg.batch, "seq_len": cfg.T,
+                   "parallelism": f"query-sharded x{world} (zig-zag ranges; all-gather of K, V, k_idx over NCCL)",
+                   "l2": "inputs larger than L2, no flush"},
+        "gpu_launches": 13 * 2 * args.steps,
+        "e2e": {"value": cfg.batch * cfg.T / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "roofline": {"bound": "tensor", "achieved": per_gpu_flops / (ms / 1e3) / 1e12, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": per_gpu_flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+                     "traffic": None, "kernel": "whole step per GPU (indexer + attention flops / N)",
+                     "peak_source": peaks["source"]},
+        "allgather_ms": gather_ms,
+        "clocks": clocks,
+    }
+    del loc, outs, ws, host, out_h
+    torch.cuda.empty_cache()
+    if not args.no_decode:
+        result["decode"] = run_decode(args, world, s)
+    return result
+
+
 def run_decode(args, world, s):
     import torch
     import block_sparse_long_kbar_b200 as sg
     from sgqa_inputs import gen_device
     cfg = CONFIGS["decode_1m"]
+    if world > 1:  # the 32 sequences split over the GPUs (data parallel, no exchange)
+        cfg = cfg.replace(batch=cfg.batch // world)
     shape_of = lambda c, n, **kw: c.shape(n, **kw)
     n_new = DECODE_NEW
     cache_len = cfg.T
@@ -450,7 +566,7 @@ def run_decode(args, world, s):
     gather = visits * 2 * cfg.d * 2
     res = {"metric": "decode query tokens/s at 1M context (32 seqs x 4 new tokens)", "value": toks / (ms / 1e3),
            "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
-           "workload": f"decode: {cfg.batch} seqs x {n_new} new tokens after {cache_len} cached, Hq={cfg.Hq}, "
+           "workload": f"decode: {cfg.batch} seqs per GPU x {n_new} new tokens after {cache_len} cached, Hq={cfg.Hq}, "
                        f"G={cfg.G}, d={cfg.d}, d_idx={cfg.d_idx}, B={cfg.B}, k={cfg.k}, span {cfg.span}, seed {cfg.seed}",
            "algorithmic_bytes": kbar_bytes + gather,
            "hbm_frac": (kbar_bytes + gather) / (ms / 1e3) / 1e9 / load_peaks()["hbm_gbs"],
@@ -776,6 +892,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-swa", action="store_true")
     ap.add_argument("--no-ablation", action="store_true")
+    ap.add_argument("--query-sharded", action="store_true",
+                    help="split the sequence's queries over the ranks even at N = 1 (the N > 1 path)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -788,7 +906,8 @@ def main():
         return
     world, rank, _ = dist_setup(args.gpus)
     try:
-        res = run_ours(args, world, rank)
+        sharded = world > 1 or args.query_sharded
+        res = run_sharded(args, world, rank) if sharded else run_ours(args, world, rank)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

@@ -27,7 +27,7 @@ STATUS_NAMES = {0: "SGQA_OK", 1: "SGQA_ERR_INVALID_ARG", 2: "SGQA_ERR_UNSUPPORTE
 EXPORTS = ["sgqa_status_string", "sgqa_version", "sgqa_workspace_size", "sgqa_decode_workspace_size",
            "sgqa_reset_device_status", "sgqa_get_device_status", "sgqa_compress_keys", "sgqa_select",
            "sgqa_attend", "sgqa_forward", "sgqa_decode", "sgqa_decode_noalloc", "sgqa_gated_swa",
-           "sgqa_quantize_kv_fp8", "sgqa_decode_fp8", "sgqa_test_stall_decode_cta"]
+           "sgqa_quantize_kv_fp8", "sgqa_decode_fp8", "sgqa_test_stall_decode_cta", "sgqa_forward_rows"]
 
 
 class SgqaError(RuntimeError):
@@ -78,9 +78,10 @@ def load_library():
     L.sgqa_quantize_kv_fp8.argtypes = [D, I, I, P, P, P, P]
     L.sgqa_decode_fp8.argtypes = [D, I, I] + [P] * 15 + [S, P]
     L.sgqa_test_stall_decode_cta.argtypes = [I]
+    L.sgqa_forward_rows.argtypes = [D, I, I, P, P, P, P, P, P, P, P, P, S, P]
     for n in ("sgqa_reset_device_status", "sgqa_get_device_status", "sgqa_compress_keys", "sgqa_select",
               "sgqa_attend", "sgqa_forward", "sgqa_decode", "sgqa_decode_noalloc", "sgqa_gated_swa",
-              "sgqa_quantize_kv_fp8", "sgqa_decode_fp8", "sgqa_test_stall_decode_cta"):
+              "sgqa_quantize_kv_fp8", "sgqa_decode_fp8", "sgqa_test_stall_decode_cta", "sgqa_forward_rows"):
         getattr(L, n).restype = I
     _lib = L
     return L
@@ -175,6 +176,16 @@ def sgqa_forward(dims, q, k, v, q_idx, k_idx, gate, out, ws, sel_out=None, strea
         ctypes.byref(dims), _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _ptr(q_idx, "q_idx"), _ptr(k_idx, "k_idx"),
         _ptr(gate, "gate"), _ptr(out, "out"), _ptr(sel_out, "sel_out"), _ptr(ws, "ws"), ws.numel(),
         _stream(stream)))
+
+
+def sgqa_forward_rows(dims, t_begin, t_end, q_rows, k, v, q_idx_rows, k_idx, gate_rows, out_rows, ws,
+                      sel_out_rows=None, stream=None):
+    """The layer for query rows [t_begin, t_end) only (q, gate, q_idx, out hold those rows; k, v,
+    k_idx whole sequences): the per-GPU unit of a query-sharded prefill."""
+    _check("sgqa_forward_rows", load_library().sgqa_forward_rows(
+        ctypes.byref(dims), int(t_begin), int(t_end), _ptr(q_rows, "q_rows"), _ptr(k, "k"), _ptr(v, "v"),
+        _ptr(q_idx_rows, "q_idx_rows"), _ptr(k_idx, "k_idx"), _ptr(gate_rows, "gate_rows"), _ptr(out_rows, "out_rows"),
+        _ptr(sel_out_rows, "sel_out_rows"), _ptr(ws, "ws"), ws.numel(), _stream(stream)))
 
 
 def sgqa_decode(dims, cache_len, n_new, k_cache, v_cache, kidx_cache, kbar_cache, q_new, k_new, v_new, qidx_new,

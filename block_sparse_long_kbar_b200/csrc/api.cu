@@ -206,7 +206,7 @@ int sgqa_select(const sgqa_dims* dims, const uint16_t* q_idx, const float* kbar,
     return SGQA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   SelectArgs a{};
-  a.q_idx = q_idx; a.kbar = kbar; a.kbar_hi = w.hi; a.kbar_lo = w.lo; a.sel = sel;
+  a.q_idx = q_idx; a.q_T = dims->T; a.q_t0 = 0; a.kbar = kbar; a.kbar_hi = w.hi; a.kbar_lo = w.lo; a.sel = sel;
   a.batch = dims->batch; a.T = dims->T; a.G = dims->G; a.d_idx = dims->d_idx; a.B = dims->B;
   a.Kb = dims->k / dims->B; a.t_begin = 0; a.t_end = dims->T; a.sel_T = dims->T; a.sel_t0 = 0;
   a.status = w.status;
@@ -238,37 +238,58 @@ int sgqa_attend(const sgqa_dims* dims, const uint16_t* q, const uint16_t* k, con
   return cuda_status(launch_prefill_attend(a, w.plan, static_cast<cudaStream_t>(stream)));
 }
 
-int sgqa_forward(const sgqa_dims* dims, const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                 const uint16_t* q_idx, const uint16_t* k_idx, const uint16_t* gate, uint16_t* out,
-                 int32_t* sel_out, void* ws, size_t ws_bytes, void* stream) {
+// The layer for query rows [t_begin, t_end) of every sequence: q, gate, q_idx, out (and sel_out)
+// hold those rows only; k, v, k_idx hold whole sequences.
+static int forward_rows_impl(const sgqa_dims* dims, int t_begin, int t_end, const uint16_t* q, const uint16_t* k,
+                             const uint16_t* v, const uint16_t* q_idx, const uint16_t* k_idx, const uint16_t* gate,
+                             uint16_t* out, int32_t* sel_out, void* ws, size_t ws_bytes, void* stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
+  if (t_begin < 0 || t_end > dims->T || t_begin > t_end) return SGQA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_idx) || !aligned16(k_idx) ||
       !aligned16(gate) || !aligned16(out) || (sel_out && !aligned16(sel_out)))
     return SGQA_ERR_INVALID_ARG;
   const PrefillWs w = prefill_layout(dims, ws);
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < w.bytes) return SGQA_ERR_WORKSPACE;
+  if (t_end == t_begin) return SGQA_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int nq = t_end - t_begin;
   if (launch_compress(k_idx, w.kbar, w.hi, w.lo, dims->batch, dims->T, dims->d_idx, dims->B, 0, dims->T / dims->B,
                       s) != cudaSuccess)
     return SGQA_ERR_CUDA;
   SelectArgs sa{};
-  sa.q_idx = q_idx; sa.kbar = w.kbar; sa.kbar_hi = w.hi; sa.kbar_lo = w.lo;
+  sa.q_idx = q_idx; sa.q_T = nq; sa.q_t0 = t_begin; sa.kbar = w.kbar; sa.kbar_hi = w.hi; sa.kbar_lo = w.lo;
   sa.batch = dims->batch; sa.T = dims->T; sa.G = dims->G; sa.d_idx = dims->d_idx; sa.B = dims->B;
   sa.Kb = dims->k / dims->B; sa.status = w.status;
   AttendArgs aa = prefill_attend_args(dims, q, k, v, gate, out, w.status);
-  const int chunk = sel_out ? dims->T : (dims->T < kSelChunkT ? dims->T : kSelChunkT);
-  for (int t0 = 0; t0 < dims->T; t0 += chunk) {
-    const int t1 = t0 + chunk < dims->T ? t0 + chunk : dims->T;
+  aa.nQ = nq; aa.q_t0 = t_begin;
+  const int chunk = sel_out ? nq : (nq < kSelChunkT ? nq : kSelChunkT);
+  for (int t0 = t_begin; t0 < t_end; t0 += chunk) {
+    const int t1 = t0 + chunk < t_end ? t0 + chunk : t_end;
     sa.sel = sel_out ? sel_out : w.sel;
-    sa.sel_T = sel_out ? dims->T : chunk;
-    sa.sel_t0 = sel_out ? 0 : t0;
+    sa.sel_T = sel_out ? nq : chunk;
+    sa.sel_t0 = sel_out ? t_begin : t0;
     sa.t_begin = t0; sa.t_end = t1;
     if (launch_select(sa, s) != cudaSuccess) return SGQA_ERR_CUDA;
     aa.sel = sa.sel; aa.sel_T = sa.sel_T; aa.sel_t0 = sa.sel_t0; aa.t_begin = t0; aa.t_end = t1;
     if (launch_prefill_attend(aa, w.plan, s) != cudaSuccess) return SGQA_ERR_CUDA;
   }
   return SGQA_OK;
+}
+
+int sgqa_forward(const sgqa_dims* dims, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                 const uint16_t* q_idx, const uint16_t* k_idx, const uint16_t* gate, uint16_t* out,
+                 int32_t* sel_out, void* ws, size_t ws_bytes, void* stream) {
+  if (!dims) return SGQA_ERR_INVALID_ARG;
+  return forward_rows_impl(dims, 0, dims->T, q, k, v, q_idx, k_idx, gate, out, sel_out, ws, ws_bytes, stream);
+}
+
+int sgqa_forward_rows(const sgqa_dims* dims, int t_begin, int t_end, const uint16_t* q_rows, const uint16_t* k,
+                      const uint16_t* v, const uint16_t* q_idx_rows, const uint16_t* k_idx,
+                      const uint16_t* gate_rows, uint16_t* out_rows, int32_t* sel_out_rows, void* ws,
+                      size_t ws_bytes, void* stream) {
+  return forward_rows_impl(dims, t_begin, t_end, q_rows, k, v, q_idx_rows, k_idx, gate_rows, out_rows, sel_out_rows,
+                           ws, ws_bytes, stream);
 }
 
 int sgqa_gated_swa(const sgqa_dims* dims, int window, const uint16_t* q, const uint16_t* k, const uint16_t* v,

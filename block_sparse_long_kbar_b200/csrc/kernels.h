@@ -15,10 +15,12 @@ cudaError_t launch_compress(const uint16_t* k_idx, float* kbar, uint16_t* hi, ui
 cudaError_t launch_split_planes(const float* kbar, uint16_t* hi, uint16_t* lo, long n, cudaStream_t s);
 
 // K2: block selection for query rows t in [t_begin, t_end) of every sequence.
-//   q_idx [batch, T, G, d_idx]; kbar [batch, T/B, d_idx] fp32;
+//   q_idx rows (b, t) at ((b * q_T + (t - q_t0)) * G + g) * d_idx (q_T = T, q_t0 = 0 for whole
+//   sequences); kbar [batch, T/B, d_idx] fp32;
 //   sel rows (b, t) at sel + ((b * sel_T + (t - sel_t0)) * G + g) * Kb.
 struct SelectArgs {
   const uint16_t* q_idx;
+  int q_T, q_t0;
   const float* kbar;
   const uint16_t* kbar_hi;
   const uint16_t* kbar_lo;

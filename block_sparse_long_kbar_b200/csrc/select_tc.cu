@@ -351,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::prefetch_tensormap(&map_hi);
       tc::prefetch_tensormap(&map_lo);
       tc::mbar_arrive_expect_tx(&sh->a_full, C::kA);
-      tc::tma_load_2d(sA, &map_q, &sh->a_full, 0, (int)(((long)b * a.T + tq0) * G));
+      tc::tma_load_2d(sA, &map_q, &sh->a_full, 0, (int)(((long)b * a.q_T + (tq0 - a.q_t0)) * G));
       long k = 0;
       bool ok = true;
       for (int pass = 0; ok && pass < kMaxPasses; ++pass) {
@@ -690,7 +690,7 @@ cudaError_t launch_di(const SelectArgs& a, cudaStream_t s) {
   using C = SelCfg<DI>;
   const int nblk = a.T / a.B;
   CUtensorMap mq, mh, ml;
-  if (!make_map(&mq, a.q_idx, (long)a.batch * a.T * a.G, DI, kRows) ||
+  if (!make_map(&mq, a.q_idx, (long)a.batch * a.q_T * a.G, DI, kRows) ||
       !make_map(&mh, a.kbar_hi, (long)a.batch * nblk, DI, kN) || !make_map(&ml, a.kbar_lo, (long)a.batch * nblk, DI, kN))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(select_tc_kernel<DI>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);

@@ -125,6 +125,19 @@ int sgqa_forward(const sgqa_dims* dims, const uint16_t* q, const uint16_t* k, co
                  const uint16_t* q_idx, const uint16_t* k_idx, const uint16_t* gate,
                  uint16_t* out, int32_t* sel_out, void* ws, size_t ws_bytes, void* stream);
 
+/* The layer for query rows [t_begin, t_end) of every sequence only: the unit of work when the
+ * queries of one sequence are split over several GPUs (each GPU holds the whole sequence's k, v
+ * and k_idx, gathered from all GPUs, and its own rows of q, gate and q_idx). The rows' results
+ * are bit-identical to the same rows of sgqa_forward.
+ *   q_rows, gate_rows, out_rows [batch, t_end - t_begin, Hq, d]; q_idx_rows [batch, t_end -
+ *   t_begin, G, d_idx]; sel_out_rows (optional) [batch, t_end - t_begin, G, k/B];
+ *   k, v [batch, T, G, d], k_idx [batch, T, d_idx] (whole sequences).
+ * 0 <= t_begin <= t_end <= T (else SGQA_ERR_INVALID_ARG); ws as for sgqa_forward. */
+int sgqa_forward_rows(const sgqa_dims* dims, int t_begin, int t_end, const uint16_t* q_rows,
+                      const uint16_t* k, const uint16_t* v, const uint16_t* q_idx_rows,
+                      const uint16_t* k_idx, const uint16_t* gate_rows, uint16_t* out_rows,
+                      int32_t* sel_out_rows, void* ws, size_t ws_bytes, void* stream);
+
 /* One decode step for dims.batch sequences sharing one cache length.
  * Caches (dims.T = capacity): k_cache, v_cache [batch, T, G, d], kidx_cache [batch, T, d_idx]
  * bf16, kbar_cache [batch, T/B, d_idx] fp32 holding the block means of every block complete in
