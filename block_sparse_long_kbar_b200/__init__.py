@@ -188,6 +188,48 @@ def sgqa_forward_rows(dims, t_begin, t_end, q_rows, k, v, q_idx_rows, k_idx, gat
         _ptr(sel_out_rows, "sel_out_rows"), _ptr(ws, "ws"), ws.numel(), _stream(stream)))
 
 
+INPUTS = ("q", "k", "v", "q_idx", "k_idx", "gate")
+
+
+def sgqa_forward_from_host(dims, host, dev, out_host, ws, chunks=8, streams=None):
+    """The whole layer (sgqa_forward's result) from pinned host buffers, with the host<->device
+    copies overlapped with the computation.
+
+    host: pinned CPU tensors q, k, v, q_idx, k_idx, gate in their natural layouts; dev: device
+    tensors of the same shapes (the staging copies) plus dev["out"]; out_host: pinned CPU tensor
+    for the output. The layer is causal, so the query rows [t0, t1) of a chunk need only the first
+    t1 rows of k, v and k_idx: for every sequence and every chunk of rows, in order, one stream
+    copies the chunk's rows of all inputs, the compute stream runs sgqa_forward_rows on the chunk
+    once they have landed, and a third stream copies the chunk's output back while later chunks
+    run. The outputs are bit-identical to sgqa_forward's. streams = (h2d, compute, d2h); by default
+    two new streams around the current one. The compute stream waits for the last copy back."""
+    import torch
+    h2d, comp, d2h = streams if streams is not None else (torch.cuda.Stream(), torch.cuda.current_stream(),
+                                                           torch.cuda.Stream())
+    T, B = dims.T, dims.B
+    one = sgqa_dims(1, T, dims.Hq, dims.G, dims.d, dims.d_idx, dims.B, dims.k)
+    h2d.wait_stream(comp)  # the device inputs may still be in use by work queued before this call
+    step = max(B, ((T + chunks - 1) // chunks + 127) // 128 * 128)
+    bounds = list(range(0, T, step)) + [T]
+    for b in range(dims.batch):
+        for t0, t1 in zip(bounds[:-1], bounds[1:]):
+            with torch.cuda.stream(h2d):
+                for n in INPUTS:
+                    dev[n][b, t0:t1].copy_(host[n][b, t0:t1], non_blocking=True)
+                ready = torch.cuda.Event()
+                ready.record(h2d)
+            comp.wait_event(ready)
+            sgqa_forward_rows(one, t0, t1, dev["q"][b, t0:t1], dev["k"][b], dev["v"][b], dev["q_idx"][b, t0:t1],
+                              dev["k_idx"][b], dev["gate"][b, t0:t1], dev["out"][b, t0:t1], ws, stream=comp)
+            done = torch.cuda.Event()
+            done.record(comp)
+            d2h.wait_event(done)
+            with torch.cuda.stream(d2h):
+                out_host[b, t0:t1].copy_(dev["out"][b, t0:t1], non_blocking=True)
+    comp.wait_stream(d2h)
+    comp.wait_stream(h2d)
+
+
 def sgqa_decode(dims, cache_len, n_new, k_cache, v_cache, kidx_cache, kbar_cache, q_new, k_new, v_new, qidx_new,
                 kidx_new, gate_new, out, ws, sel_out=None, stream=None):
     _check("sgqa_decode", load_library().sgqa_decode(

@@ -45,3 +45,27 @@ def test_query_sharded_prefill_equals_single_gpu_forward(cfg, world):
     assert sg.sgqa_get_device_status(ws) == 0
     assert torch.equal(sel_s, sel)
     assert torch.equal(out_s.view(torch.int16), out.view(torch.int16))
+
+
+def test_forward_from_host_equals_forward():
+    """The host-buffer entry point (chunked copies overlapped with sgqa_forward_rows) gives
+    sgqa_forward's bits, for two sequences and a ragged last chunk."""
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    cfg = Config("from_host", 2, 3000, 32, 4, 128, 64, 8, 512, 400, 63)
+    dims = sg.sgqa_dims.of(cfg)
+    d = device_inputs(cfg)
+    ws = sg.alloc_workspace(sg.sgqa_workspace_size(dims))
+    sg.sgqa_reset_device_status(ws)
+    out = torch.empty(cfg.shape("q"), dtype=torch.bfloat16, device="cuda")
+    sg.sgqa_forward(dims, d["q"], d["k"], d["v"], d["q_idx"], d["k_idx"], d["gate"], out, ws)
+    host = {n: torch.empty(d[n].shape, dtype=torch.bfloat16, pin_memory=True).copy_(d[n]) for n in d}
+    dev = {n: torch.zeros_like(d[n]) for n in d}
+    dev["out"] = torch.zeros_like(out)
+    out_h = torch.empty(out.shape, dtype=torch.bfloat16, pin_memory=True)
+    for _ in range(2):
+        out_h.zero_()
+        sg.sgqa_forward_from_host(dims, host, dev, out_h, ws, chunks=5)
+        torch.cuda.synchronize()
+        assert sg.sgqa_get_device_status(ws) == 0
+        assert torch.equal(out_h.view(torch.int16), out.cpu().view(torch.int16))
