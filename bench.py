@@ -42,9 +42,17 @@ CLOCK_FIELDS = ["pci.bus_id", "clocks.sm", "clocks.max.sm", "power.draw", "clock
 # kernels, keyed by (stage, workload), each with the SHA-256 (first 16 hex digits) of the kernel's
 # source file at capture time: an entry is reported only while that source is unchanged, else the
 # traffic is null. The figures and the commands that produced them are under profiles/.
-NCU_TRAFFIC: dict = {}
+NCU_TRAFFIC: dict = {
+    # profiles/traffic_prefill128k_decode1m.md: one launch each, the bench's own 128K / 1M workloads
+    ("attend", "128k"): (6576556544 + 1069653760, "8545fe13f12f383c"),
+    ("select", "128k"): (76668928 + 1018871040, "1adee091c006784c"),
+    ("decode_scores", "decode_1m"): (1074586880 + 255890688, "99064a99bc73bfeb"),
+    ("decode_select", "decode_1m"): (509419776 + 123904, "6b1e39bfc032a2cd"),
+    ("decode_attend", "decode_1m"): (1073816064 + 169472, "f2a6bae20073fbb6"),
+}
 STAGE_SOURCES = {"compress": "compress.cu", "select": "select_tc.cu", "attend": "attend_tc.cu",
-                 "decode_scores": "decode.cu", "decode_attend": "decode_attend.cu"}
+                 "decode_scores": "decode_scores_tc.cu", "decode_select": "decode.cu",
+                 "decode_attend": "decode_attend.cu"}
 
 
 def source_sha(stage: str) -> str | None:
@@ -569,6 +577,8 @@ def run_decode(args, world, s):
                        f"G={cfg.G}, d={cfg.d}, d_idx={cfg.d_idx}, B={cfg.B}, k={cfg.k}, span {cfg.span}, seed {cfg.seed}",
            "algorithmic_bytes": kbar_bytes + gather,
            "hbm_frac": (kbar_bytes + gather) / (ms / 1e3) / 1e9 / load_peaks()["hbm_gbs"],
+           "kernel_traffic_bytes": {k: measured_traffic(k, "decode_1m")
+                                    for k in ("decode_scores", "decode_select", "decode_attend")},
            "gpu_launches_per_step": 7}  # append x3, scores, select, union, attend
     del caches, kbar, new, out, ws
     torch.cuda.empty_cache()
