@@ -13,7 +13,8 @@ selected tokens scaled by 1/sqrt(d), and an elementwise sigmoid output gate. Als
 layer that alternates 3:1 with it (same section): the gated attention over a sliding window of
 keys, the window size being a parameter (the pages give none). And the FP8 storage of the KV
 cache (section "long-horizon RL and run cost"): e4m3 values with a power-of-two scale per
-(token, group) row; decode over an FP8 cache is attention over the dequantized values.
+(token, group) row; decode over an FP8 cache is attention over the dequantized values. And the
+backward of the gated attention through a fixed selection (dq, dk, dv, dgate).
 
 Parity pins: every function here is pinned by tests/test_oracle_pins.py (brute force on
 T <= 64, dense reduction against torch's SDPA in fp64, closed forms and invariants).
@@ -57,9 +58,11 @@ def load(path: str):
                                   ctypes.c_int]
     L.oracle_swa.argtypes = [ctypes.POINTER(Dims), ctypes.c_int, P, P, P, P, P, ctypes.c_int, P, ctypes.c_int]
     L.oracle_quantize_fp8.argtypes = [ctypes.c_int, ctypes.c_int, P, P, P]
+    L.oracle_attend_backward.argtypes = [ctypes.POINTER(Dims), ctypes.c_int, P, P, P, P, P, P, P, P, P, P, P]
     L.oracle_dequantize_fp8.argtypes = [ctypes.c_int, ctypes.c_int, P, P, P]
     for f in (L.oracle_compress, L.oracle_scores, L.oracle_select, L.oracle_attend, L.oracle_coverage,
-              L.oracle_swa, L.oracle_max_threads, L.oracle_quantize_fp8, L.oracle_dequantize_fp8):
+              L.oracle_swa, L.oracle_max_threads, L.oracle_quantize_fp8, L.oracle_dequantize_fp8,
+              L.oracle_attend_backward):
         f.restype = ctypes.c_int
     return L
 
@@ -185,6 +188,28 @@ def coverage(dm: Dims, rows_bt, q_rows, k, sel, ktop: int = 2048, n_threads: int
     if rc != 0:
         raise ValueError(f"oracle_coverage: {rc}")
     return cov
+
+
+def attend_backward(dm: Dims, rows_bt, q_rows, k, v, gate_rows, sel, dy_rows):
+    """Gradients of the gated attention through a fixed selection, for query rows (b, t):
+    returns (dq [n, Hq, d], dk [batch, T, G, d], dv [batch, T, G, d], dgate [n, Hq, d]) in fp64,
+    dk and dv summed over the listed rows."""
+    rows = _rows(rows_bt)
+    n = rows.shape[0]
+    q_rows, gate_rows, k, v, dy_rows = _u16(q_rows), _u16(gate_rows), _u16(k), _u16(v), _u16(dy_rows)
+    assert q_rows.size == n * dm.Hq * dm.d and gate_rows.size == q_rows.size and dy_rows.size == q_rows.size
+    assert k.size == dm.batch * dm.T * dm.G * dm.d and v.size == k.size
+    sel = np.ascontiguousarray(sel, dtype=np.int32)
+    assert sel.size == n * dm.G * (dm.k // dm.B)
+    dq = np.zeros((n, dm.Hq, dm.d))
+    dgate = np.zeros((n, dm.Hq, dm.d))
+    dk = np.zeros((dm.batch, dm.T, dm.G, dm.d))
+    dv = np.zeros((dm.batch, dm.T, dm.G, dm.d))
+    rc = lib().oracle_attend_backward(ctypes.byref(dm), n, _p(rows), _p(q_rows), _p(k), _p(v), _p(gate_rows),
+                                      _p(sel), _p(dy_rows), _p(dq), _p(dk), _p(dv), _p(dgate))
+    if rc != 0:
+        raise ValueError(f"oracle_attend_backward: {rc}")
+    return dq, dk, dv, dgate
 
 
 def quantize_fp8(x) -> tuple:

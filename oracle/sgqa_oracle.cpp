@@ -358,4 +358,82 @@ int oracle_dequantize_fp8(int n_rows, int d, const uint8_t* q, const double* sca
   return 0;
 }
 
+
+// Backward of steps (3) and (4) through a given selection (the selection is a discrete choice and
+// carries no gradient; the pages train the 1M-context model with this layer: mo.ai.kr, "Step 5
+// Preview agentic work design", section "model structure and training stability"). For every
+// query row (b, t) and head h of group g, with U the selected tokens u <= t:
+//   z_u = q . k_u / sqrt(d),  p = softmax_U(z),  o = sum_u p_u v_u,  s = sigmoid(gate),  y = o * s
+// and dy the gradient of y:
+//   dgate = dy * o * s * (1 - s)          do = dy * s
+//   dv_u += p_u do                         dp_u = do . v_u
+//   dz_u = p_u (dp_u - sum_w p_w dp_w)     dq = sum_u dz_u k_u / sqrt(d)     dk_u += dz_u q / sqrt(d)
+// dq, dgate [n_rows, Hq, d] (the listed rows); dk, dv [batch, T, G, d] accumulate over all listed
+// rows (zeroed here). All fp64; rows are processed one after another.
+int oracle_attend_backward(const Dims* dm, int n_rows, const int32_t* rows_bt, const uint16_t* q,
+                           const uint16_t* k, const uint16_t* v, const uint16_t* gate, const int32_t* sel,
+                           const uint16_t* dy, double* dq, double* dk, double* dv, double* dgate) {
+  if (!dims_ok(dm)) return -1;
+  const int Kb = dm->k / dm->B, R = dm->Hq / dm->G, d = dm->d;
+  const double inv_sqrt_d = 1.0 / std::sqrt((double)d);
+  const long kv_elems = (long)dm->batch * dm->T * dm->G * d;
+  std::fill(dk, dk + kv_elems, 0.0);
+  std::fill(dv, dv + kv_elems, 0.0);
+  for (long rh = 0; rh < (long)n_rows * dm->Hq; ++rh) {
+    const long row = rh / dm->Hq;
+    const int h = (int)(rh % dm->Hq), g = h / R;
+    const long b = rows_bt[2 * row];
+    const int t = rows_bt[2 * row + 1];
+    const int32_t* S = sel + (row * dm->G + g) * Kb;
+    std::vector<int> U;
+    for (int i = 0; i < Kb; ++i) {
+      const int j = S[i];
+      if (j < 0) continue;
+      if (j > t / dm->B) return -3;
+      for (int u = j * dm->B; u < (j + 1) * dm->B && u <= t; ++u) U.push_back(u);
+    }
+    const uint16_t* qv = q + rh * d;
+    auto kat = [&](int u, int e) { return bf16_to_f64(k[((b * dm->T + u) * dm->G + g) * d + e]); };
+    auto vat = [&](int u, int e) { return bf16_to_f64(v[((b * dm->T + u) * dm->G + g) * d + e]); };
+    std::vector<double> z(U.size()), p(U.size()), o(d, 0.0), dov(d), dp(U.size());
+    double zmax = -INFINITY;
+    for (size_t n = 0; n < U.size(); ++n) {
+      double dot = 0.0;
+      for (int e = 0; e < d; ++e) dot += bf16_to_f64(qv[e]) * kat(U[n], e);
+      z[n] = dot * inv_sqrt_d;
+      zmax = std::max(zmax, z[n]);
+    }
+    double l = 0.0;
+    for (size_t n = 0; n < U.size(); ++n) l += (p[n] = std::exp(z[n] - zmax));
+    for (size_t n = 0; n < U.size(); ++n) {
+      p[n] /= l;
+      for (int e = 0; e < d; ++e) o[e] += p[n] * vat(U[n], e);
+    }
+    for (int e = 0; e < d; ++e) {
+      const double s = 1.0 / (1.0 + std::exp(-bf16_to_f64(gate[rh * d + e])));
+      const double dye = bf16_to_f64(dy[rh * d + e]);
+      dgate[rh * d + e] = dye * o[e] * s * (1.0 - s);
+      dov[e] = dye * s;
+    }
+    double sum_pdp = 0.0;
+    for (size_t n = 0; n < U.size(); ++n) {
+      double dot = 0.0;
+      for (int e = 0; e < d; ++e) dot += dov[e] * vat(U[n], e);
+      dp[n] = dot;
+      sum_pdp += p[n] * dot;
+    }
+    for (int e = 0; e < d; ++e) dq[rh * d + e] = 0.0;
+    for (size_t n = 0; n < U.size(); ++n) {
+      const double dz = p[n] * (dp[n] - sum_pdp);
+      const long kvrow = ((b * dm->T + U[n]) * dm->G + g) * d;
+      for (int e = 0; e < d; ++e) {
+        dq[rh * d + e] += dz * kat(U[n], e) * inv_sqrt_d;
+        dk[kvrow + e] += dz * bf16_to_f64(qv[e]) * inv_sqrt_d;
+        dv[kvrow + e] += p[n] * dov[e];
+      }
+    }
+  }
+  return 0;
+}
+
 }  // extern "C"

@@ -11,7 +11,8 @@ coverage of the ablation, a reversed ranking, an interleaved head->group mapping
 the higher token, a top set one token short, and the query's own token left out (these are
 checked against the coverage pins); and in the FP8 KV storage, ties rounded away from even, a
 scale one power of two off either way, the subnormal range cut at the wrong binade, and a dropped
-sign (checked against the FP8 pins).
+sign (checked against the FP8 pins); and in the backward, the softmax Jacobian's subtracted term
+dropped, dk unscaled, dv ungated, the gate's derivative without (1 - s) (backward pins).
 """
 import os
 import subprocess
@@ -107,6 +108,26 @@ def _fp8_pin_calls():
     ]
 
 
+# Backward: the softmax Jacobian's subtracted term dropped, dk without the 1/sqrt(d) scale, dv from
+# dy instead of dy * sigmoid(gate), the gate's derivative without its (1 - s) factor
+BACKWARD_MUTANTS = {
+    "bw_no_softmax_correction": ("const double dz = p[n] * (dp[n] - sum_pdp);", "const double dz = p[n] * dp[n];"),
+    "bw_dk_unscaled": ("dk[kvrow + e] += dz * bf16_to_f64(qv[e]) * inv_sqrt_d;",
+                       "dk[kvrow + e] += dz * bf16_to_f64(qv[e]);"),
+    "bw_dv_ungated": ("dov[e] = dye * s;", "dov[e] = dye;"),
+    "bw_gate_derivative": ("dgate[rh * d + e] = dye * o[e] * s * (1.0 - s);", "dgate[rh * d + e] = dye * o[e] * s;"),
+}
+
+
+def _backward_pin_calls():
+    import tests.test_oracle_backward_pins as bw
+    return [
+        lambda: bw.test_backward_dense_reduction_matches_sdpa_autograd(None, 40, 8),
+        lambda: bw.test_backward_sparse_selection_matches_masked_autograd(None),
+        lambda: bw.test_backward_matches_finite_differences_of_the_forward(None),
+    ]
+
+
 def _coverage_pin_calls():
     return [
         lambda: pins.test_coverage_brute_force(None, False),
@@ -127,17 +148,18 @@ def _swa_pin_calls():
     ]
 
 
-ALL_MUTANTS = {**MUTANTS, **SWA_MUTANTS, **COVERAGE_MUTANTS, **FP8_MUTANTS}
+ALL_MUTANTS = {**MUTANTS, **SWA_MUTANTS, **COVERAGE_MUTANTS, **FP8_MUTANTS, **BACKWARD_MUTANTS}
 
 
 @pytest.mark.parametrize("name", sorted(ALL_MUTANTS))
 def test_pins_catch_mutant(tmp_path, name):
     old, new = ALL_MUTANTS[name]
     calls = (PIN_CALLS if name in MUTANTS else _swa_pin_calls() if name in SWA_MUTANTS
-             else _coverage_pin_calls() if name in COVERAGE_MUTANTS else _fp8_pin_calls())
+             else _coverage_pin_calls() if name in COVERAGE_MUTANTS
+             else _fp8_pin_calls() if name in FP8_MUTANTS else _backward_pin_calls())
     src = open(oracle.SRC).read()
     assert src.count(old) >= 1, f"mutation anchor not found: {name}"
-    if name in COVERAGE_MUTANTS or name in FP8_MUTANTS:
+    if name in COVERAGE_MUTANTS or name in FP8_MUTANTS or name in BACKWARD_MUTANTS:
         assert src.count(old) == 1, f"mutation anchor not unique: {name}"
     mutated = src.replace(old, new)
     cpp = tmp_path / "mut.cpp"
