@@ -404,6 +404,8 @@ def run_ours(args, world, rank):
         result["decode_fp8"] = run_decode_fp8(args, world, s)
     if not args.no_ablation and world == 1:
         result["ablation"] = run_ablation(args, world, s)
+    if not args.no_backward and world == 1:
+        result["backward"] = run_backward(args, world, s)
     if not args.no_swa:
         result["swa"] = run_swa(args, world, s)
     if cpu_in is not None:
@@ -659,6 +661,62 @@ def run_decode_fp8(args, world, s):
     return res
 
 
+def run_backward(args, world, s):
+    """Gradients of the gated attention (dq, dk, dv, dgate, fp32) through the selection of the 128K
+    prefill, via sgqa_attend_backward, inputs resident in HBM."""
+    import torch
+    import block_sparse_long_kbar_b200 as sg
+    from sgqa_inputs import gen_device
+    cfg = CONFIGS["128k"]
+    dims = sg.sgqa_dims.of(cfg)
+    dev = {}
+    for n in ("q", "k", "v", "gate", "q_idx", "k_idx"):
+        dev[n] = torch.empty(cfg.shape(n), dtype=torch.bfloat16, device="cuda")
+        gen_device(cfg, n, dev[n])
+    out = torch.empty(cfg.shape("q"), dtype=torch.bfloat16, device="cuda")
+    sel = torch.empty((cfg.batch, cfg.T, cfg.G, cfg.Kb), dtype=torch.int32, device="cuda")
+    ws = sg.alloc_workspace(sg.sgqa_workspace_size(dims))
+    sg.sgqa_reset_device_status(ws)
+    sg.sgqa_forward(dims, dev["q"], dev["k"], dev["v"], dev["q_idx"], dev["k_idx"], dev["gate"], out, ws,
+                    sel_out=sel, stream=s)
+    del ws
+    dy = torch.empty(cfg.shape("q"), dtype=torch.bfloat16, device="cuda")
+    gen_device(cfg.replace(seed=cfg.seed + 1000), "q", dy)  # an independent N(0,1) output gradient
+    grads = {n: torch.empty(cfg.shape("q" if n in ("dq", "dgate") else "k"), dtype=torch.float32, device="cuda")
+             for n in ("dq", "dk", "dv", "dgate")}
+    bws = sg.alloc_workspace(sg.sgqa_backward_workspace_size(dims))
+    sg.sgqa_reset_device_status(bws)
+    torch.cuda.synchronize()
+
+    def step():
+        sg.sgqa_attend_backward(dims, dev["q"], dev["k"], dev["v"], dev["gate"], sel, dy, grads["dq"], grads["dk"],
+                                grads["dv"], grads["dgate"], bws, stream=s)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    steps = 1  # a step takes seconds (CUDA-core kernels); one timed step after the warm-up
+    e0.record(s)
+    for _ in range(steps):
+        step()
+    e1.record(s)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    assert sg.sgqa_get_device_status(bws) == 0
+    wc = work_counts(cfg)
+    res = {"metric": "Sparse GQA backward (dq, dk, dv, dgate through the selection) tokens/s at 128K",
+           "value": cfg.batch * cfg.T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+           "workload": f"backward 128k: the 128K prefill's inputs and GPU selection, dout ~ N(0,1); fp32 gradients",
+           "flops": 2 * wc["attn_flops"], "achieved_tflops": 2 * wc["attn_flops"] / (ms / 1e3) / 1e12,
+           "note": "CUDA-core kernels (row-centric dq/dgate, a warp per head; key-centric dk/dv over a reverse "
+                   "index); flops = 2x the forward attention's (the recomputations of z and p are not counted)",
+           "gpu_launches_per_step": 6}
+    del dev, out, sel, dy, grads, bws
+    torch.cuda.empty_cache()
+    return res
+
+
 ABLATION_COV_STRIDE = 2048  # coverage rows: every 2048th query of the 64K sequence (all 32 heads)
 
 
@@ -901,6 +959,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-swa", action="store_true")
     ap.add_argument("--no-ablation", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--query-sharded", action="store_true",
                     help="split the sequence's queries over the ranks even at N = 1 (the N > 1 path)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -27,7 +27,8 @@ STATUS_NAMES = {0: "SGQA_OK", 1: "SGQA_ERR_INVALID_ARG", 2: "SGQA_ERR_UNSUPPORTE
 EXPORTS = ["sgqa_status_string", "sgqa_version", "sgqa_workspace_size", "sgqa_decode_workspace_size",
            "sgqa_reset_device_status", "sgqa_get_device_status", "sgqa_compress_keys", "sgqa_select",
            "sgqa_attend", "sgqa_forward", "sgqa_decode", "sgqa_decode_noalloc", "sgqa_gated_swa",
-           "sgqa_quantize_kv_fp8", "sgqa_decode_fp8", "sgqa_test_stall_decode_cta", "sgqa_forward_rows"]
+           "sgqa_quantize_kv_fp8", "sgqa_decode_fp8", "sgqa_test_stall_decode_cta", "sgqa_forward_rows",
+           "sgqa_backward_workspace_size", "sgqa_attend_backward"]
 
 
 class SgqaError(RuntimeError):
@@ -79,9 +80,12 @@ def load_library():
     L.sgqa_decode_fp8.argtypes = [D, I, I] + [P] * 15 + [S, P]
     L.sgqa_test_stall_decode_cta.argtypes = [I]
     L.sgqa_forward_rows.argtypes = [D, I, I, P, P, P, P, P, P, P, P, P, S, P]
+    L.sgqa_backward_workspace_size.restype = S
+    L.sgqa_backward_workspace_size.argtypes = [D]
+    L.sgqa_attend_backward.argtypes = [D] + [P] * 11 + [S, P]
     for n in ("sgqa_reset_device_status", "sgqa_get_device_status", "sgqa_compress_keys", "sgqa_select",
               "sgqa_attend", "sgqa_forward", "sgqa_decode", "sgqa_decode_noalloc", "sgqa_gated_swa",
-              "sgqa_quantize_kv_fp8", "sgqa_decode_fp8", "sgqa_test_stall_decode_cta", "sgqa_forward_rows"):
+              "sgqa_quantize_kv_fp8", "sgqa_decode_fp8", "sgqa_test_stall_decode_cta", "sgqa_forward_rows", "sgqa_attend_backward"):
         getattr(L, n).restype = I
     _lib = L
     return L
@@ -186,6 +190,18 @@ def sgqa_forward_rows(dims, t_begin, t_end, q_rows, k, v, q_idx_rows, k_idx, gat
         ctypes.byref(dims), int(t_begin), int(t_end), _ptr(q_rows, "q_rows"), _ptr(k, "k"), _ptr(v, "v"),
         _ptr(q_idx_rows, "q_idx_rows"), _ptr(k_idx, "k_idx"), _ptr(gate_rows, "gate_rows"), _ptr(out_rows, "out_rows"),
         _ptr(sel_out_rows, "sel_out_rows"), _ptr(ws, "ws"), ws.numel(), _stream(stream)))
+
+
+def sgqa_backward_workspace_size(dims: sgqa_dims) -> int:
+    return int(load_library().sgqa_backward_workspace_size(ctypes.byref(dims)))
+
+
+def sgqa_attend_backward(dims, q, k, v, gate, sel, dout, dq, dk, dv, dgate, ws, stream=None):
+    """Gradients (fp32) of the gated attention through the given selection: dq, dk, dv, dgate."""
+    _check("sgqa_attend_backward", load_library().sgqa_attend_backward(
+        ctypes.byref(dims), _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _ptr(gate, "gate"), _ptr(sel, "sel"),
+        _ptr(dout, "dout"), _ptr(dq, "dq"), _ptr(dk, "dk"), _ptr(dv, "dv"), _ptr(dgate, "dgate"), _ptr(ws, "ws"),
+        ws.numel(), _stream(stream)))
 
 
 INPUTS = ("q", "k", "v", "q_idx", "k_idx", "gate")

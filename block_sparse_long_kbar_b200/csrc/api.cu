@@ -128,6 +128,49 @@ DecodeWs decode_layout(const sgqa_dims* d, int n_new, void* ws) {
   return w;
 }
 
+struct BackwardWs {
+  int* status;
+  float* lse;
+  float* dsum;
+  float* dov;
+  int* rcount;
+  int* ccount;
+  int* roff;
+  int* rlist;
+  int nblkc, rchunk, nchunk;
+  size_t bytes;
+};
+
+BackwardWs backward_layout(const sgqa_dims* d, void* ws) {
+  BackwardWs w{};
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  const size_t rows = (size_t)d->batch * d->T;
+  const size_t segs = (size_t)d->batch * d->G;
+  w.nblkc = (d->T + d->B - 1) / d->B;
+  // chunks of at least 256 rows, at most 256 chunks (bounds the per-chunk count table)
+  w.rchunk = 256;
+  while ((d->T + w.rchunk - 1) / w.rchunk > 256) w.rchunk *= 2;
+  w.nchunk = (d->T + w.rchunk - 1) / w.rchunk;
+  size_t off = kStatusBytes;
+  w.status = reinterpret_cast<int*>(base);
+  w.lse = reinterpret_cast<float*>(base + off);
+  off += align256(rows * d->Hq * 4);
+  w.dsum = reinterpret_cast<float*>(base + off);
+  off += align256(rows * d->Hq * 4);
+  w.dov = reinterpret_cast<float*>(base + off);
+  off += align256(rows * d->Hq * (size_t)d->d * 4);
+  w.rcount = reinterpret_cast<int*>(base + off);
+  off += align256(segs * w.nblkc * 4);
+  w.roff = reinterpret_cast<int*>(base + off);
+  off += align256(segs * (w.nblkc + 1) * 4);
+  w.ccount = reinterpret_cast<int*>(base + off);
+  off += align256(segs * (size_t)w.nchunk * w.nblkc * 4);
+  w.rlist = reinterpret_cast<int*>(base + off);
+  off += align256(segs * (size_t)d->T * (d->k / d->B) * 4);
+  w.bytes = off;
+  return w;
+}
+
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? SGQA_OK : SGQA_ERR_CUDA; }
 
 // Prefill attention for query rows [a.t_begin, a.t_end): schedule the rows by selection
@@ -452,6 +495,31 @@ int sgqa_decode_fp8(const sgqa_dims* dims, int cache_len, int n_new, uint8_t* k8
   kv.v_scale = v_scale;
   return decode_impl(dims, cache_len, n_new, kv, kidx_cache, kbar_cache, q_new, k_new, v_new, qidx_new, kidx_new,
                      gate_new, out, sel_out, ws, ws_bytes, stream);
+}
+
+size_t sgqa_backward_workspace_size(const sgqa_dims* dims) {
+  if (check_dims(dims) != SGQA_OK || !backward_supported(dims->Hq, dims->G, dims->d, dims->B)) return 0;
+  return backward_layout(dims, nullptr).bytes;
+}
+
+int sgqa_attend_backward(const sgqa_dims* dims, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                         const uint16_t* gate, const int32_t* sel, const uint16_t* dout, float* dq, float* dk,
+                         float* dv, float* dgate, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (!backward_supported(dims->Hq, dims->G, dims->d, dims->B)) return SGQA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gate) || !aligned16(sel) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(dgate))
+    return SGQA_ERR_INVALID_ARG;
+  const BackwardWs w = backward_layout(dims, ws);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < w.bytes) return SGQA_ERR_WORKSPACE;
+  BackwardArgs a{};
+  a.q = q; a.k = k; a.v = v; a.gate = gate; a.dy = dout; a.sel = sel;
+  a.dq = dq; a.dk = dk; a.dv = dv; a.dgate = dgate; a.lse = w.lse; a.dsum = w.dsum; a.dov = w.dov;
+  a.rcount = w.rcount; a.ccount = w.ccount; a.roff = w.roff; a.rlist = w.rlist;
+  a.batch = dims->batch; a.T = dims->T; a.Hq = dims->Hq; a.G = dims->G; a.d = dims->d; a.B = dims->B;
+  a.Kb = dims->k / dims->B; a.nblkc = w.nblkc; a.rchunk = w.rchunk; a.nchunk = w.nchunk; a.status = w.status;
+  return cuda_status(launch_backward(a, static_cast<cudaStream_t>(stream)));
 }
 
 int sgqa_test_stall_decode_cta(int cta) {

@@ -137,4 +137,33 @@ cudaError_t launch_decode_attend_tc(const DecodeAttendArgs& a, cudaStream_t s);
 cudaError_t launch_quantize_fp8(const uint16_t* src, uint8_t* dst8, float* dscale, int batch, int n_t, int G, int T,
                                 int t0, cudaStream_t s);
 
+// Backward through a fixed selection (d in {64, 128}, B in {4, 8, 16}, Hq/G <= 16). dq, dgate
+// [batch, T, Hq, d], dk, dv [batch, T, G, d] fp32; lse, dsum [batch, T, Hq]; the reverse index:
+// rcount [batch * G][nblkc], ccount [batch * G][nchunk][nblkc] (rows of each chunk of rchunk rows
+// that select each block, then their prefixes), roff [batch * G][nblkc + 1],
+// rlist [batch * G][T * Kb].
+struct BackwardArgs {
+  const uint16_t* q;
+  const uint16_t* k;
+  const uint16_t* v;
+  const uint16_t* gate;
+  const uint16_t* dy;
+  const int32_t* sel;
+  float* dq;
+  float* dk;
+  float* dv;
+  float* dgate;
+  float* lse;
+  float* dsum;
+  float* dov;  // dy * sigmoid(gate) [batch, T, Hq, d] fp32, written by the row-centric pass
+  int* rcount;
+  int* ccount;
+  int* roff;
+  int* rlist;
+  int batch, T, Hq, G, d, B, Kb, nblkc, rchunk, nchunk;
+  int* status;
+};
+bool backward_supported(int Hq, int G, int d, int B);
+cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t s);
+
 }  // namespace sgqa

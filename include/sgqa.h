@@ -138,6 +138,26 @@ int sgqa_forward_rows(const sgqa_dims* dims, int t_begin, int t_end, const uint1
                       const uint16_t* k_idx, const uint16_t* gate_rows, uint16_t* out_rows,
                       int32_t* sel_out_rows, void* ws, size_t ws_bytes, void* stream);
 
+/* Bytes of workspace sgqa_attend_backward needs; 0 if the dims are invalid or unsupported. */
+size_t sgqa_backward_workspace_size(const sgqa_dims* dims);
+
+/* Gradients of steps (3) and (4) through a given selection (the selection is a discrete choice
+ * and carries no gradient; the pages train the 1M-context model with this layer: mo.ai.kr, "Step 5
+ * Preview agentic work design", section "model structure and training stability"). With
+ * z_u = q . k_u / sqrt(d), p = softmax over the selected tokens u <= t, o = sum p_u v_u,
+ * s = sigmoid(gate) and dout the gradient of out = o * s:
+ *   dgate = dout * o * s * (1 - s);  do = dout * s;  dz_u = p_u (do . v_u - do . o);
+ *   dq = sum_u dz_u k_u / sqrt(d);  dk_u = sum over rows dz_u q / sqrt(d);  dv_u = sum over rows p_u do.
+ * q, gate, dout [batch, T, Hq, d], k, v [batch, T, G, d] bf16; sel [batch, T, G, k/B] in
+ * sgqa_select's format -> dq, dgate [batch, T, Hq, d] and dk, dv [batch, T, G, d], fp32 (every
+ * element written). Deterministic: the same inputs give the same bits (no floating-point atomics).
+ * Supported: d in {64, 128}, B in {4, 8, 16}, Hq/G <= 16 (else SGQA_ERR_UNSUPPORTED); ws of
+ * sgqa_backward_workspace_size bytes, its first 256 bytes the status word as for the others. */
+int sgqa_attend_backward(const sgqa_dims* dims, const uint16_t* q, const uint16_t* k,
+                         const uint16_t* v, const uint16_t* gate, const int32_t* sel,
+                         const uint16_t* dout, float* dq, float* dk, float* dv, float* dgate,
+                         void* ws, size_t ws_bytes, void* stream);
+
 /* One decode step for dims.batch sequences sharing one cache length.
  * Caches (dims.T = capacity): k_cache, v_cache [batch, T, G, d], kidx_cache [batch, T, d_idx]
  * bf16, kbar_cache [batch, T/B, d_idx] fp32 holding the block means of every block complete in
