@@ -14,11 +14,12 @@
 // at the bf16 tensor rate with fp32-accurate scores, hi products first, then lo, as in prefill.
 //
 // Pipeline (one CTA per (sequence, range of 128-candidate tiles)): warp 0 TMA-loads fp32 tiles
-// (32 KB) into a 4-stage ring; warps 2-9 convert a staged tile into the two bf16 operand planes
-// (128B-swizzled K-major, double-buffered); warp 1 allocates TMEM and issues the MMAs into two
-// accumulators; warps 10-13 (one per TMEM lane quadrant, a candidate per lane) write each row's fp32
+// (32 KB) into a 2-stage ring; warps 2-5 convert a staged tile into the two bf16 operand planes
+// (128B-swizzled K-major); warp 1 allocates TMEM and issues the MMAs into two accumulators;
+// warps 6-9 (one per TMEM lane quadrant, a candidate per lane) write each row's fp32
 // scores for the candidates it has, and per row the largest order-preserving key of every 32
-// consecutive candidates (a lower bound on the row's selection threshold comes from these). Every
+// consecutive candidates (a lower bound on the row's selection threshold comes from these). Two
+// CTAs run per SM, so one's hand-offs overlap the other's work. Every
 // wait is bounded by %globaltimer: on expiry the kernel records SGQA_ERR_TIMEOUT, drains its
 // copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
@@ -32,15 +33,17 @@ namespace {
 
 constexpr int kCand = 128;                 // candidates per tile (MMA M)
 constexpr int kDI = 64;                    // indexer dim of this kernel
-constexpr int kStg = 4;                    // fp32 staging stages
+constexpr int kStg = 2;                    // fp32 staging stages
+constexpr int kNOp = 1;                    // bf16 operand buffers (hi + lo planes)
+constexpr int kCtasPerSm = 2;              // two pipelines per SM hide each other's hand-offs
 constexpr int kStgBytes = kCand * kDI * 4; // 32 KB
 constexpr int kPlane = kCand * kDI * 2;    // one bf16 plane: 16 KB
 constexpr int kOp = 2 * kPlane;            // hi then lo
-constexpr int kConvWarps = 8;              // converter warps (2 .. 9); epilogue warps 10 .. 13
+constexpr int kConvWarps = 4;              // converter warps (2 .. 5); epilogue warps 6 .. 9
 constexpr int kThr = (2 + kConvWarps + 4) * 32;
 
 struct ScShared {
-  uint64_t full[kStg], empty[kStg], op_full[2], op_empty[2], acc_full[2], acc_empty[2];
+  uint64_t full[kStg], empty[kStg], op_full[kNOp], op_empty[kNOp], acc_full[2], acc_empty[2];
   uint32_t tmem;
   volatile int abort_flag;
 };
@@ -48,8 +51,8 @@ struct ScShared {
 template <int NR>
 struct ScCfg {
   static constexpr int kQ = NR * 128;
-  static constexpr int kSmem = 1024 + kStg * kStgBytes + 2 * kOp + kQ + (int)sizeof(ScShared) + 64;
-  static_assert(kSmem <= 232448, "shared memory of one CTA");
+  static constexpr int kSmem = 1024 + kStg * kStgBytes + kNOp * kOp + kQ + (int)sizeof(ScShared) + 64;
+  static_assert(kCtasPerSm * (kSmem + 1024) <= 233472, "shared memory of the resident CTAs");
 };
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, const int* gstatus) {
@@ -59,14 +62,14 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 template <int NR>
-__global__ void __launch_bounds__(kThr, 1)
+__global__ void __launch_bounds__(kThr, kCtasPerSm)
     decode_scores_tc_kernel(const __grid_constant__ CUtensorMap map_kbar, DecodeScoreArgs a) {
   using C = ScCfg<NR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_align<1024>(smem_raw);
   uint8_t* sStg = smem;
-  uint8_t* sOp = sStg + kStg * kStgBytes;  // [2][hi | lo]
-  uint8_t* sQ = sOp + 2 * kOp;
+  uint8_t* sOp = sStg + kStg * kStgBytes;  // [kNOp][hi | lo]
+  uint8_t* sQ = sOp + kNOp * kOp;
   ScShared* sh = reinterpret_cast<ScShared*>(sQ + C::kQ);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -86,9 +89,11 @@ __global__ void __launch_bounds__(kThr, 1)
       tc::mbar_init(&sh->full[s], 1);
       tc::mbar_init(&sh->empty[s], kConvWarps);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kNOp; ++s) {
       tc::mbar_init(&sh->op_full[s], kConvWarps);
       tc::mbar_init(&sh->op_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&sh->acc_full[s], 1);
       tc::mbar_init(&sh->acc_empty[s], 4);
     }
@@ -134,16 +139,16 @@ __global__ void __launch_bounds__(kThr, 1)
       const uint32_t idesc = tc::idesc_bf16_f32(kCand, NR);
       int k = 0;
       for (; k < n && !sh->abort_flag; ++k) {
-        const int op = k & 1;
-        if (!tc::mbar_wait(&sh->op_full[op], (uint32_t)((k >> 1) & 1), &sh->abort_flag, a.status) ||
-            (k >= 2 && !tc::mbar_wait(&sh->acc_empty[op], (uint32_t)(((k >> 1) - 1) & 1), &sh->abort_flag, a.status))) {
+        const int op = k % kNOp, ab = k & 1;
+        if (!tc::mbar_wait(&sh->op_full[op], (uint32_t)((k / kNOp) & 1), &sh->abort_flag, a.status) ||
+            (k >= 2 && !tc::mbar_wait(&sh->acc_empty[ab], (uint32_t)(((k >> 1) - 1) & 1), &sh->abort_flag, a.status))) {
           if (!sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
           sh->abort_flag = 1;
           break;
         }
         tc::fence_after_sync();
         const uint8_t* hi = sOp + op * kOp;
-        const uint32_t d = tmem + (uint32_t)(op * NR);
+        const uint32_t d = tmem + (uint32_t)(ab * NR);
 #pragma unroll
         for (int kk = 0; kk < kDI / 16; ++kk)
           tc::mma_bf16_ss(d, tc::smem_desc_kmajor(hi + kk * 32, 128), tc::smem_desc_kmajor(sQ + kk * 32, 128), idesc,
@@ -153,7 +158,7 @@ __global__ void __launch_bounds__(kThr, 1)
           tc::mma_bf16_ss(d, tc::smem_desc_kmajor(hi + kPlane + kk * 32, 128), tc::smem_desc_kmajor(sQ + kk * 32, 128),
                           idesc, 1u);
         tc::mma_commit(&sh->op_empty[op]);
-        tc::mma_commit(&sh->acc_full[op]);
+        tc::mma_commit(&sh->acc_full[ab]);
       }
       if (k > 0) {  // the last MMAs complete before TMEM is freed
         volatile int no_abort = 0;
@@ -164,9 +169,9 @@ __global__ void __launch_bounds__(kThr, 1)
     // ---- converters: fp32 tile -> bf16 hi and lo planes (128B-swizzled K-major rows) ----
     const int ct = tid - 64;
     for (int k = 0; k < n; ++k) {
-      const int st = k % kStg, op = k & 1;
+      const int st = k % kStg, op = k % kNOp;
       if (!warp_wait(&sh->full[st], (uint32_t)((k / kStg) & 1), &sh->abort_flag, a.status) ||
-          (k >= 2 && !warp_wait(&sh->op_empty[op], (uint32_t)(((k >> 1) - 1) & 1), &sh->abort_flag, a.status))) {
+          (k >= kNOp && !warp_wait(&sh->op_empty[op], (uint32_t)(((k / kNOp) - 1) & 1), &sh->abort_flag, a.status))) {
         if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
         sh->abort_flag = 1;
         break;
@@ -286,9 +291,9 @@ cudaError_t launch_nr(const DecodeScoreArgs& a, cudaStream_t s) {
 bool decode_scores_tc_supported(int d_idx, int n_new, int G) { return d_idx == kDI && n_new * G <= 32; }
 
 int decode_scores_ctas(int batch, int c_max) {
-  // one CTA per SM (the staging ring fills its shared memory), one wave over all sequences
+  // two CTAs per SM, one wave over all sequences
   const int ntile = (c_max + kCand - 1) / kCand;
-  int cps = 148 / (batch > 0 ? batch : 1);
+  int cps = kCtasPerSm * 148 / (batch > 0 ? batch : 1);
   if (cps > ntile) cps = ntile;
   if (cps < 1) cps = 1;
   return cps;
