@@ -109,11 +109,13 @@ def work_counts(cfg):
 
 # Per-key instruction counts of the select kernel's epilogue (select_tc.cu), per pass over the
 # scored candidates: a histogram pass spends about 8 thread-instructions per key (order-preserving
-# key, bin address, prefix test, shared reduction); the emit pass about 12 (key, two compares,
-# mask updates, predicated staging); the tile's TMEM load adds 2 per key per pass. A typical
-# 128K row resolves its threshold after 3 histogram passes, then emits.
-SELECT_INSTR_PER_KEY = {"hist": 8 + 2, "emit": 12 + 2}
-SELECT_PASSES = {"hist": 3, "emit": 1}
+# key, bin address, prefix test, shared reduction); the emit pass about 8 (key, two compares, two
+# bit updates) plus a bitmap store per 32 keys; the tile's TMEM load adds 2 per key per pass. A
+# typical 128K row (topic-clustered scores) resolves its threshold bucket after 2 histogram passes:
+# the first isolates its topic's blocks, the second leaves a bucket of a few keys, collected in the
+# emit pass.
+SELECT_INSTR_PER_KEY = {"hist": 8 + 2, "emit": 8 + 2}
+SELECT_PASSES = {"hist": 2, "emit": 1}
 
 
 def select_alu_model(wc, sm_mhz):
@@ -122,7 +124,7 @@ def select_alu_model(wc, sm_mhz):
     instr = wc["scored"] * sum(SELECT_INSTR_PER_KEY[p] * SELECT_PASSES[p] for p in SELECT_PASSES)
     rate = 148 * 4 * 32 * sm_mhz * 1e6
     return {"thread_instructions": instr, "issue_rate_per_s": rate, "min_ms": instr / rate * 1e3,
-            "model": "per-key instructions x passes (histogram 3, emit 1) / SM issue rate"}
+            "model": "per-key instructions x passes (histogram 2, emit 1) / SM issue rate"}
 
 
 # ---- clocks sampled during the timed region -------------------------------------------------

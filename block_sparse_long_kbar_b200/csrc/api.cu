@@ -12,6 +12,7 @@ using namespace sgqa;
 namespace {
 
 constexpr int kSelChunkT = 32768;  // query rows per selection chunk when sel stays in ws
+constexpr size_t kSelBitsBudget = 256ull << 20;  // bitmaps of the taken candidates (K2 -> block lists)
 int g_test_stall_cta = -1;         // sgqa_test_stall_decode_cta (failure-detection tests only)
 
 bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -39,6 +40,8 @@ struct PrefillWs {
   float* kbar;
   uint16_t* hi;
   uint16_t* lo;
+  uint32_t* bits;
+  int bstride, bits_q;
   int32_t* sel;
   size_t bytes;
 };
@@ -59,6 +62,9 @@ PrefillWs prefill_layout(const sgqa_dims* d, void* ws) {
   off += align256(nk * 2);
   w.lo = reinterpret_cast<uint16_t*>(base + off);
   off += align256(nk * 2);
+  select_bits_dims(d->batch, d->T, d->G, d->B, kSelBitsBudget, &w.bstride, &w.bits_q);
+  w.bits = reinterpret_cast<uint32_t*>(base + off);
+  off += align256((size_t)d->batch * w.bits_q * d->G * (size_t)w.bstride * 4);
   w.sel = reinterpret_cast<int32_t*>(base + off);
   off += align256((size_t)d->batch * chunk * d->G * (d->k / d->B) * 4);
   w.bytes = off;
@@ -252,6 +258,7 @@ int sgqa_select(const sgqa_dims* dims, const uint16_t* q_idx, const float* kbar,
   a.q_idx = q_idx; a.q_T = dims->T; a.q_t0 = 0; a.kbar = kbar; a.kbar_hi = w.hi; a.kbar_lo = w.lo; a.sel = sel;
   a.batch = dims->batch; a.T = dims->T; a.G = dims->G; a.d_idx = dims->d_idx; a.B = dims->B;
   a.Kb = dims->k / dims->B; a.t_begin = 0; a.t_end = dims->T; a.sel_T = dims->T; a.sel_t0 = 0;
+  a.bits = w.bits; a.bstride = w.bstride; a.bits_q = w.bits_q;
   a.status = w.status;
   if (launch_split_planes(kbar, w.hi, w.lo, (long)dims->batch * (dims->T / dims->B) * dims->d_idx, s) !=
       cudaSuccess)
@@ -304,6 +311,7 @@ static int forward_rows_impl(const sgqa_dims* dims, int t_begin, int t_end, cons
   sa.q_idx = q_idx; sa.q_T = nq; sa.q_t0 = t_begin; sa.kbar = w.kbar; sa.kbar_hi = w.hi; sa.kbar_lo = w.lo;
   sa.batch = dims->batch; sa.T = dims->T; sa.G = dims->G; sa.d_idx = dims->d_idx; sa.B = dims->B;
   sa.Kb = dims->k / dims->B; sa.status = w.status;
+  sa.bits = w.bits; sa.bstride = w.bstride; sa.bits_q = w.bits_q;
   AttendArgs aa = prefill_attend_args(dims, q, k, v, gate, out, w.status);
   aa.nQ = nq; aa.q_t0 = t_begin;
   const int chunk = sel_out ? nq : (nq < kSelChunkT ? nq : kSelChunkT);

@@ -28,9 +28,15 @@ struct SelectArgs {
   int batch, T, G, d_idx, B, Kb;
   int t_begin, t_end;
   int sel_T, sel_t0;
+  // bitmaps of the taken candidates, one row of bstride words per (token, group) of a query range
+  // of at most bits_q tokens: row ((b * n + (t - range start)) * G + g), n the range's length
+  uint32_t* bits;
+  int bstride, bits_q;
   int* status;
 };
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s);
+// bitmap row stride (words) and the query rows per range for a workspace budget of `budget` bytes
+void select_bits_dims(int batch, int T, int G, int B, size_t budget, int* bstride, int* bits_q);
 
 // K3: gated attention over selected blocks for query positions [t_begin, t_end).
 //   q, gate rows (b, t) at ((b * nQ + (t - q_t0)) * Hq + h) * d; out likewise;

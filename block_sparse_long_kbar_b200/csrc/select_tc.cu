@@ -16,21 +16,21 @@
 // q_idx is exactly bf16, so the contraction runs at the bf16 tensor rate.
 //
 // Warp roles: warp 8 issues TMA loads, warp 9 allocates TMEM and issues MMAs, warps 0-7 are the
-// epilogue, two per TMEM lane quadrant (TMEM lane = row). The epilogue performs an exact radix
-// select of the m-th largest order-preserving 32-bit score key per row: every pass re-streams the
-// same score tiles (recomputed, bit-identical); in a histogram pass the two threads of a row take
-// half of every tile's columns each and add 0 or 1 per key to the row's 256-bin shared histogram
-// of the next 8 key bits (1 for keys that still match the resolved prefix; branch-free). Once
-// every row's threshold bucket is resolved or taken whole, the emit pass streams the candidates
-// in ascending j: keys above the threshold are taken, bucket keys are taken in j order up to the
-// remaining count (so ties go to the lower block index and the output is ascending without a
-// sort). From the third pass on, if every unresolved row's bucket holds at most kCap keys, the
-// emit pass comes early: it also collects those keys with the number of keys taken before each,
-// resolves them exactly afterwards and places the chosen ones by moving blocks of the row. The
-// emit marks taken candidates in bit masks (ALU only), stages the indices in a 128-entry shared
-// ring per row at positions from population counts, and the warp writes each row out 64 indices
-// at a time as whole lines. The epilogue tells the producer and MMA warps at the start of each
-// pass whether another pass follows, so they run up to one pass ahead.
+// epilogue, two per TMEM lane quadrant (TMEM lane = row); each of the two takes half of every
+// tile's columns. The epilogue performs an exact radix select of the m-th largest order-preserving
+// 32-bit score key per row: every pass re-streams the same score tiles (recomputed,
+// bit-identical); in a histogram pass each thread adds its keys that still match the resolved
+// prefix to the row's 256-bin shared histogram of the next 8 key bits (keys that do not match go
+// to a spare slot of the row, so the shared-memory reductions stay branch-free and mostly free of
+// bank conflicts). Once every row's threshold bucket is resolved or taken whole, the emit pass
+// marks the taken candidates of each 64-column half-tile in two 32-bit words and stores them to
+// the row's bitmap in global memory: keys above the threshold; bucket keys taken whole; exact ties
+// in j order (the two threads of a row exchange their tie counts through shared memory, so ties
+// go to the lower block index); or, when every unresolved row's bucket is small (from the third
+// pass on), the bucket keys are collected and resolved exactly afterwards, their bits set with
+// atomics. A separate kernel expands every row's bitmap into the ascending block list, appends
+// the own block and pads with -1. The epilogue tells the producer and MMA warps at the start of
+// each pass whether another pass follows, so they run up to one pass ahead.
 //
 // Every wait is bounded (globaltimer): on timeout the kernel records SGQA_ERR_TIMEOUT, stops all
 // roles, waits (bounded) for its own copies and MMAs in flight, frees TMEM and returns.
@@ -51,8 +51,9 @@ constexpr int kEpiWarps = 8;     // two per TMEM lane quadrant: each histograms 
 constexpr int kThreads = (kEpiWarps + 2) * 32;
 constexpr int kProducerWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
 constexpr int kMaxPasses = 5;
-constexpr int kCap = 42;         // bucket keys a row may collect for an early exact finish (3 words each)
-constexpr int kRing = 129;       // the row's output staging ring (128 words) starts at this word
+constexpr int kCap = 63;         // bucket keys a row may collect for an early exact finish (per half, 2 words each)
+constexpr int kTrash = 256;      // the row's spare histogram slot: target of the keys that do not count
+constexpr int kCnt1 = 254;       // the upper half's collected count and taken count of the row (emit pass)
 
 template <int DI>
 struct SelCfg {
@@ -130,18 +131,10 @@ __device__ __forceinline__ int pass_exists(SelShared* sh, int p, const int* gsta
 __device__ __forceinline__ void red_shared_inc(uint32_t addr) {
   asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(addr) : "memory");
 }
-// Adds 0 or 1: every lane stays active, which measured faster than a predicated reduction.
-__device__ __forceinline__ void red_shared_add(uint32_t addr, uint32_t val) {
-  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(addr), "r"(val) : "memory");
-}
-
-__device__ __forceinline__ void st_shared_u32_if(uint32_t addr, uint32_t v, uint32_t pred) {
-  asm volatile("{ .reg .pred p; setp.ne.u32 p, %2, 0; @p st.shared.u32 [%0], %1; }" ::"r"(addr), "r"(v), "r"(pred)
-               : "memory");
-}
 
 // Histogram pass: count, in the row's 256 bins, the next 8 key bits (at `shift`) of the keys
-// whose resolved bits (mask) equal prefix. kFull: all 64 candidates exist (else only q < lim).
+// whose resolved bits (mask) equal prefix; every other key increments the row's spare slot, so
+// every lane stays active. kFull: all 64 candidates exist (else only q < lim).
 template <bool kFull, bool kFirst>
 __device__ __forceinline__ void hist_chunk(const uint32_t (&v)[64], int lim, uint32_t mask, uint32_t prefix, int shift,
                                            uint32_t hbase) {
@@ -150,7 +143,7 @@ __device__ __forceinline__ void hist_chunk(const uint32_t (&v)[64], int lim, uin
     const uint32_t key = score_key(__uint_as_float(v[q]));
     const uint32_t addr = hbase + (((key >> shift) & 255u) << 2);
     if (kFull && kFirst) red_shared_inc(addr);
-    else red_shared_add(addr, ((kFull || q < lim) && (kFirst || (key & mask) == prefix)) ? 1u : 0u);
+    else red_shared_inc(((kFull || q < lim) && (kFirst || (key & mask) == prefix)) ? addr : hbase + kTrash * 4u);
   }
 }
 
@@ -225,75 +218,42 @@ __device__ __forceinline__ uint32_t pick64(const uint32_t (&v)[64], int q) {
   }
 }
 
-// Emit pass: mark (bits of tb) the candidates taken: keys >= thr, plus, among the keys of the
-// bucket [blo, blo + bw], the first tie_lim in j order; the first col_lim bucket keys are also
-// stored in cand as (key, j, number of taken keys of lower j) triples. eqn counts the bucket keys
-// seen so far in this row; pos0 is the number of keys taken before this chunk. The per-key work
-// is ALU only; the few bucket keys are handled afterwards, one set bit at a time.
-template <bool kFull>
-__device__ __forceinline__ void emit_chunk(const uint32_t (&v)[64], int lim, uint32_t thr, uint32_t blo, uint32_t bw,
-                                           int tie_lim, int col_lim, uint32_t* cand, int j0, int pos0, int& eqn,
-                                           uint32_t (&tb)[2]) {
-  uint32_t bb[2] = {0u, 0u};
+// Emit pass, 64 consecutive candidates of a row: bits of the taken keys (key >= thr) in tb and,
+// with kBucket, of the bucket keys (blo <= key <= blo + bw) in bb. ALU only.
+template <bool kFull, bool kBucket>
+__device__ __forceinline__ void emit_bits(const uint32_t (&v)[64], int lim, uint32_t thr, uint32_t blo, uint32_t bw,
+                                          uint32_t (&tb)[2], uint32_t (&bb)[2]) {
 #pragma unroll
   for (int q = 0; q < 64; ++q) {
     const uint32_t key = score_key(__uint_as_float(v[q]));
     const bool in = kFull || q < lim;
     tb[q >> 5] |= (in && key >= thr) ? (1u << (q & 31)) : 0u;
-    bb[q >> 5] |= (in && key - blo <= bw) ? (1u << (q & 31)) : 0u;
+    if (kBucket) bb[q >> 5] |= (in && key - blo <= bw) ? (1u << (q & 31)) : 0u;
   }
-#pragma unroll
-  for (int w = 0; w < 2; ++w) {
-    uint32_t bits = bb[w];
-    while (bits) {
-      const int q = __ffs(bits) - 1;
-      bits &= bits - 1u;
-      if (eqn < tie_lim) tb[w] |= 1u << q;
-      if (eqn < col_lim) {  // collecting (no ties are taken then, so tb holds only keys above)
-        const int before = pos0 + (w ? __popc(tb[0]) : 0) + __popc(tb[w] & ((1u << q) - 1u));
-        cand[3 * eqn] = score_key(__uint_as_float(pick64(v, 32 * w + q)));
-        cand[3 * eqn + 1] = (uint32_t)(j0 + 32 * w + q);
-        cand[3 * eqn + 2] = (uint32_t)before;
-      }
-      ++eqn;
+}
+
+__device__ __forceinline__ bool act_row(bool valid, int m) { return valid && m > 0; }
+
+// The lowest n set bits of x (all of them if n >= popc(x), none if n <= 0).
+__device__ __forceinline__ uint32_t first_bits(uint32_t x, int n) {
+  if (n <= 0) return 0u;
+  if (n >= __popc(x)) return x;
+  return x & ((1u << __fns(x, 0u, n + 1)) - 1u);
+}
+
+// Per-lane bounded wait for the partner half's tie count of a tile: the slot holds
+// (tile + 1) << 8 | count once written. Returns the count, or -1 on giving up.
+__device__ __forceinline__ int wait_tie_count(volatile uint32_t* slot, uint32_t tag, SelShared* sh,
+                                              const int* gstatus) {
+  const uint64_t t0 = tc::globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    const uint32_t v = *slot;
+    if ((v >> 8) == tag) return (int)(v & 255u);
+    if (sh->abort_flag || tc::globaltimer() - t0 > tc::kWaitLimitNs) return -1;
+    if ((it & 1023u) == 0u && tc::grid_timed_out(gstatus)) {
+      sh->abort_flag = 1;
+      return -1;
     }
-  }
-}
-
-// Writes, cooperatively across the warp, the staged block indices of every row whose staging
-// ring holds at least `least` unwritten entries (all of them when least is 1, else 64): each
-// selected row goes out as whole 128-byte lines instead of one scattered 4-byte store per index.
-// Rows are 32 * quad + lane; `out` and the ring state (pos, flushed) belong to the lane's row.
-__device__ __forceinline__ void flush_rows(const uint32_t* hist, int quad, int lane, int32_t* out, int pos,
-                                           int& flushed, int least) {
-  unsigned need = __ballot_sync(0xFFFFFFFFu, pos - flushed >= least);
-  while (need) {
-    const int L = __ffs(need) - 1;
-    need &= need - 1u;
-    const int fl = __shfl_sync(0xFFFFFFFFu, flushed, L);
-    const int cnt = min(64, __shfl_sync(0xFFFFFFFFu, pos, L) - fl);
-    int32_t* rout = reinterpret_cast<int32_t*>(__shfl_sync(0xFFFFFFFFu, reinterpret_cast<long long>(out), L));
-    const uint32_t* ring = hist + (32 * quad + L) * kHistStride + kRing + (fl & 127);
-    if (lane < cnt) rout[fl + lane] = (int32_t)ring[lane];
-    if (lane + 32 < cnt) rout[fl + 32 + lane] = (int32_t)ring[lane + 32];
-    if (lane == L) flushed = fl + cnt;
-  }
-}
-
-// Moves out[lo, hi) up by sh slots (sh >= 1), top down, eight independent loads at a time.
-__device__ __forceinline__ void shift_up(int32_t* out, int lo, int hi, int sh) {
-  int p = hi;
-  while (p - lo >= 8) {
-    int x[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) x[u] = out[p - 1 - u];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) out[p - 1 - u + sh] = x[u];
-    p -= 8;
-  }
-  while (p > lo) {
-    --p;
-    out[p + sh] = out[p];
   }
 }
 
@@ -434,10 +394,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------- epilogue: one row per thread pair ----------------
-    // Warps w and w + 4 read TMEM lane quadrant w % 4 (row r = 32 * (w % 4) + lane); in histogram
-    // passes each takes half of every tile's columns (atomics on the row's shared histogram); in
-    // the emit pass the lower warp streams all columns in order and the upper one only releases
-    // the accumulators.
+    // Warps w and w + 4 read TMEM lane quadrant w % 4 (row r = 32 * (w % 4) + lane); each takes
+    // half of every tile's columns, in the histogram passes and in the emit pass.
     const int quad = warp & 3, half = warp >> 2;
     const int r = quad * 32 + lane;
     const int t = tq0 + r / G, g = r % G;
@@ -449,17 +407,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool done = (rem == nb);
     if (rem == 0) { prefix = 0xFFFFFFFFu; mask = 0xFFFFFFFFu; done = true; }
     uint32_t* my_hist = hist + r * kHistStride;
-    int32_t* out = a.sel + (((long)b * a.sel_T + (t - a.sel_t0)) * G + g) * (long)a.Kb;
+    // the row's bitmap of taken candidates (bit j of word j / 32)
+    uint32_t* brow = a.bits + (((long)b * (a.t_end - a.t_begin) + (t - a.t_begin)) * G + g) * (long)a.bstride;
     const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
     const uint32_t hbase = smem_u32(my_hist);
     long k = 0;
-    uint32_t* ring = my_hist + kRing;  // emit pass: taken indices staged here, 128 in flight at most
-    int pos = 0, flushed = 0;
-    bool aborted = false;
+    bool aborted = false, emitted = false, collect = false;
+    int eqn = 0, taken = 0;
     for (int pass = 0; pass < kMaxPasses; ++pass) {
-      // zero the histograms for this pass, then a barrier+vote: is any row still unresolved?
+      // zero the histograms for this pass (a resolved row: its tie-count slots), then a
+      // barrier+vote: is any row still unresolved?
       if (half == 0 && !done && pass < kMaxPasses - 1)
         for (int i = 0; i < 256; ++i) my_hist[i] = 0;
+      if (half == 0 && done)
+        for (int i = 0; i < 4; ++i) my_hist[i] = 0;
       const int vote = epi_vote_any(sh, 4 * pass, !done, a.status);
       // from the third pass on, if every unresolved row's threshold bucket is small, this pass is
       // the last: it also collects those buckets' keys, which are then resolved exactly
@@ -467,6 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (vote < 0 || vote_big < 0) {
         if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
         sh->abort_flag = 1;
+        aborted = true;
         break;
       }
       const bool is_emit = vote == 0 || vote_big == 0 || pass == kMaxPasses - 1;
@@ -475,24 +437,94 @@ __global__ void __launch_bounds__(kThreads, 1)
         __threadfence_block();
         sh->signals = pass + 1;
       }
-      // emit rule of this row: take keys >= thr; bucket [blo, blo + bw] handled by ties or collection
-      uint32_t thr = 0xFFFFFFFFu, blo = 0xFFFFFFFFu, bw = 0u;
-      int tie_lim = 0, col_lim = 0;
-      if (!done) {  // collecting: everything above the bucket, the bucket's keys kept aside
-        const uint32_t pend = prefix | ~mask;
-        thr = pend == 0xFFFFFFFFu ? 0xFFFFFFFFu : pend + 1u;
-        blo = prefix;
-        bw = ~mask;
-        col_lim = kCap;
-      } else if (rem == nb) {  // the whole bucket is taken
-        thr = prefix;
-      } else {  // fully resolved key with ties: the first rem of them in j order
-        thr = prefix == 0xFFFFFFFFu ? 0xFFFFFFFFu : prefix + 1u;
-        blo = prefix;
-        tie_lim = rem;
+      if (!is_emit) {
+        const int shift = 24 - 8 * pass;
+        // a resolved row matches nothing (its histogram is not read; in the first pass it may
+        // count, harmlessly)
+        const uint32_t mk = done ? 0u : mask, pf = done ? 1u : prefix;
+        for (int i = 0; i < n_nt; ++i, ++k) {
+          const int buf = (int)(k & 1);
+          if (!warp_wait(&sh->acc_full[buf], (uint32_t)((k >> 1) & 1), &sh->abort_flag, a.status)) {
+            if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
+            sh->abort_flag = 1;
+            aborted = true;
+            break;
+          }
+          tc::fence_after_sync();
+          uint32_t v[64];
+          tc::tmem_ld64(tmem + lane_base + (uint32_t)(buf * kN + half * 64), v);
+          tc::fence_before_sync();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&sh->acc_empty[buf]);
+          const int lim = c - (i * kN + half * 64);
+          if (__all_sync(0xFFFFFFFFu, lim >= 64)) {
+            if (pass == 0) hist_chunk<true, true>(v, lim, mk, pf, shift, hbase);
+            else hist_chunk<true, false>(v, lim, mk, pf, shift, hbase);
+          } else if (lim > 0) {
+            if (pass == 0) hist_chunk<false, true>(v, lim, mk, pf, shift, hbase);
+            else hist_chunk<false, false>(v, lim, mk, pf, shift, hbase);
+          }
+        }
+        if (aborted) break;
+        // both halves' histogram updates are complete before either reads the histogram
+        if (epi_vote_any(sh, 4 * pass + 1, false, a.status) < 0) {
+          if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
+          sh->abort_flag = 1;
+          aborted = true;
+          break;
+        }
+        if (!done) {
+          int above = 0;
+          for (int bin = 255; bin >= 0; --bin) {
+            const int h = (int)my_hist[bin];
+            if (above + h >= rem) {
+              prefix |= (uint32_t)bin << shift;
+              mask |= 255u << shift;
+              rem -= above;
+              nb = h;
+              break;
+            }
+            above += h;
+          }
+          done = (rem == nb) || (mask == 0xFFFFFFFFu);
+        }
+        // both halves have read the histogram before the next pass zeroes it
+        if (epi_vote_any(sh, 4 * pass + 2, false, a.status) < 0) {
+          if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
+          sh->abort_flag = 1;
+          aborted = true;
+          break;
+        }
+        continue;
       }
-      int eqn = 0;
-      const int shift = 24 - 8 * pass;
+
+      // ---- emit pass: this half's 64 columns of every tile become two bitmap words ----
+      // rule of this row: take keys >= thr; the bucket [blo, blo + bw] is collected (unresolved
+      // row), taken whole (thr = prefix), or holds exact ties taken in j order up to rem
+      const bool act = valid && m > 0;
+      uint32_t thr = 0xFFFFFFFFu, blo = 0xFFFFFFFFu, bw = 0u;
+      bool ties = false;
+      if (act) {
+        if (!done) {
+          const uint32_t pend = prefix | ~mask;
+          thr = pend == 0xFFFFFFFFu ? 0xFFFFFFFFu : pend + 1u;
+          blo = prefix;
+          bw = ~mask;
+          collect = true;
+        } else if (rem == nb) {
+          thr = prefix;
+        } else {
+          thr = prefix == 0xFFFFFFFFu ? 0xFFFFFFFFu : prefix + 1u;
+          blo = prefix;
+          ties = true;
+        }
+      }
+      // identical in the two warps of a row pair (same rows, same state)
+      const bool any_bucket = __any_sync(0xFFFFFFFFu, collect || ties);
+      const bool any_ties = __any_sync(0xFFFFFFFFu, ties);
+      uint32_t* cand = my_hist + 128 * half;  // collected (key, j) pairs of this half
+      volatile uint32_t* slot = my_hist;      // tie counts: [half][tile parity]
+      int run = 0;                            // exact ties before this half's columns of the tile
       for (int i = 0; i < n_nt; ++i, ++k) {
         const int buf = (int)(k & 1);
         if (!warp_wait(&sh->acc_full[buf], (uint32_t)((k >> 1) & 1), &sh->abort_flag, a.status)) {
@@ -502,136 +534,105 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc::fence_after_sync();
-        if (!is_emit) {
+        const int j0 = i * kN + half * 64;
+        const int lim = act ? c - j0 : 0;
+        uint32_t tb[2] = {0u, 0u}, bb[2] = {0u, 0u};
+        if (__any_sync(0xFFFFFFFFu, lim > 0)) {
           uint32_t v[64];
           tc::tmem_ld64(tmem + lane_base + (uint32_t)(buf * kN + half * 64), v);
-          const int j0 = i * kN + half * 64;
-          const int lim = c - j0;
-          // a resolved row matches nothing (its histogram is not read; in the first pass it may
-          // count, harmlessly)
-          const uint32_t mk = done ? 0u : mask, pf = done ? 1u : prefix;
-          if (__all_sync(0xFFFFFFFFu, lim >= 64)) {
-            if (pass == 0) hist_chunk<true, true>(v, lim, mk, pf, shift, hbase);
-            else hist_chunk<true, false>(v, lim, mk, pf, shift, hbase);
-          } else if (lim > 0) {
-            if (pass == 0) hist_chunk<false, true>(v, lim, mk, pf, shift, hbase);
-            else hist_chunk<false, false>(v, lim, mk, pf, shift, hbase);
+          const bool full = __all_sync(0xFFFFFFFFu, lim >= 64);
+          if (any_bucket) {
+            if (full) emit_bits<true, true>(v, lim, thr, blo, bw, tb, bb);
+            else emit_bits<false, true>(v, lim, thr, blo, bw, tb, bb);
+          } else {
+            if (full) emit_bits<true, false>(v, lim, thr, blo, bw, tb, bb);
+            else emit_bits<false, false>(v, lim, thr, blo, bw, tb, bb);
           }
-        } else if (half == 0) {
-#pragma unroll 1
-          for (int hh = 0; hh < 2; ++hh) {
-            uint32_t v[64];
-            tc::tmem_ld64(tmem + lane_base + (uint32_t)(buf * kN + hh * 64), v);
-            const int j0 = i * kN + hh * 64;
-            const int lim = valid ? c - j0 : 0;
-            uint32_t tb[2] = {0u, 0u};
-            if (__all_sync(0xFFFFFFFFu, lim >= 64))
-              emit_chunk<true>(v, lim, thr, blo, bw, tie_lim, col_lim, my_hist, j0, pos, eqn, tb);
-            else if (lim > 0)
-              emit_chunk<false>(v, lim, thr, blo, bw, tie_lim, col_lim, my_hist, j0, pos, eqn, tb);
-            // stage the taken indices in order, each at the position the population count of
-            // the taken bits below it gives (predicated stores, no loop over set bits), then
-            // write out the rows that have 64 staged
-            const uint32_t ring_base = smem_u32(ring);
+          if (collect) {  // the few bucket keys of an unresolved row, kept as (key, j) pairs
 #pragma unroll
             for (int w = 0; w < 2; ++w) {
-              const uint32_t bits = tb[w];
-              if (__any_sync(0xFFFFFFFFu, bits != 0u)) {
-                const int base = pos;
-#pragma unroll
-                for (int q = 0; q < 32; ++q) {
-                  const int ps = base + __popc(bits & ((1u << q) - 1u));
-                  st_shared_u32_if(ring_base + ((uint32_t)(ps & 127) << 2), (uint32_t)(j0 + 32 * w + q),
-                                   (((bits >> q) & 1u) != 0u && ps < m) ? 1u : 0u);
+              uint32_t bits = bb[w];
+              while (bits) {
+                const int q = __ffs(bits) - 1;
+                bits &= bits - 1u;
+                if (eqn < kCap) {
+                  cand[2 * eqn] = score_key(__uint_as_float(pick64(v, 32 * w + q)));
+                  cand[2 * eqn + 1] = (uint32_t)(j0 + 32 * w + q);
                 }
-                pos = min(m, base + __popc(bits));
+                ++eqn;
               }
             }
-            flush_rows(hist, quad, lane, out, pos, flushed, 64);
           }
         }
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&sh->acc_empty[buf]);
-      }
-      if (aborted) break;
-      if (is_emit) {
-        if (half == 0) {
-          flush_rows(hist, quad, lane, out, pos, flushed, 1);
-          __syncwarp();  // the row's lines written by other lanes are visible to its owner below
-        }
-        if (half == 0 && valid && !done) {
-          // the collected bucket (ascending j): candidate i ranks behind every larger key and every
-          // equal key of lower j, and is chosen when fewer than rem rank ahead of it
-          uint32_t* cand = my_hist;
-          int nch = 0;
-          if (eqn > kCap) report(a.status, SGQA_ERR_DEVICE_CHECK);
-          const int ncand = min(eqn, kCap);
-          for (int ci = 0; ci < ncand; ++ci) {
-            const uint32_t key = cand[3 * ci];
-            int ahead = 0;
-            for (int c2 = 0; c2 < ncand; ++c2) {
-              const uint32_t k2 = cand[3 * c2];
-              ahead += (k2 > key || (k2 == key && c2 < ci)) ? 1 : 0;
+        if (any_ties) {
+          // exact ties in j order: the lower half's columns of tile i precede the upper half's
+          const int cnt = ties ? __popc(bb[0]) + __popc(bb[1]) : 0;
+          int got = 0;
+          if (half == 0) {
+            if (ties) slot[i & 1] = ((uint32_t)(i + 1) << 8) | (uint32_t)cnt;
+            if (ties && i > 0) {
+              got = wait_tie_count(slot + 2 + ((i - 1) & 1), (uint32_t)i, sh, a.status);
+              run += got;
             }
-            if (ahead < rem) {  // keys stay in place; the chosen (j, before) pairs move to the front
-              cand[3 * nch + 1] = cand[3 * ci + 1];
-              cand[3 * nch + 2] = cand[3 * ci + 2];
-              ++nch;
-            }
+          } else if (ties) {
+            got = wait_tie_count(slot + (i & 1), (uint32_t)(i + 1), sh, a.status);
+            run += got;
+            slot[2 + (i & 1)] = ((uint32_t)(i + 1) << 8) | (uint32_t)cnt;
           }
-          if (pos + nch > m) {
-            report(a.status, SGQA_ERR_DEVICE_CHECK);
-            nch = m - pos;
-          }
-          // chosen i (ascending j) lands at before_i + i; the keys taken between before_i and
-          // before_{i+1} move up by i + 1. Done from the last chosen down, so nothing is overwritten.
-          int hi = pos;
-          for (int i = nch - 1; i >= 0; --i) {
-            const int before = min((int)cand[3 * i + 2], hi);
-            shift_up(out, before, hi, i + 1);
-            out[before + i] = (int)cand[3 * i + 1];
-            hi = before;
-          }
-          pos += nch;
-        }
-        if (half == 0 && valid) {
-          if (pos != m) report(a.status, SGQA_ERR_DEVICE_CHECK);
-          out[pos++] = c;
-          for (; pos < a.Kb; ++pos) out[pos] = -1;
-        }
-        break;
-      }
-      // both halves' histogram updates are complete before either reads the histogram
-      if (epi_vote_any(sh, 4 * pass + 1, false, a.status) < 0) {
-        if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
-        sh->abort_flag = 1;
-        break;
-      }
-      if (!done) {
-        int above = 0;
-        for (int bin = 255; bin >= 0; --bin) {
-          const int h = (int)my_hist[bin];
-          if (above + h >= rem) {
-            prefix |= (uint32_t)bin << shift;
-            mask |= 255u << shift;
-            rem -= above;
-            nb = h;
+          if (__any_sync(0xFFFFFFFFu, got < 0)) {
+            if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
+            sh->abort_flag = 1;
+            aborted = true;
             break;
           }
-          above += h;
+          if (ties) {
+            const int n = rem - run;
+            tb[0] |= first_bits(bb[0], n);
+            tb[1] |= first_bits(bb[1], n - __popc(bb[0]));
+            run += cnt;
+          }
         }
-        done = (rem == nb) || (mask == 0xFFFFFFFFu);
+        if (lim > 0) *reinterpret_cast<uint2*>(brow + (j0 >> 5)) = make_uint2(tb[0], tb[1]);
+        taken += __popc(tb[0]) + __popc(tb[1]);
       }
-      // both halves have read the histogram before the next pass zeroes it
-      if (epi_vote_any(sh, 4 * pass + 2, false, a.status) < 0) {
-        if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
-        sh->abort_flag = 1;
-        break;
+      if (!aborted && half == 1 && act) {
+        my_hist[kCnt1] = (uint32_t)eqn;
+        my_hist[kCnt1 + 1] = (uint32_t)taken;
       }
+      emitted = !aborted;
+      break;
+    }
+    // every epilogue warp gets here (all waits above are bounded): the bitmap words and the
+    // collected keys of both halves are complete
+    asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
+    if (emitted && half == 0 && act_row(valid, m) && !sh->abort_flag) {
+      int total = taken + (int)my_hist[kCnt1 + 1];
+      if (collect) {
+        // the collected bucket keys of both halves: key x ranks behind every larger key and every
+        // equal key of lower j, and is taken when fewer than rem rank ahead of it
+        const int e1 = (int)my_hist[kCnt1];
+        if (eqn > kCap || e1 > kCap) report(a.status, SGQA_ERR_DEVICE_CHECK);
+        const int n0 = min(eqn, kCap), n1 = min(e1, kCap);
+        for (int x = 0; x < n0 + n1; ++x) {
+          const uint32_t* px = x < n0 ? my_hist + 2 * x : my_hist + 128 + 2 * (x - n0);
+          const uint32_t kx = px[0], jx = px[1];
+          int ahead = 0;
+          for (int y = 0; y < n0 + n1; ++y) {
+            const uint32_t* py = y < n0 ? my_hist + 2 * y : my_hist + 128 + 2 * (y - n0);
+            ahead += (py[0] > kx || (py[0] == kx && py[1] < jx)) ? 1 : 0;
+          }
+          if (ahead < rem) {
+            atomicOr(brow + (jx >> 5), 1u << (jx & 31u));
+            ++total;
+          }
+        }
+      }
+      if (total != m) report(a.status, SGQA_ERR_DEVICE_CHECK);
     }
   }
-
   tc::fence_before_sync();
   __syncthreads();
   if (warp == kMmaWarp) {
@@ -652,6 +653,46 @@ __global__ void own_block_only_kernel(SelectArgs a) {
     out[0] = t / a.B;
     for (int i = 1; i < a.Kb; ++i) out[i] = -1;
   }
+}
+
+// The selection from the bitmaps: per (token, group) row, the set bits of words [0, ceil(c/32))
+// in ascending order (m of them), then the own block c, then -1 up to Kb. One warp per row: each
+// lane takes one word of every 32, a warp scan of the population counts places its indices.
+__global__ void __launch_bounds__(256) sel_from_bits_kernel(SelectArgs a) {
+  const long row = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int nq = a.t_end - a.t_begin;
+  if (row >= (long)a.batch * nq * a.G) return;
+  const int g = (int)(row % a.G);
+  const long bt = row / a.G;
+  const int t = a.t_begin + (int)(bt % nq);
+  const int b = (int)(bt / nq);
+  const int c = t / a.B, m = min(a.Kb - 1, c);
+  const uint32_t* bits = a.bits + row * (long)a.bstride;
+  int32_t* out = a.sel + (((long)b * a.sel_T + (t - a.sel_t0)) * a.G + g) * (long)a.Kb;
+  const int nw = m > 0 ? (c + 31) >> 5 : 0;
+  int pos = 0;
+  for (int w0 = 0; w0 < nw && pos < m; w0 += 32) {
+    const int w = w0 + lane;
+    uint32_t x = w < nw ? __ldg(bits + w) : 0u;
+    const int n = __popc(x);
+    int inc = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    int p = pos + inc - n;
+    while (x) {
+      const int q = __ffs(x) - 1;
+      x &= x - 1u;
+      if (p < m) out[p] = 32 * w + q;
+      ++p;
+    }
+    pos += __shfl_sync(0xFFFFFFFFu, inc, 31);
+  }
+  if (pos != m && lane == 0) report(a.status, SGQA_ERR_DEVICE_CHECK);
+  for (int i = min(pos, m) + lane; i < a.Kb; i += 32) out[i] = i == m ? c : -1;
 }
 
 using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -703,15 +744,36 @@ cudaError_t launch_di(const SelectArgs& a, cudaStream_t s) {
 
 }  // namespace
 
+void select_bits_dims(int batch, int T, int G, int B, size_t budget, int* bstride, int* bits_q) {
+  const long nblk = T / B;
+  *bstride = (int)(4 * ((nblk + kN - 1) / kN));  // whole tiles: a tile's two words per half stay in the row
+  const size_t per_q = (size_t)batch * G * (size_t)*bstride * 4;
+  long q = per_q ? (long)(budget / per_q) : (long)T;
+  q = q / 128 * 128;  // whole K2 tiles (128 / G tokens) per range
+  if (q < 128) q = 128;
+  if (q > T) q = T;
+  *bits_q = (int)q;
+}
+
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) {
   if (a.t_end <= a.t_begin) return cudaSuccess;
   if (a.T / a.B == 0) {
     own_block_only_kernel<<<148, 256, 0, s>>>(a);
     return cudaGetLastError();
   }
-  if (a.d_idx == 64) return launch_di<64>(a, s);
-  if (a.d_idx == 32) return launch_di<32>(a, s);
-  return cudaErrorInvalidValue;
+  if ((a.d_idx != 64 && a.d_idx != 32) || !a.bits || a.bits_q <= 0) return cudaErrorInvalidValue;
+  // query ranges of at most bits_q rows, each: scores + select into the bitmaps, then the lists
+  for (int t0 = a.t_begin; t0 < a.t_end; t0 += a.bits_q) {
+    SelectArgs p = a;
+    p.t_begin = t0;
+    p.t_end = a.t_end - t0 > a.bits_q ? t0 + a.bits_q : a.t_end;
+    cudaError_t e = a.d_idx == 64 ? launch_di<64>(p, s) : launch_di<32>(p, s);
+    if (e != cudaSuccess) return e;
+    const long rows = (long)p.batch * (p.t_end - p.t_begin) * p.G;
+    sel_from_bits_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace sgqa

@@ -74,7 +74,11 @@ def test_workspace_size_formula(lib):
     al = lambda x: (x + 255) // 256 * 256
     units = 2 * 32768 * 4
     plan = 4 * al(units * 4) + al(8 * 256 * ((32768 + 2047) // 2048) * 4)
-    want = 256 + plan + al(2 * nblk * 64 * 4) + 2 * al(2 * nblk * 64 * 2) + al(2 * 32768 * 4 * 512 * 4)
+    # taken-candidate bitmaps: 4 words per 128 blocks per (token, group), query ranges within 256 MiB
+    bstride = 4 * ((nblk + 127) // 128)
+    bits_q = min(32768, (256 << 20) // (2 * 4 * bstride * 4) // 128 * 128)
+    want = (256 + plan + al(2 * nblk * 64 * 4) + 2 * al(2 * nblk * 64 * 2) + al(2 * bits_q * 4 * bstride * 4)
+            + al(2 * 32768 * 4 * 512 * 4))
     assert sg.sgqa_workspace_size(d) == want
     assert sg.sgqa_decode_workspace_size(D(batch=32, T=(1 << 20) + 8, Hq=32, G=4, d=128, d_idx=64, B=8, k=4096), 4) > 0
     assert sg.sgqa_decode_workspace_size(D(), 0) == 0
