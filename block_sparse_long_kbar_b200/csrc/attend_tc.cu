@@ -11,30 +11,36 @@
 //   * Q tile: 128 rows x d bf16 in shared memory (K-major, 128B swizzle), loaded once.
 //   * The union of the tile's selections is built window by window over block ids (a shared
 //     bitmap of 32-bit query masks per block) and consumed as 16-token superblocks aligned on
-//     block ids, two per chunk. Each chunk's K and V rows of the group arrive by 3-D TMA boxes
-//     (16 tokens x 64 dims, 128B swizzle) into a 3-stage ring; a missing superblock of the last
-//     chunk is loaded from out of bounds, which fills zeros.
-//   * S[128 x 32] = Q K^T per chunk: tcgen05.mma (kind::f16, M=128, N=32) into TMEM, double
+//     block ids, four per chunk. Each chunk's K and V rows of the group arrive by 3-D TMA boxes
+//     (16 tokens x 64 dims, 128B swizzle) into a 2-stage K ring and a 2-stage V ring (a K stage
+//     is reused as soon as Q K^T has read it), with chunks ahead prefetched into L2; a missing
+//     superblock of the last chunk is loaded from out of bounds, which fills zeros.
+//   * S[128 x 64] = Q K^T per chunk: tcgen05.mma (kind::f16, M=128, N=64) into TMEM, double
 //     buffered.
-//   * Softmax: two threads per row (TMEM lane), each taking one of the chunk's two superblocks;
-//     masks from the bitmap (the query selected the block, token <= query position).
-//     Every row is scaled by a reference maximum computed up front on the CUDA cores from its
-//     own block (always selected), so there is a single streaming pass and no rescaling of O:
-//     P = exp2((S - m_ref) log2(e) / sqrt(d)), rounded to bf16 into shared memory. A row whose
-//     sum of P exceeds 2^60 or is not finite is flagged, and if any row is, the tile streams the
-//     union again for exact maxima and then repeats the main pass (flagged rows with their exact
-//     maximum, the others with exactly the same arithmetic as before).
-//   * O[128 x d] += P V with tcgen05.mma (V as an MN-major operand) in TMEM, and the row sums
-//     l[128] += P 1 by one more MMA against a tile of ones, so l adds exactly the bf16 P that O
-//     adds, in the same order. Because superblocks are aligned on block ids, each is one K=16
-//     accumulation step, and unselected slots contribute exact zeros, every row's arithmetic is
-//     the same whatever rows share its tile (bitwise causal, chunk-invariant).
+//   * Softmax: two threads per row (TMEM lane); the thread with shalf = (superblock id & 1)
+//     takes a superblock. Masks from the bitmap (the query selected the block, token <= query
+//     position). Every row is scaled by a reference maximum computed up front on the CUDA cores
+//     from its own block (always selected), so there is a single streaming pass and no rescaling
+//     of O: P = exp2((S - m_ref) log2(e) / sqrt(d)), rounded to bf16 and written back into TMEM
+//     over the superblock's first 8 S columns. A row whose sum of P exceeds 2^60 or is not finite
+//     is flagged, and if any row is, the tile streams the union again for exact maxima and then
+//     repeats the main pass (flagged rows with their exact maximum, the others with exactly the
+//     same arithmetic as before).
+//   * O[128 x d] += P V with tcgen05.mma, P read from TMEM (A operand) and V from shared memory
+//     (an MN-major operand), one K=16 step per superblock. The row sums l add the same bf16 P on
+//     the CUDA cores: each thread sums its superblocks (one id parity) in ascending id order and
+//     l = l_even + l_odd. Because superblocks are aligned on block ids, each is one K=16
+//     accumulation step and one parity class, and unselected slots contribute exact zeros, every
+//     row's arithmetic is the same whatever rows share its tile (bitwise causal, chunk-invariant).
 //   * Epilogue: O / l times sigmoid(gate_logits), bf16.
-// Warp roles: warp 0 issues TMA, warp 1 allocates TMEM and issues MMAs, warps 2-9 run the
-// softmax and the epilogue; all ten build the union. Two tiles are resident per SM (shared memory
-// and TMEM are sized for it), so one tile's union, setup and epilogue overlap the other's chunks. Every wait is bounded by %globaltimer: on
-// expiry the kernel records SGQA_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and
-// returns.
+// Warp roles: warp 0 issues TMA, warp 1 allocates TMEM and issues MMAs (Q K^T of a chunk and
+// P V of an earlier one, whichever is ready first; neither role blocks on one barrier while the
+// other kind of work could proceed; an S/P buffer is refilled only after the P V that reads it
+// has been issued, and MMAs of one thread execute in issue order), warps 2-9 run the softmax and
+// the epilogue; all ten build the union. Two tiles are resident per SM (shared memory and TMEM
+// are sized for it), so one tile's union, setup and epilogue overlap the other's chunks. Every
+// wait is bounded by %globaltimer: on expiry the kernel records SGQA_ERR_TIMEOUT, drains its own
+// copies and MMAs, frees TMEM and returns.
 #include <cmath>
 #include <cuda.h>
 
@@ -46,12 +52,13 @@ namespace sgqa {
 namespace {
 
 constexpr int kUnit = 16;    // tokens per superblock
-constexpr int kCH = 2;       // superblocks per chunk (one handshake between MMA and softmax)
+constexpr int kCH = 4;       // superblocks per chunk (one handshake between MMA and softmax)
 constexpr int kCT = kCH * kUnit;  // token slots per chunk
 constexpr int kWin = 1024;   // block ids per union window
 constexpr int kWinWords = 16;     // occupancy bits for up to 512 windows
-constexpr int kNS = 3;       // K/V chunk stages
-constexpr int kPB = 2;       // P buffers in shared memory
+constexpr int kNK = 2;       // K chunk stages
+constexpr int kNV = 2;       // V chunk stages
+constexpr int kPF = 2;       // chunks ahead of the current K load that are prefetched into L2
 constexpr int kSmWarps = 8;  // softmax warps: two per TMEM lane quadrant
 constexpr int kThreads = (2 + kSmWarps) * 32;
 constexpr int kCtasPerSm = 2;  // two tiles resident per SM: one's union, setup and epilogue overlap
@@ -67,22 +74,19 @@ struct AtcCfg {
   static constexpr int kHalves = D / 64;
   static constexpr int kQ = kM * D * 2;                 // [half][128 rows][128 B]
   static constexpr int kHalfRows = kCT * 128;           // one 64-dim half of a chunk: [kCT tokens][128 B]
-  static constexpr int kKc = kHalves * kHalfRows;       // K (or V) of one chunk: [half][64][128 B]
-  static constexpr int kStage = 2 * kKc;                // K then V
-  static constexpr int kPsb = kM * kUnit * 2;           // P of one superblock: 128 x 16 bf16
-  static constexpr int kP = kCH * kPsb;                 // P of one chunk
-  static constexpr int kOnes = 16 * 128;                // 16 x 64 bf16 ones: B operand of the row-sum MMA
-  static constexpr int kSmem = 1024 + kQ + kNS * kStage + kPB * kP + kOnes + 2 * kWin * 4 + 4096;
+  static constexpr int kKc = kHalves * kHalfRows;       // K (or V) of one chunk: [half][kCT][128 B]
+  static constexpr int kSmem = 1024 + kQ + (kNK + kNV) * kKc + 2 * kWin * 4 + 4096;
   static_assert(kCtasPerSm * (kSmem + 1024) <= 233472, "shared memory for the resident tiles");
-  static constexpr int kSCols = 2 * kCT;                // TMEM: S buffers, then O (D), then l (16)
-  static constexpr int kTmemCols = kSCols + D + 16 <= 256 ? 256 : 512;
+  static constexpr int kSCols = 2 * kCT;                // TMEM: two S/P buffers, then O (D)
+  static constexpr int kTmemCols = kSCols + D <= 256 ? 256 : 512;
   static_assert(kCtasPerSm * kTmemCols <= 512, "TMEM for the resident tiles");
 };
 
 struct AtcShared {
-  uint64_t kv_full[kNS], kv_empty[kNS], s_full[2], s_empty[2], p_full[kPB], p_empty[kPB], o_done;
+  uint64_t k_full[kNK], k_empty[kNK], v_full[kNV], v_empty[kNV], s_full[2], p_full[2], o_done;
   float ref_part[2][kM];  // per-row reference maxima from the own block (two halves of its tokens)
   float max_part[2][kM];  // per-row exact maxima by superblock parity (fallback pass)
+  float l_part[2][kM];    // per-row sums of P by superblock parity
   uint32_t wbits[kWinWords];
   uint32_t tmem;
   volatile int abort_flag;
@@ -90,6 +94,26 @@ struct AtcShared {
   int scan[kThreads / 32];
   int nu, maxc, all_windows;
 };
+static_assert(sizeof(AtcShared) <= 4096, "the shared-memory budget reserves 4 KB for AtcShared");
+
+// Idle step of a polling role (producer, MMA issuer): sleep briefly; every 256 idle rounds check
+// for a grid-wide timeout and for no progress within the wait limit (then record the timeout and
+// raise the CTA's abort flag). Returns false when the role must stop.
+__device__ __forceinline__ bool poll_idle(uint32_t spins, uint64_t t_prog, AtcShared* sh, int* gstatus) {
+  if ((spins & 255u) == 0u) {
+    if (tc::grid_timed_out(gstatus)) {
+      sh->abort_flag = 1;
+      return false;
+    }
+    if (tc::globaltimer() - t_prog > tc::kWaitLimitNs) {
+      if (!sh->abort_flag) report(gstatus, SGQA_ERR_TIMEOUT);
+      sh->abort_flag = 1;
+      return false;
+    }
+  }
+  __nanosleep(20);
+  return true;
+}
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, const int* gstatus) {
   int ok = 1;
@@ -142,10 +166,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_align<1024>(smem_raw);
   uint8_t* sQ = smem;
-  uint8_t* sKV = sQ + C::kQ;                             // [stage][K|V][half][kCT tokens][128 B]
-  uint8_t* sP = sKV + kNS * C::kStage;                   // [kPB][superblock][16 groups][2][8 rows][16 B]
-  uint8_t* sOnes = sP + kPB * C::kP;                     // [16 rows][128 B] of bf16 1.0
-  uint32_t* wmask = reinterpret_cast<uint32_t*>(sOnes + C::kOnes);
+  uint8_t* sK = sQ + C::kQ;                              // [kNK][half][kCT tokens][128 B]
+  uint8_t* sV = sK + kNK * C::kKc;                       // [kNV][half][kCT tokens][128 B]
+  uint32_t* wmask = reinterpret_cast<uint32_t*>(sV + kNV * C::kKc);
   int32_t* usb = reinterpret_cast<int32_t*>(wmask + kWin);
   AtcShared* sh = reinterpret_cast<AtcShared*>(usb + kWin);
 
@@ -158,17 +181,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   // do nothing (the decision is the CTA's, before any barrier or TMEM is set up)
   if (__syncthreads_or(tid == 0 && tc::grid_timed_out(a.status))) return;
   if (tid == 0) {
-    for (int i = 0; i < kNS; ++i) {
-      tc::mbar_init(&sh->kv_full[i], 1);
-      tc::mbar_init(&sh->kv_empty[i], 1);
+    for (int i = 0; i < kNK; ++i) {
+      tc::mbar_init(&sh->k_full[i], 1);
+      tc::mbar_init(&sh->k_empty[i], 1);
+    }
+    for (int i = 0; i < kNV; ++i) {
+      tc::mbar_init(&sh->v_full[i], 1);
+      tc::mbar_init(&sh->v_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&sh->s_full[i], 1);
-      tc::mbar_init(&sh->s_empty[i], kSmWarps);
-    }
-    for (int i = 0; i < kPB; ++i) {
       tc::mbar_init(&sh->p_full[i], kSmWarps);
-      tc::mbar_init(&sh->p_empty[i], 1);
     }
     tc::mbar_init(&sh->o_done, 1);
     sh->abort_flag = 0;
@@ -178,7 +201,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   }
   if (tid < kWinWords) sh->wbits[tid] = 0;
   for (int i = tid; i < kWin; i += kThreads) wmask[i] = 0;
-  for (int i = tid; i < C::kOnes / 4; i += kThreads) reinterpret_cast<uint32_t*>(sOnes)[i] = 0x3F803F80u;
   __syncthreads();
   if (tid < QT) {
     const int idx = tile * QT + tid;
@@ -221,8 +243,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = sh->tmem;
-  const uint32_t tmem_o = tmem + C::kSCols;  // O: D columns after the two S buffers
-  const uint32_t tmem_l = tmem_o + D;        // row sums of P: 16 columns (all equal)
+  const uint32_t tmem_o = tmem + C::kSCols;  // O: D columns after the two S/P buffers
 
   // softmax role state (warps 2..9): TMEM lane quadrant warp % 4; `shalf` also picks the
   // half of every chunk (superblocks 2 shalf, 2 shalf + 1) and the own-block tokens this thread
@@ -274,14 +295,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   int o_phase = 0, o_commits = 0;
 
   const int spb = kUnit >> lb;  // blocks per superblock
-  long kc = 0;                  // chunks streamed (producer & MMA ring position)
-  long scnt = 0;                // S buffer uses (MMA & softmax)
-  long pcnt = 0;                // P buffer uses (MMA & softmax)
+  long kck = 0, kcv = 0;        // K and V ring positions (producer & MMA: chunks loaded / consumed)
+  long scnt = 0;                // S/P buffer uses (MMA: Q K^T issued; softmax: chunks processed)
+  long pcnt = 0;                // S/P buffer uses whose P (or exact-max pass) the MMA issuer consumed
   const uint32_t idesc_s = tc::idesc_bf16_f32(kM, kCT);
   const uint32_t idesc_pv = tc::idesc_bf16_f32(kM, D, true);
-  const uint32_t idesc_l = tc::idesc_bf16_f32(kM, 16);
-  const uint64_t d_ones = tc::smem_desc_kmajor(sOnes, 128);
   bool rerun = false;
+  float l_sum = 0.f;            // this thread's sum of P (its superblock parity), per main pass
 
   // pass 0: main (P V with the reference maximum); passes 1-2 only if some row was risky:
   // exact maxima, then the main pass again (risky rows use their exact maximum, all other rows
@@ -291,6 +311,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const bool main_pass = pass != 1;
     bool first_pv = true;
     if (main_pass && pass == 2) m_use = risky ? m_exact : m_ref;
+    l_sum = 0.f;
     for (int win = 0; win < nwin; ++win) {
       if (!sh->all_windows && !((sh->wbits[win >> 5] >> (win & 31)) & 1u)) continue;  // uniform
       const int w0 = win * kWin, w1 = w0 + kWin;
@@ -345,90 +366,136 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
       if (warp == 0) {
         // ---- TMA producer: one chunk = kCH superblocks; missing ones (partial last chunk) are
-        // loaded from out of bounds, which fills zeros ----
+        // loaded from out of bounds, which fills zeros. K and V have rings of their own (a K
+        // stage is free once Q K^T has read it, a V stage once P V has), and the thread issues
+        // whichever load has a free stage, never blocking on one ring while the other could
+        // move. Every K load also prefetches into L2 the chunk kPF ahead. ----
         if (lane == 0) {
-          for (int ch = 0; ch < nch && !sh->abort_flag; ++ch, ++kc) {
-            const int st = (int)(kc % kNS);
-            if (kc >= kNS && !tc::mbar_wait(&sh->kv_empty[st], (uint32_t)(((kc / kNS) - 1) & 1), &sh->abort_flag, a.status)) {
-              if (!sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
-              sh->abort_flag = 1;
-              break;
-            }
-            uint8_t* dst = sKV + st * C::kStage;
-            tc::mbar_arrive_expect_tx(&sh->kv_full[st], main_pass ? C::kStage : C::kKc);
+          int nk = 0, nv = 0;
+          uint64_t t_prog = tc::globaltimer();
+          uint32_t spins = 0;
+          auto chunk_z = [&](int e) { return e < nu ? b * a.T_kv + usb[e] * kUnit : 0x7FFFFFF0; };
+          while (!sh->abort_flag && (nk < nch || (main_pass && nv < nch))) {
+            bool prog = false;
+            if (nk < nch && (kck < kNK || tc::mbar_try_wait(&sh->k_empty[kck % kNK], (uint32_t)(((kck / kNK) - 1) & 1)))) {
+              const int st = (int)(kck % kNK);
+              uint8_t* dst = sK + st * C::kKc;
+              tc::mbar_arrive_expect_tx(&sh->k_full[st], C::kKc);
 #pragma unroll
-            for (int i = 0; i < kCH; ++i) {
-              const int e = ch * kCH + i;
-              const int z = e < nu ? b * a.T_kv + usb[e] * kUnit : 0x7FFFFFF0;
+              for (int i = 0; i < kCH; ++i) {
+                const int z = chunk_z(nk * kCH + i);
 #pragma unroll
-              for (int h = 0; h < C::kHalves; ++h) {
-                tc::tma_load_3d(dst + h * C::kHalfRows + i * (kUnit * 128), &map_k, &sh->kv_full[st], h * 64, g, z);
-                if (main_pass)
-                  tc::tma_load_3d(dst + C::kKc + h * C::kHalfRows + i * (kUnit * 128), &map_v, &sh->kv_full[st], h * 64,
-                                  g, z);
+                for (int h = 0; h < C::kHalves; ++h)
+                  tc::tma_load_3d(dst + h * C::kHalfRows + i * (kUnit * 128), &map_k, &sh->k_full[st], h * 64, g, z);
               }
+#pragma unroll
+              for (int i = 0; i < kCH; ++i) {
+                const int e = (nk + kPF) * kCH + i;
+                if (e < nu) {
+#pragma unroll
+                  for (int h = 0; h < C::kHalves; ++h) {
+                    tc::tma_prefetch_3d(&map_k, h * 64, g, b * a.T_kv + usb[e] * kUnit);
+                    if (main_pass) tc::tma_prefetch_3d(&map_v, h * 64, g, b * a.T_kv + usb[e] * kUnit);
+                  }
+                }
+              }
+              ++nk;
+              ++kck;
+              prog = true;
+            }
+            if (main_pass && nv < nk &&
+                (kcv < kNV || tc::mbar_try_wait(&sh->v_empty[kcv % kNV], (uint32_t)(((kcv / kNV) - 1) & 1)))) {
+              const int st = (int)(kcv % kNV);
+              uint8_t* dst = sV + st * C::kKc;
+              tc::mbar_arrive_expect_tx(&sh->v_full[st], C::kKc);
+#pragma unroll
+              for (int i = 0; i < kCH; ++i) {
+                const int z = chunk_z(nv * kCH + i);
+#pragma unroll
+                for (int h = 0; h < C::kHalves; ++h)
+                  tc::tma_load_3d(dst + h * C::kHalfRows + i * (kUnit * 128), &map_v, &sh->v_full[st], h * 64, g, z);
+              }
+              ++nv;
+              ++kcv;
+              prog = true;
+            }
+            if (prog) {
+              t_prog = tc::globaltimer();
+              spins = 0;
+            } else if (!poll_idle(++spins, t_prog, sh, a.status)) {
+              break;
             }
           }
         }
       } else if (warp == 1) {
-        // ---- MMA issuer ----
+        // ---- MMA issuer: Q K^T of the next chunk as soon as its K is there and the S/P buffer it
+        // reuses has been read (its softmax done and, in a main pass, its P V issued: MMAs of this
+        // thread execute in issue order), and P V of the oldest chunk whose P and V are there,
+        // whichever is ready first ----
         if (lane == 0) {
-          long pend_stage = -1;  // ring position of the chunk whose P V is still to issue
-          auto issue_pv = [&](long stage_of) -> bool {
-            const int pb = (int)(pcnt % kPB);
-            if (!tc::mbar_wait(&sh->p_full[pb], (uint32_t)((pcnt / kPB) & 1), &sh->abort_flag, a.status)) return false;
-            tc::fence_after_sync();
-            const int st = (int)(stage_of % kNS);
-            const uint8_t* vbase = sKV + st * C::kStage + C::kKc;
+          int nq = 0, np = 0;
+          uint64_t t_prog = tc::globaltimer();
+          uint32_t spins = 0;
+          while (!sh->abort_flag && np < nch) {
+            bool prog = false;
+            if (nq < nch && nq < np + 2) {
+              const int st = (int)(kck % kNK);
+              const int sb = (int)(scnt & 1);
+              if (tc::mbar_try_wait(&sh->k_full[st], (uint32_t)((kck / kNK) & 1))) {
+                tc::fence_after_sync();
+                const uint8_t* kst = sK + st * C::kKc;
 #pragma unroll
-            for (int i = 0; i < kCH; ++i) {
-              const uint64_t dp = tc::smem_desc_kmajor_noswz(sP + pb * C::kP + i * C::kPsb, 128, 256);
-              const uint64_t dv = tc::smem_desc_mnmajor_sw128(vbase + i * (kUnit * 128), C::kHalfRows, 1024);
-              const uint32_t acc = first_pv ? 0u : 1u;
-              tc::mma_bf16_ss(tmem_o, dp, dv, idesc_pv, acc);
-              tc::mma_bf16_ss(tmem_l, dp, d_ones, idesc_l, acc);  // l += P 1: the row sums, same order as O
-              first_pv = false;
+                for (int kk = 0; kk < D / 16; ++kk) {
+                  const int h = kk >> 2, off = (kk & 3) * 32;
+                  const uint64_t da = tc::smem_desc_kmajor(sQ + h * (kM * 128) + off, 128);
+                  const uint64_t db = tc::smem_desc_kmajor(kst + h * C::kHalfRows + off, 128);
+                  tc::mma_bf16_ss(tmem + (uint32_t)(sb * kCT), da, db, idesc_s, kk > 0 ? 1u : 0u);
+                }
+                tc::mma_commit(&sh->s_full[sb]);
+                tc::mma_commit(&sh->k_empty[st]);
+                ++nq;
+                ++kck;
+                ++scnt;
+                prog = true;
+              }
             }
-            tc::mma_commit(&sh->kv_empty[st]);
-            tc::mma_commit(&sh->p_empty[pb]);
-            ++pcnt;
-            return true;
-          };
-          bool ok = true;
-          for (int ch = 0; ch < nch && ok && !sh->abort_flag; ++ch, ++kc, ++scnt) {
-            const int st = (int)(kc % kNS);
-            const int sb = (int)(scnt & 1);
-            if (!tc::mbar_wait(&sh->kv_full[st], (uint32_t)((kc / kNS) & 1), &sh->abort_flag, a.status) ||
-                (scnt >= 2 && !tc::mbar_wait(&sh->s_empty[sb], (uint32_t)(((scnt >> 1) - 1) & 1), &sh->abort_flag, a.status))) {
-              ok = false;
+            if (np < nq) {
+              // chunk np: its S/P buffer is (pcnt & 1); pcnt counts buffer uses like scnt
+              const int pb = (int)(pcnt & 1);
+              const int st = (int)(kcv % kNV);
+              if (tc::mbar_try_wait(&sh->p_full[pb], (uint32_t)((pcnt >> 1) & 1)) &&
+                  (!main_pass || tc::mbar_try_wait(&sh->v_full[st], (uint32_t)((kcv / kNV) & 1)))) {
+                tc::fence_after_sync();
+                if (main_pass) {
+                  const uint8_t* vbase = sV + st * C::kKc;
+#pragma unroll
+                  for (int i = 0; i < kCH; ++i) {
+                    if (np * kCH + i >= nu) break;  // missing superblocks: P and V are zero
+                    const uint32_t pa = tmem + (uint32_t)(pb * kCT + i * kUnit);
+                    const uint64_t dv = tc::smem_desc_mnmajor_sw128(vbase + i * (kUnit * 128), C::kHalfRows, 1024);
+                    tc::mma_bf16_ts(tmem_o, pa, dv, idesc_pv, first_pv ? 0u : 1u);
+                    first_pv = false;
+                  }
+                  tc::mma_commit(&sh->v_empty[st]);
+                  ++kcv;
+                }
+                ++np;
+                ++pcnt;
+                prog = true;
+              }
+            }
+            if (prog) {
+              t_prog = tc::globaltimer();
+              spins = 0;
+            } else if (!poll_idle(++spins, t_prog, sh, a.status)) {
               break;
             }
-            tc::fence_after_sync();
-            const uint8_t* kst = sKV + st * C::kStage;
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const int h = kk >> 2, off = (kk & 3) * 32;
-              const uint64_t da = tc::smem_desc_kmajor(sQ + h * (kM * 128) + off, 128);
-              const uint64_t db = tc::smem_desc_kmajor(kst + h * C::kHalfRows + off, 128);
-              tc::mma_bf16_ss(tmem + (uint32_t)(sb * kCT), da, db, idesc_s, kk > 0 ? 1u : 0u);
-            }
-            tc::mma_commit(&sh->s_full[sb]);
-            if (!main_pass) {
-              tc::mma_commit(&sh->kv_empty[st]);
-            } else {
-              if (pend_stage >= 0 && !issue_pv(pend_stage)) { ok = false; break; }
-              pend_stage = kc;
-            }
-          }
-          if (ok && main_pass && pend_stage >= 0 && !sh->abort_flag) ok = issue_pv(pend_stage);
-          if (!ok) {
-            if (!sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
-            sh->abort_flag = 1;
           }
         }
       } else {
-        // ---- softmax: one row per thread pair, each taking half of every chunk (the split
-        // does not enter the arithmetic: P is elementwise, the row sums come from the MMA) ----
+        // ---- softmax: one row per thread pair; the thread with shalf = (superblock id & 1) takes
+        // a superblock: its 16 S columns become 8 columns of bf16 P in place (TMEM) and the same
+        // bf16 values are added to the thread's row sum, in token order ----
         for (int ch = 0; ch < nch; ++ch, ++scnt) {
           const int sb = (int)(scnt & 1);
           if (!warp_wait(&sh->s_full[sb], (uint32_t)((scnt >> 1) & 1), &sh->abort_flag, a.status)) {
@@ -437,42 +504,31 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             break;
           }
           tc::fence_after_sync();
-          constexpr int kHalfCT = kCT / 2;
-          uint32_t v[kHalfCT];
-          static_assert(kHalfCT == 16, "one superblock of S per softmax thread and chunk");
-          tc::tmem_ld16(tmem + lane_base + (uint32_t)(sb * kCT + shalf * kHalfCT), v);
-          tc::fence_before_sync();
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(&sh->s_empty[sb]);
-          const int pb = (int)(pcnt % kPB);
-          if (main_pass && pcnt >= kPB &&
-              !warp_wait(&sh->p_empty[pb], (uint32_t)(((pcnt / kPB) - 1) & 1), &sh->abort_flag, a.status)) {
-            if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
-            sh->abort_flag = 1;
-            break;
-          }
           const float base = m_use * sc;
-#pragma unroll
-          for (int ii = 0; ii < kCH / 2; ++ii) {
-            const int i = shalf * (kCH / 2) + ii;
+#pragma unroll 1
+          for (int i = 0; i < kCH; ++i) {
             const int e = ch * kCH + i;
-            const int sbid = e < nu ? usb[e] : -1;
+            if (e >= nu) break;                 // warp-uniform
+            const int sbid = usb[e];
+            if ((sbid & 1) != shalf) continue;  // warp-uniform
+            const uint32_t col = tmem + lane_base + (uint32_t)(sb * kCT + i * kUnit);
+            uint32_t v[kUnit];
+            tc::tmem_ld16(col, v);
             const int u0 = sbid * kUnit;
-            const bool live = sbid >= 0 && t_r >= 0;
+            const bool live = t_r >= 0;
             uint32_t pk[8];
             if (main_pass && lb >= 3 && live && u0 + (kUnit - 1) <= t_r && u0 >= lo_r) {
               // blocks of 8 or 16 tokens wholly before the row's token (and inside its window, if
-              // any): the selection bit of each
-              // half superblock becomes the additive term of the exponent (-inf when unselected,
-              // whose exp2 is an exact 0); no per-token mask
+              // any): the selection bit of each half superblock becomes the additive term of the
+              // exponent (-inf when unselected, whose exp2 is an exact 0); no per-token mask
               const int jb = (u0 >> lb) - w0;
               const float bias0 = ((wmask[jb] >> q_r) & 1u) ? -base : -INFINITY;
               const float bias1 = ((wmask[jb + spb - 1] >> q_r) & 1u) ? -base : -INFINITY;
 #pragma unroll
               for (int k2 = 0; k2 < 8; ++k2) {
                 const float bias = k2 < 4 ? bias0 : bias1;
-                const float ta = fmaf(__uint_as_float(v[ii * kUnit + 2 * k2]), sc, bias);
-                const float tb = fmaf(__uint_as_float(v[ii * kUnit + 2 * k2 + 1]), sc, bias);
+                const float ta = fmaf(__uint_as_float(v[2 * k2]), sc, bias);
+                const float tb = fmaf(__uint_as_float(v[2 * k2 + 1]), sc, bias);
                 pk[k2] = pack_bf16x2(ex2_approx(ta), ex2_approx(tb));
               }
             } else {
@@ -490,28 +546,31 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
               if (!main_pass) {
 #pragma unroll
                 for (int k2 = 0; k2 < kUnit; ++k2)
-                  if ((vmask >> k2) & 1u) m_exact = fmaxf(m_exact, __uint_as_float(v[ii * kUnit + k2]));
+                  if ((vmask >> k2) & 1u) m_exact = fmaxf(m_exact, __uint_as_float(v[k2]));
                 continue;
               }
-              // masked slots get -inf, whose exp2 is an exact 0; the row sums come from the MMA
+              // masked slots get -inf, whose exp2 is an exact 0
 #pragma unroll
               for (int k2 = 0; k2 < 8; ++k2) {
                 const bool va = (vmask >> (2 * k2)) & 1u, vb = (vmask >> (2 * k2 + 1)) & 1u;
-                const float ta = va ? fmaf(__uint_as_float(v[ii * kUnit + 2 * k2]), sc, -base) : -INFINITY;
-                const float tb = vb ? fmaf(__uint_as_float(v[ii * kUnit + 2 * k2 + 1]), sc, -base) : -INFINITY;
+                const float ta = va ? fmaf(__uint_as_float(v[2 * k2]), sc, -base) : -INFINITY;
+                const float tb = vb ? fmaf(__uint_as_float(v[2 * k2 + 1]), sc, -base) : -INFINITY;
                 pk[k2] = pack_bf16x2(ex2_approx(ta), ex2_approx(tb));
               }
             }
-            uint8_t* prow = sP + pb * C::kP + i * C::kPsb + (r >> 3) * 256 + (r & 7) * 16;
-            *reinterpret_cast<uint4*>(prow) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            *reinterpret_cast<uint4*>(prow + 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            tc::tmem_st8(col, pk);
+#pragma unroll
+            for (int k2 = 0; k2 < 8; ++k2) {
+              l_sum += bf16_lo(pk[k2]);
+              l_sum += bf16_hi(pk[k2]);
+            }
           }
-          if (main_pass) {
-            tc::fence_proxy_async();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&sh->p_full[pb]);
-            ++pcnt;
-          }
+          // P of this chunk is in TMEM (or, in the exact-maximum pass, S has been read): the MMA
+          // issuer may take the buffer
+          tc::tmem_wait_st();
+          tc::fence_before_sync();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&sh->p_full[sb]);
         }
       }
       __syncthreads();
@@ -532,14 +591,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         if (!o_ok) {
           if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
           sh->abort_flag = 1;
-        } else if (pass == 0) {
-          tc::fence_after_sync();
-          uint32_t lv[16];
-          tc::tmem_ld16(tmem_l + lane_base, lv);
-          risky = !(__uint_as_float(lv[0]) <= kRiskSum);
         }
+        sh->l_part[shalf][r] = l_sum;
       }
       o_phase ^= 1;
+      __syncthreads();
+      if (is_sm && pass == 0) risky = !(sh->l_part[0][r] + sh->l_part[1][r] <= kRiskSum);
     }
     if (pass == 0) {
       rerun = __syncthreads_or(is_sm && risky) != 0;
@@ -554,9 +611,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   if (is_sm) {
     if (o_ok) {
       tc::fence_after_sync();
-      uint32_t lv[16];
-      tc::tmem_ld16(tmem_l + lane_base, lv);
-      const float l_r = __uint_as_float(lv[0]);
+      const float l_r = sh->l_part[0][r] + sh->l_part[1][r];
       const float inv = l_r > 0.f ? 1.f / l_r : 0.f;
       const long orow = t_r >= 0 ? ((long)b * a.nQ + (t_r - a.q_t0)) * a.Hq + (long)g * R + h_r : -1;
 #pragma unroll 1
@@ -588,10 +643,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   // ---- drain and release ----
   if (warp == 0 && lane == 0) {
     // copies issued for the last stages must land before the CTA exits
-    for (long k2 = kc - kNS; k2 < kc; ++k2) {
+    for (long k2 = kck - kNK; k2 < kck; ++k2) {
       if (k2 < 0) continue;
       volatile int no_abort = 0;
-      tc::mbar_wait(&sh->kv_full[k2 % kNS], (uint32_t)((k2 / kNS) & 1), &no_abort);
+      tc::mbar_wait(&sh->k_full[k2 % kNK], (uint32_t)((k2 / kNK) & 1), &no_abort);
+    }
+    for (long k2 = kcv - kNV; k2 < kcv; ++k2) {
+      if (k2 < 0) continue;
+      volatile int no_abort = 0;
+      tc::mbar_wait(&sh->v_full[k2 % kNV], (uint32_t)((k2 / kNV) & 1), &no_abort);
     }
   }
   if (warp == 1 && lane == 0 && o_commits > 0) {  // every MMA issued must finish before TMEM is freed
