@@ -12,8 +12,10 @@
 //   * The union of the tile's selections is built window by window over block ids (a shared
 //     bitmap of 32-bit query masks per block) and consumed as 16-token superblocks aligned on
 //     block ids, four per chunk. Each chunk's K and V rows of the group arrive by 3-D TMA boxes
-//     (16 tokens x 64 dims, 128B swizzle) into a 2-stage K ring and a 2-stage V ring (a K stage
-//     is reused as soon as Q K^T has read it), with chunks ahead prefetched into L2; a missing
+//     (64 dims x 16, 32 or 64 tokens, 128B swizzle) into a 2-stage K ring and a 2-stage V ring
+//     (a K stage is reused as soon as Q K^T has read it). A run of consecutive superblock ids in
+//     a chunk (the common case: selections cluster) is fetched by one box per 64-dim half, since
+//     every box costs the issuing thread about 100 cycles whatever its size; a missing
 //     superblock of the last chunk is loaded from out of bounds, which fills zeros.
 //   * S[128 x 64] = Q K^T per chunk: tcgen05.mma (kind::f16, M=128, N=64) into TMEM, double
 //     buffered.
@@ -58,7 +60,6 @@ constexpr int kWin = 1024;   // block ids per union window
 constexpr int kWinWords = 16;     // occupancy bits for up to 512 windows
 constexpr int kNK = 2;       // K chunk stages
 constexpr int kNV = 2;       // V chunk stages
-constexpr int kPF = 2;       // chunks ahead of the current K load that are prefetched into L2
 constexpr int kSmWarps = 8;  // softmax warps: two per TMEM lane quadrant
 constexpr int kThreads = (2 + kSmWarps) * 32;
 constexpr int kCtasPerSm = 2;  // two tiles resident per SM: one's union, setup and epilogue overlap
@@ -80,6 +81,13 @@ struct AtcCfg {
   static constexpr int kSCols = 2 * kCT;                // TMEM: two S/P buffers, then O (D)
   static constexpr int kTmemCols = kSCols + D <= 256 ? 256 : 512;
   static_assert(kCtasPerSm * kTmemCols <= 512, "TMEM for the resident tiles");
+};
+
+// K and V maps with boxes of 16, 32 and 64 tokens (one, two or four superblocks); boxes longer
+// than the tensor's token count are not encoded and not used (max_run).
+struct KvMaps {
+  CUtensorMap k[3], v[3];
+  int max_run;  // largest usable box: 16 << max_run tokens
 };
 
 struct AtcShared {
@@ -159,8 +167,8 @@ __device__ __forceinline__ void for_each_selected(const int32_t* row, int Kb, in
 
 template <int D, int R>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
-    attend_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
-                     AttendArgs a, const uint32_t* __restrict__ perm, int n_per_seg, int tiles_per_seg, int lb) {
+    attend_tc_kernel(const __grid_constant__ KvMaps maps, AttendArgs a, const uint32_t* __restrict__ perm,
+                     int n_per_seg, int tiles_per_seg, int lb) {
   using C = AtcCfg<D>;
   constexpr int QT = kM / R;  // queries per tile (<= 32)
   extern __shared__ uint8_t smem_raw[];
@@ -369,36 +377,36 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         // loaded from out of bounds, which fills zeros. K and V have rings of their own (a K
         // stage is free once Q K^T has read it, a V stage once P V has), and the thread issues
         // whichever load has a free stage, never blocking on one ring while the other could
-        // move. Every K load also prefetches into L2 the chunk kPF ahead. ----
+        // move. ----
         if (lane == 0) {
           int nk = 0, nv = 0;
           uint64_t t_prog = tc::globaltimer();
           uint32_t spins = 0;
-          auto chunk_z = [&](int e) { return e < nu ? b * a.T_kv + usb[e] * kUnit : 0x7FFFFFF0; };
+          // one chunk of K or V: a box per run of consecutive superblock ids (4, 2 or 1 of them,
+          // aligned in the chunk) and 64-dim half
+          auto load_chunk = [&](uint8_t* dst, const CUtensorMap* m, uint64_t* bar, int chunk) {
+            const int e0 = chunk * kCH;
+            for (int i = 0; i < kCH;) {
+              const int e = e0 + i;
+              int mi = 0;  // box of 16 << mi tokens
+              if (e < nu) {
+                if (maps.max_run >= 2 && i == 0 && e + 3 < nu && usb[e + 3] == usb[e] + 3) mi = 2;
+                else if (maps.max_run >= 1 && (i & 1) == 0 && e + 1 < nu && usb[e + 1] == usb[e] + 1) mi = 1;
+              }
+              const int z = e < nu ? b * a.T_kv + usb[e] * kUnit : 0x7FFFFFF0;
+#pragma unroll
+              for (int h = 0; h < C::kHalves; ++h)
+                tc::tma_load_3d(dst + h * C::kHalfRows + i * (kUnit * 128), &m[mi], bar, h * 64, g, z);
+              i += 1 << mi;
+            }
+          };
           while (!sh->abort_flag && (nk < nch || (main_pass && nv < nch))) {
             bool prog = false;
             if (nk < nch && (kck < kNK || tc::mbar_try_wait(&sh->k_empty[kck % kNK], (uint32_t)(((kck / kNK) - 1) & 1)))) {
               const int st = (int)(kck % kNK);
               uint8_t* dst = sK + st * C::kKc;
               tc::mbar_arrive_expect_tx(&sh->k_full[st], C::kKc);
-#pragma unroll
-              for (int i = 0; i < kCH; ++i) {
-                const int z = chunk_z(nk * kCH + i);
-#pragma unroll
-                for (int h = 0; h < C::kHalves; ++h)
-                  tc::tma_load_3d(dst + h * C::kHalfRows + i * (kUnit * 128), &map_k, &sh->k_full[st], h * 64, g, z);
-              }
-#pragma unroll
-              for (int i = 0; i < kCH; ++i) {
-                const int e = (nk + kPF) * kCH + i;
-                if (e < nu) {
-#pragma unroll
-                  for (int h = 0; h < C::kHalves; ++h) {
-                    tc::tma_prefetch_3d(&map_k, h * 64, g, b * a.T_kv + usb[e] * kUnit);
-                    if (main_pass) tc::tma_prefetch_3d(&map_v, h * 64, g, b * a.T_kv + usb[e] * kUnit);
-                  }
-                }
-              }
+              load_chunk(dst, maps.k, &sh->k_full[st], nk);
               ++nk;
               ++kck;
               prog = true;
@@ -408,13 +416,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
               const int st = (int)(kcv % kNV);
               uint8_t* dst = sV + st * C::kKc;
               tc::mbar_arrive_expect_tx(&sh->v_full[st], C::kKc);
-#pragma unroll
-              for (int i = 0; i < kCH; ++i) {
-                const int z = chunk_z(nv * kCH + i);
-#pragma unroll
-                for (int h = 0; h < C::kHalves; ++h)
-                  tc::tma_load_3d(dst + h * C::kHalfRows + i * (kUnit * 128), &map_v, &sh->v_full[st], h * 64, g, z);
-              }
+              load_chunk(dst, maps.v, &sh->v_full[st], nv);
               ++nv;
               ++kcv;
               prog = true;
@@ -682,14 +684,14 @@ EncodeTiled get_encode() {
   return fn;
 }
 
-// 3-D map over k or v [batch * T_kv tokens][G][d] bf16: box = 64 dims x 1 group x 16 tokens,
-// 128B swizzle (one 128-byte row per token).
-bool make_kv_map(CUtensorMap* map, const void* base, long tokens, int G, int d) {
+// 3-D map over k or v [batch * T_kv tokens][G][d] bf16: box = 64 dims x 1 group x box_tokens
+// tokens, 128B swizzle (one 128-byte row per token).
+bool make_kv_map(CUtensorMap* map, const void* base, long tokens, int G, int d, int box_tokens) {
   EncodeTiled enc = get_encode();
   if (!enc) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)G, (cuuint64_t)tokens};
   const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)G * d * 2};
-  const cuuint32_t box[3] = {64, 1, (cuuint32_t)kUnit};
+  const cuuint32_t box[3] = {64, 1, (cuuint32_t)box_tokens};
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -705,12 +707,17 @@ cudaError_t launch_dr(const AttendArgs& a, const uint32_t* perm, cudaStream_t s)
   const int n_seg = a.batch * a.G;
   int lb = 0;
   while ((1 << lb) < a.B) ++lb;
-  CUtensorMap mk, mv;
-  if (!make_kv_map(&mk, a.k, (long)a.batch * a.T_kv, a.G, D) || !make_kv_map(&mv, a.v, (long)a.batch * a.T_kv, a.G, D))
-    return cudaErrorInvalidValue;
+  KvMaps maps;
+  const long tokens = (long)a.batch * a.T_kv;
+  maps.max_run = tokens >= 4 * kUnit ? 2 : (tokens >= 2 * kUnit ? 1 : 0);
+  for (int i = 0; i < 3; ++i) {
+    const int box = kUnit << (i <= maps.max_run ? i : 0);
+    if (!make_kv_map(&maps.k[i], a.k, tokens, a.G, D, box) || !make_kv_map(&maps.v[i], a.v, tokens, a.G, D, box))
+      return cudaErrorInvalidValue;
+  }
   cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
-  attend_tc_kernel<D, R><<<(unsigned)((long)tiles * n_seg), kThreads, C::kSmem, s>>>(mk, mv, a, perm, n, tiles, lb);
+  attend_tc_kernel<D, R><<<(unsigned)((long)tiles * n_seg), kThreads, C::kSmem, s>>>(maps, a, perm, n, tiles, lb);
   return cudaGetLastError();
 }
 
