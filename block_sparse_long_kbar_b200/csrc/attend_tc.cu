@@ -29,8 +29,9 @@
 //     repeats the main pass (flagged rows with their exact maximum, the others with exactly the
 //     same arithmetic as before).
 //   * O[128 x d] += P V with tcgen05.mma, P read from TMEM (A operand) and V from shared memory
-//     (an MN-major operand), one K=16 step per superblock. The row sums l add the same bf16 P on
-//     the CUDA cores: each thread sums its superblocks (one id parity) in ascending id order and
+//     (an MN-major operand), one K=16 step per superblock. The row sums l add the fp32 values of
+//     P (before their rounding to bf16, which changes l by at most 2^-9 relative) on the CUDA
+//     cores: each thread sums its superblocks (one id parity) in ascending id order and
 //     l = l_even + l_odd. Because superblocks are aligned on block ids, each is one K=16
 //     accumulation step and one parity class, and unselected slots contribute exact zeros, every
 //     row's arithmetic is the same whatever rows share its tile (bitwise causal, chunk-invariant).
@@ -496,8 +497,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         }
       } else {
         // ---- softmax: one row per thread pair; the thread with shalf = (superblock id & 1) takes
-        // a superblock: its 16 S columns become 8 columns of bf16 P in place (TMEM) and the same
-        // bf16 values are added to the thread's row sum, in token order ----
+        // a superblock: its 16 S columns become 8 columns of bf16 P in place (TMEM) and the fp32
+        // values are added to the thread's row sum, in token order ----
         for (int ch = 0; ch < nch; ++ch, ++scnt) {
           const int sb = (int)(scnt & 1);
           if (!warp_wait(&sh->s_full[sb], (uint32_t)((scnt >> 1) & 1), &sh->abort_flag, a.status)) {
@@ -529,9 +530,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 #pragma unroll
               for (int k2 = 0; k2 < 8; ++k2) {
                 const float bias = k2 < 4 ? bias0 : bias1;
-                const float ta = fmaf(__uint_as_float(v[2 * k2]), sc, bias);
-                const float tb = fmaf(__uint_as_float(v[2 * k2 + 1]), sc, bias);
-                pk[k2] = pack_bf16x2(ex2_approx(ta), ex2_approx(tb));
+                const float pa = ex2_approx(fmaf(__uint_as_float(v[2 * k2]), sc, bias));
+                const float pb = ex2_approx(fmaf(__uint_as_float(v[2 * k2 + 1]), sc, bias));
+                pk[k2] = pack_bf16x2(pa, pb);
+                l_sum += pa;
+                l_sum += pb;
               }
             } else {
               uint32_t vmask = 0;  // bit k: token sbid * 16 + k is valid for this row
@@ -555,17 +558,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 #pragma unroll
               for (int k2 = 0; k2 < 8; ++k2) {
                 const bool va = (vmask >> (2 * k2)) & 1u, vb = (vmask >> (2 * k2 + 1)) & 1u;
-                const float ta = va ? fmaf(__uint_as_float(v[2 * k2]), sc, -base) : -INFINITY;
-                const float tb = vb ? fmaf(__uint_as_float(v[2 * k2 + 1]), sc, -base) : -INFINITY;
-                pk[k2] = pack_bf16x2(ex2_approx(ta), ex2_approx(tb));
+                const float pa = ex2_approx(va ? fmaf(__uint_as_float(v[2 * k2]), sc, -base) : -INFINITY);
+                const float pb = ex2_approx(vb ? fmaf(__uint_as_float(v[2 * k2 + 1]), sc, -base) : -INFINITY);
+                pk[k2] = pack_bf16x2(pa, pb);
+                l_sum += pa;
+                l_sum += pb;
               }
             }
             tc::tmem_st8(col, pk);
-#pragma unroll
-            for (int k2 = 0; k2 < 8; ++k2) {
-              l_sum += bf16_lo(pk[k2]);
-              l_sum += bf16_hi(pk[k2]);
-            }
           }
           // P of this chunk is in TMEM (or, in the exact-maximum pass, S has been read): the MMA
           // issuer may take the buffer
