@@ -17,7 +17,8 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-SO_PATH = os.path.join(_HERE, "libsgqa.so")
+# SGQA_LIBRARY=checks selects the debug build with device-side bounds checks (libsgqa_checks.so)
+SO_PATH = os.path.join(_HERE, "libsgqa_checks.so" if os.environ.get("SGQA_LIBRARY") == "checks" else "libsgqa.so")
 
 SGQA_OK = 0
 STATUS_NAMES = {0: "SGQA_OK", 1: "SGQA_ERR_INVALID_ARG", 2: "SGQA_ERR_UNSUPPORTED", 3: "SGQA_ERR_WORKSPACE",
@@ -55,7 +56,7 @@ def load_library():
     if _lib is not None:
         return _lib
     if not os.path.exists(SO_PATH):
-        raise RuntimeError(f"libsgqa.so is not built at {SO_PATH}: run __graft_entry__.build()")
+        raise RuntimeError(f"{os.path.basename(SO_PATH)} is not built at {SO_PATH}: run __graft_entry__.build()")
     L = ctypes.CDLL(SO_PATH)
     P, S, I = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
     D = ctypes.POINTER(sgqa_dims)

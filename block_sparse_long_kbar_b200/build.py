@@ -1,4 +1,9 @@
-"""Build libsgqa.so in-tree for sm_100a with nvcc (object files compiled in parallel)."""
+"""Build libsgqa.so in-tree for sm_100a with nvcc (object files compiled in parallel).
+
+variant="checks" builds libsgqa_checks.so, the same sources with -DSGQA_CHECKS: the kernels test
+the indices they compute from data against their buffers and record SGQA_ERR_DEVICE_CHECK
+instead of making an out-of-range access (the debug build the tests run alongside the normal
+one)."""
 from __future__ import annotations
 
 import concurrent.futures
@@ -12,6 +17,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 SO = os.path.join(HERE, "libsgqa.so")
+SO_CHECKS = os.path.join(HERE, "libsgqa_checks.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", os.path.join(ROOT, "include"),
          "--expt-relaxed-constexpr"]
@@ -26,21 +32,31 @@ def _deps():
         os.path.join(ROOT, "include", "sgqa.h")]
 
 
-def needs_build() -> bool:
-    if not os.path.exists(SO):
+def _variant(variant: str):
+    if variant == "checks":
+        return os.path.join(HERE, "_build_checks"), SO_CHECKS, ["-DSGQA_CHECKS"]
+    if variant:
+        raise ValueError(f"unknown library variant {variant!r}")
+    return BUILD, SO, []
+
+
+def needs_build(variant: str = "") -> bool:
+    so = _variant(variant)[1]
+    if not os.path.exists(so):
         return True
-    t = os.path.getmtime(SO)
+    t = os.path.getmtime(so)
     return any(os.path.getmtime(p) > t for p in _deps())
 
 
-def build(force: bool = False, verbose: bool = False, extra=None) -> str:
-    if not force and not needs_build():
-        return SO
-    os.makedirs(BUILD, exist_ok=True)
-    extra = list(extra or [])
+def build(force: bool = False, verbose: bool = False, extra=None, variant: str = "") -> str:
+    build_dir, so, vflags = _variant(variant)
+    if not force and not needs_build(variant):
+        return so
+    os.makedirs(build_dir, exist_ok=True)
+    extra = vflags + list(extra or [])
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src) + ".o")
         cmd = ["nvcc", *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
@@ -51,16 +67,16 @@ def build(force: bool = False, verbose: bool = False, extra=None) -> str:
 
     with concurrent.futures.ThreadPoolExecutor(max_workers=8) as ex:
         objs = list(ex.map(compile_one, sources()))
-    tmp = SO + ".tmp"
+    tmp = so + ".tmp"
     cmd = ["nvcc", *ARCH, "-shared", "-o", tmp, *objs, "-lcudart"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stderr}")
-    os.replace(tmp, SO)
-    return SO
+    os.replace(tmp, so)
+    return so
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="-v" in sys.argv,
-          extra=["-Xptxas", "-v"] if "--ptxas" in sys.argv else None)
-    print(SO)
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv,
+                extra=["-Xptxas", "-v"] if "--ptxas" in sys.argv else None,
+                variant="checks" if "--checks" in sys.argv else ""))

@@ -452,7 +452,7 @@ int decode_impl(const sgqa_dims* dims, int cache_len, int n_new, const KvCaches&
   }
   // 4. gated attention over the selection
   if (w.tc) {
-    if (launch_decode_union(sel, dims->batch, n_new, G, Kb, w.ublk, w.umask, w.ucount, n_new * Kb, s) != cudaSuccess)
+    if (launch_decode_union(sel, dims->batch, n_new, G, Kb, w.ublk, w.umask, w.ucount, n_new * Kb, w.status, s) != cudaSuccess)
       return SGQA_ERR_CUDA;
     DecodeAttendArgs da{};
     da.q = q_new; da.gate = gate_new; da.out = out; da.k = kv.k; da.v = kv.v;

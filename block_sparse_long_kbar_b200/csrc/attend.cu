@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(kWarps * 32) attend_kernel(AttendArgs a) {
     const int j = s_sel[e];
     if (j < 0) return -1;
     const int u = j * B + s % B;
-    return u <= t ? u : -1;
+    return (u <= t && SGQA_CHECK(u < a.T_kv, a.status)) ? u : -1;
   };
   auto issue = [&](int ci, int stage) {
     uint8_t* kd = wbase + stage * L::kStage;

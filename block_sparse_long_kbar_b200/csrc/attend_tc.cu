@@ -213,7 +213,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   __syncthreads();
   if (tid < QT) {
     const int idx = tile * QT + tid;
-    const int t = idx < n_per_seg ? a.t_begin + (int)__ldg(perm + (long)seg * n_per_seg + idx) : -1;
+    int t = idx < n_per_seg ? a.t_begin + (int)__ldg(perm + (long)seg * n_per_seg + idx) : -1;
+    // the permutation maps the tile's slots onto the query range, and q rows exist for it
+    if (t >= 0 && !SGQA_CHECK(t < a.t_end && t - a.q_t0 >= 0 && t - a.q_t0 < a.nQ, a.status)) t = -1;
     sh->t[tid] = t;
     if (t >= 0) atomicMax(&sh->maxc, t / B);
   }
@@ -366,7 +368,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         for (int sb = sb0; sb < sb1; ++sb) {
           uint32_t any = 0;
           for (int i = 0; i < spb; ++i) any |= wmask[sb * spb + i];
-          if (any) usb[pos++] = (w0 >> (4 - lb)) + sb;
+          if (any) {
+            // a superblock holding a selected block starts inside the sequence (recorded only:
+            // the TMA fetch of any coordinate is safe, out-of-range tokens read zeros)
+            (void)SGQA_CHECK(((w0 >> (4 - lb)) + sb) * kUnit < a.T_kv, a.status);
+            usb[pos++] = (w0 >> (4 - lb)) + sb;
+          }
         }
       }
       __syncthreads();

@@ -269,7 +269,10 @@ __global__ void __launch_bounds__(512) rev_fill_kernel(BackwardArgs a) {
     const int32_t* srow = a.sel + ((b * a.T + t) * a.G + g) * (long)a.Kb;
     for (int i = threadIdx.x; i < a.Kb; i += blockDim.x) {
       const int j = __ldg(srow + i);
-      if (j >= 0 && j <= t / a.B) list[off[j] + cur[j]++] = t;
+      if (j >= 0 && j <= t / a.B) {
+        const int at = off[j] + cur[j]++;
+        if (SGQA_CHECK(at < off[j + 1], a.status)) list[at] = t;  // inside the block's slice
+      }
     }
     __syncthreads();
   }
@@ -303,7 +306,8 @@ __global__ void __launch_bounds__(128) backward_kv_kernel(BackwardArgs a) {
   const int* list = a.rlist + seg * (long)a.T * a.Kb;
   const int r0 = off[j], r1 = off[j + 1];
   for (int ri = r0; ri < r1; ++ri) {
-    const int t = __ldg(list + ri);
+    int t = __ldg(list + ri);
+    if (!SGQA_CHECK(t >= 0 && t < a.T, a.status)) t = 0;  // a query position of the sequence
     const bool vis = live && u <= t;
     const long bt = b * a.T + t;
     for (int hr = 0; hr < R; ++hr) {

@@ -16,6 +16,21 @@ __device__ __forceinline__ void report(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// Debug bounds checks. The library built with -DSGQA_CHECKS (libsgqa_checks.so) tests the
+// indices and coordinates its kernels compute from data (selections, union lists, permutations,
+// cache positions) against their buffers before use: a failed check records
+// SGQA_ERR_DEVICE_CHECK and the access is skipped, so a logic error shows as a status instead of
+// a fault. Without the flag every check compiles to `true`.
+__device__ __forceinline__ bool check_or_report(bool ok, int* status) {
+  if (!ok) report(status, SGQA_ERR_DEVICE_CHECK);
+  return ok;
+}
+#ifdef SGQA_CHECKS
+#define SGQA_CHECK(cond, status) (::sgqa::check_or_report((cond), (status)))
+#else
+#define SGQA_CHECK(cond, status) (true)
+#endif
+
 __device__ __forceinline__ float bf16_lo(uint32_t packed) { return __uint_as_float(packed << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t packed) { return __uint_as_float(packed & 0xFFFF0000u); }
 __device__ __forceinline__ float bf16_to_f32(uint16_t u) { return __uint_as_float((uint32_t)u << 16); }

@@ -423,7 +423,14 @@ __global__ void __launch_bounds__(DaCfg<F8>::kThr, 1)
         // (row of the cache, K scale, V scale) of a tile's token slot r
         auto meta = [&](int i, long& srow, float& ks, float& vs) {
           const int idx = i * NB + e;
-          srow = (i < tile1 && idx < count) ? ((long)b * a.T_kv + __ldg(ublk + idx) * B + (r % B)) * a.G + g : -1;
+          srow = -1;
+          if (i < tile1 && idx < count) {
+            // tokens of a partial last block past the cache capacity do not exist (their slots
+            // are masked): no scale is read for them
+            const int blk = __ldg(ublk + idx);
+            const int u = blk * B + (r % B);
+            if (SGQA_CHECK(blk >= 0 && blk * B < a.T_kv, a.status) && u < a.T_kv) srow = ((long)b * a.T_kv + u) * a.G + g;
+          }
           ks = srow >= 0 ? __ldg(a.k_scale + srow) : 0.f;
           vs = (srow >= 0 && main_pass) ? __ldg(a.v_scale + srow) : 0.f;
         };
@@ -639,7 +646,7 @@ __global__ void __launch_bounds__(DaCfg<F8>::kThr, 1)
 // elements below it that their lowest lists own (binary searches; no sort).
 __global__ void __launch_bounds__(256) decode_union_kernel(const int32_t* __restrict__ sel, int n_new, int G, int Kb,
                                                            int32_t* __restrict__ ublk, uint32_t* __restrict__ umask,
-                                                           int* __restrict__ ucount, int ucap) {
+                                                           int* __restrict__ ucount, int ucap, int* status) {
   extern __shared__ int su[];
   int* lists = su;                 // [n_new][Kb]
   int* incl = su + n_new * Kb;     // [n_new][Kb]: owners among the first i + 1 entries
@@ -714,6 +721,7 @@ __global__ void __launch_bounds__(256) decode_union_kernel(const int32_t* __rest
       }
       rank += lo > 0 ? incl[q2 * Kb + lo - 1] : 0;
     }
+    if (!SGQA_CHECK(rank < ucap, status)) continue;
     ublk[(long)unit * ucap + rank] = x;
     umask[(long)unit * ucap + rank] = msk[idx];
   }
@@ -827,11 +835,11 @@ size_t decode_part_bytes(int units, int splits) {
 }
 
 cudaError_t launch_decode_union(const int32_t* sel, int batch, int n_new, int G, int Kb, int32_t* ublk,
-                                uint32_t* umask, int* ucount, int ucap, cudaStream_t s) {
+                                uint32_t* umask, int* ucount, int ucap, int* status, cudaStream_t s) {
   const size_t shmem = (size_t)n_new * Kb * 12;
   cudaError_t e = cudaFuncSetAttribute(decode_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shmem);
   if (e != cudaSuccess) return e;
-  decode_union_kernel<<<(unsigned)(batch * G), 256, shmem, s>>>(sel, n_new, G, Kb, ublk, umask, ucount, ucap);
+  decode_union_kernel<<<(unsigned)(batch * G), 256, shmem, s>>>(sel, n_new, G, Kb, ublk, umask, ucount, ucap, status);
   return cudaGetLastError();
 }
 

@@ -135,7 +135,7 @@ bool decode_attend_tc_supported(int Hq, int G, int d, int B, int n_new, int Kb);
 int decode_attend_splits(int units, int n_new, int Kb, int B);
 size_t decode_part_bytes(int units, int splits);
 cudaError_t launch_decode_union(const int32_t* sel, int batch, int n_new, int G, int Kb, int32_t* ublk,
-                                uint32_t* umask, int* ucount, int ucap, cudaStream_t s);
+                                uint32_t* umask, int* ucount, int ucap, int* status, cudaStream_t s);
 cudaError_t launch_decode_attend_tc(const DecodeAttendArgs& a, cudaStream_t s);
 
 // FP8 KV storage: rows (b, t, g) of src [batch, n_t, G, 128] bf16 -> dst8 [batch, T, G, 128] e4m3

@@ -595,7 +595,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             run += cnt;
           }
         }
-        if (lim > 0) *reinterpret_cast<uint2*>(brow + (j0 >> 5)) = make_uint2(tb[0], tb[1]);
+        if (lim > 0 && SGQA_CHECK((j0 >> 5) + 1 < a.bstride && t < a.t_end, a.status))
+          *reinterpret_cast<uint2*>(brow + (j0 >> 5)) = make_uint2(tb[0], tb[1]);
         taken += __popc(tb[0]) + __popc(tb[1]);
       }
       if (!aborted && half == 1 && act) {
@@ -624,7 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t* py = y < n0 ? my_hist + 2 * y : my_hist + 128 + 2 * (y - n0);
             ahead += (py[0] > kx || (py[0] == kx && py[1] < jx)) ? 1 : 0;
           }
-          if (ahead < rem) {
+          if (ahead < rem && SGQA_CHECK(jx < (uint32_t)c && (int)(jx >> 5) < a.bstride, a.status)) {
             atomicOr(brow + (jx >> 5), 1u << (jx & 31u));
             ++total;
           }
@@ -670,7 +671,7 @@ __global__ void __launch_bounds__(256) sel_from_bits_kernel(SelectArgs a) {
   const int c = t / a.B, m = min(a.Kb - 1, c);
   const uint32_t* bits = a.bits + row * (long)a.bstride;
   int32_t* out = a.sel + (((long)b * a.sel_T + (t - a.sel_t0)) * a.G + g) * (long)a.Kb;
-  const int nw = m > 0 ? (c + 31) >> 5 : 0;
+  const int nw = m > 0 && SGQA_CHECK(((c + 31) >> 5) <= a.bstride, a.status) ? (c + 31) >> 5 : 0;
   int pos = 0;
   for (int w0 = 0; w0 < nw && pos < m; w0 += 32) {
     const int w = w0 + lane;

@@ -43,6 +43,15 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(lib, s)
 
 
+def test_bounds_checking_build_exports_every_declared_symbol():
+    """libsgqa_checks.so (-DSGQA_CHECKS) is the same library with device-side index checks."""
+    so = sg_build.build(variant="checks")
+    out = subprocess.run(["nm", "-D", "--defined-only", so], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\b(sgqa_[a-z_0-9]+)\b", out))
+    for s in declared_symbols():
+        assert s in exported, s
+
+
 def test_header_compiles_as_c(tmp_path):
     src = tmp_path / "t.c"
     src.write_text('#include "sgqa.h"\nint main(void){ sgqa_dims d = {1,8,2,1,64,32,8,8}; '

@@ -77,8 +77,9 @@ def _dequant_bf16_bits(q, s):
     return b
 
 
-def _fp8_decode_case(cfg, cache_len, n_new, check_seqs, compare_bf16=True):
-    T_cap = ((cache_len + n_new + cfg.B - 1) // cfg.B) * cfg.B
+def _fp8_decode_case(cfg, cache_len, n_new, check_seqs, compare_bf16=True, T_cap=None):
+    if T_cap is None:
+        T_cap = ((cache_len + n_new + cfg.B - 1) // cfg.B) * cfg.B
     dims, c8, csc, kidx, kbar = _fp8_caches(cfg, T_cap, cache_len)
     new = {}
     for n in NAMES:
@@ -156,6 +157,13 @@ def _fp8_decode_case(cfg, cache_len, n_new, check_seqs, compare_bf16=True):
 ])
 def test_fp8_decode_matches_oracle(cfg, cache_len, n_new, seqs):
     _fp8_decode_case(cfg, cache_len, n_new, seqs)
+
+
+def test_fp8_decode_capacity_ending_inside_a_block():
+    """The caches hold exactly cache_len + n_new tokens and that count is not a multiple of B:
+    the last block is partial, and its missing tokens (past the capacity) have no scale to read."""
+    cfg = Config("f8_ragged_cap", 2, 5000, 32, 4, 128, 64, 8, 512, 600, 44)
+    _fp8_decode_case(cfg, 4993, 4, [0, 1], T_cap=4997)
 
 
 def test_fp8_decode_rejects_shapes_without_the_tensor_core_path():
