@@ -38,17 +38,18 @@ CLOCK_FIELDS = ["pci.bus_id", "clocks.sm", "clocks.max.sm", "power.draw", "clock
                 "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
 
 
-# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from ncu captures of the
-# kernels, keyed by (stage, workload), each with the SHA-256 (first 16 hex digits) of the kernel's
-# source file at capture time: an entry is reported only while that source is unchanged, else the
-# traffic is null. The figures and the commands that produced them are under profiles/.
+# DRAM bytes per stage call (dram__bytes_read.sum + dram__bytes_write.sum summed over the call's
+# launches of the stage's kernels) from ncu captures, keyed by (stage, workload), each with the
+# SHA-256 (first 16 hex digits) of the kernels' source file at capture time: an entry is reported
+# only while that source is unchanged, else the traffic is null. The figures and the commands
+# that produced them are under profiles/.
 NCU_TRAFFIC: dict = {
-    # profiles/traffic_prefill128k_decode1m.md: one launch each, the bench's own 128K / 1M workloads
-    ("attend", "128k"): (6576556544 + 1069653760, "8545fe13f12f383c"),
-    ("select", "128k"): (76668928 + 1018871040, "1adee091c006784c"),
-    ("decode_scores", "decode_1m"): (1074586880 + 255890688, "99064a99bc73bfeb"),
-    ("decode_select", "decode_1m"): (509419776 + 123904, "6b1e39bfc032a2cd"),
-    ("decode_attend", "decode_1m"): (1073816064 + 169472, "f2a6bae20073fbb6"),
+    # profiles/traffic_prefill128k_decode1m.md, the bench's own 128K / 1M workloads
+    ("attend", "128k"): (6479270656 + 1068269312, "90290afbbced3240"),   # one attend_tc launch
+    ("select", "128k"): (443320832 + 1218017024, "5fefe859bf2faa3c"),    # 4 select_tc + 4 sel_from_bits
+    ("decode_scores", "decode_1m"): (1074968832 + 252713216, "0669c7900a2898e8"),
+    ("decode_select", "decode_1m"): (509710080 + 136960, "6b1e39bfc032a2cd"),
+    ("decode_attend", "decode_1m"): (1073845760 + 239104, "0b27aa0c5434674b"),
 }
 STAGE_SOURCES = {"compress": "compress.cu", "select": "select_tc.cu", "attend": "attend_tc.cu",
                  "decode_scores": "decode_scores_tc.cu", "decode_select": "decode.cu",
