@@ -657,8 +657,10 @@ __global__ void own_block_only_kernel(SelectArgs a) {
 }
 
 // The selection from the bitmaps: per (token, group) row, the set bits of words [0, ceil(c/32))
-// in ascending order (m of them), then the own block c, then -1 up to Kb. One warp per row: each
-// lane takes one word of every 32, a warp scan of the population counts places its indices.
+// in ascending order (m of them), then the own block c, then -1 up to Kb. One warp per row: the
+// lanes load 32 words at a time and a warp scan of their population counts gives each word's
+// output position; then the warp expands the non-zero words one at a time, lane b writing the
+// index of bit b when it is set (one coalesced store per word, no per-lane loops over bits).
 __global__ void __launch_bounds__(256) sel_from_bits_kernel(SelectArgs a) {
   const long row = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -672,10 +674,11 @@ __global__ void __launch_bounds__(256) sel_from_bits_kernel(SelectArgs a) {
   const uint32_t* bits = a.bits + row * (long)a.bstride;
   int32_t* out = a.sel + (((long)b * a.sel_T + (t - a.sel_t0)) * a.G + g) * (long)a.Kb;
   const int nw = m > 0 && SGQA_CHECK(((c + 31) >> 5) <= a.bstride, a.status) ? (c + 31) >> 5 : 0;
+  const uint32_t below = (1u << lane) - 1u;
   int pos = 0;
   for (int w0 = 0; w0 < nw && pos < m; w0 += 32) {
     const int w = w0 + lane;
-    uint32_t x = w < nw ? __ldg(bits + w) : 0u;
+    const uint32_t x = w < nw ? __ldg(bits + w) : 0u;
     const int n = __popc(x);
     int inc = n;
 #pragma unroll
@@ -683,12 +686,14 @@ __global__ void __launch_bounds__(256) sel_from_bits_kernel(SelectArgs a) {
       const int y = __shfl_up_sync(0xFFFFFFFFu, inc, o);
       if (lane >= o) inc += y;
     }
-    int p = pos + inc - n;
-    while (x) {
-      const int q = __ffs(x) - 1;
-      x &= x - 1u;
-      if (p < m) out[p] = 32 * w + q;
-      ++p;
+    const int start = pos + inc - n;  // output position of this lane's word
+    unsigned nz = __ballot_sync(0xFFFFFFFFu, x != 0u);
+    while (nz) {
+      const int L = __ffs(nz) - 1;
+      nz &= nz - 1u;
+      const uint32_t xw = __shfl_sync(0xFFFFFFFFu, x, L);
+      const int p = __shfl_sync(0xFFFFFFFFu, start, L) + __popc(xw & below);
+      if (((xw >> lane) & 1u) && p < m) out[p] = 32 * (w0 + L) + lane;
     }
     pos += __shfl_sync(0xFFFFFFFFu, inc, 31);
   }
