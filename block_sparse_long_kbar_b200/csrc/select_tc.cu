@@ -46,7 +46,7 @@ namespace {
 constexpr int kRows = 128;
 constexpr int kN = 128;          // candidate blocks per MMA tile
 constexpr int kStages = 2;
-constexpr int kHistStride = 257;
+constexpr int kHistStride = 257;  // words per row (256 bins + spare slot); stored bin-major, below
 constexpr int kEpiWarps = 8;     // two per TMEM lane quadrant: each histograms half the columns
 constexpr int kThreads = (kEpiWarps + 2) * 32;
 constexpr int kProducerWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
@@ -141,9 +141,9 @@ __device__ __forceinline__ void hist_chunk(const uint32_t (&v)[64], int lim, uin
 #pragma unroll
   for (int q = 0; q < 64; ++q) {
     const uint32_t key = score_key(__uint_as_float(v[q]));
-    const uint32_t addr = hbase + (((key >> shift) & 255u) << 2);
+    const uint32_t addr = hbase + (((key >> shift) & 255u) * (kRows * 4u));
     if (kFull && kFirst) red_shared_inc(addr);
-    else red_shared_inc(((kFull || q < lim) && (kFirst || (key & mask) == prefix)) ? addr : hbase + kTrash * 4u);
+    else red_shared_inc(((kFull || q < lim) && (kFirst || (key & mask) == prefix)) ? addr : hbase + kTrash * (kRows * 4u));
   }
 }
 
@@ -406,7 +406,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     int rem = m, nb = c;
     bool done = (rem == nb);
     if (rem == 0) { prefix = 0xFFFFFFFFu; mask = 0xFFFFFFFFu; done = true; }
-    uint32_t* my_hist = hist + r * kHistStride;
+    // the row's words are stored bin-major: word w of row r at hist[w * kRows + r], so the lanes of
+    // a warp (32 consecutive rows) always address 32 different banks, whatever bins their keys
+    // fall in (row-major rows collided whenever neighbouring rows' keys fell in nearby bins)
+    uint32_t* my_hist = hist + r;
     // the row's bitmap of taken candidates (bit j of word j / 32)
     uint32_t* brow = a.bits + (((long)b * (a.t_end - a.t_begin) + (t - a.t_begin)) * G + g) * (long)a.bstride;
     const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
@@ -418,9 +421,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // zero the histograms for this pass (a resolved row: its tie-count slots), then a
       // barrier+vote: is any row still unresolved?
       if (half == 0 && !done && pass < kMaxPasses - 1)
-        for (int i = 0; i < 256; ++i) my_hist[i] = 0;
+        for (int i = 0; i < 256; ++i) my_hist[i * kRows] = 0;
       if (half == 0 && done)
-        for (int i = 0; i < 4; ++i) my_hist[i] = 0;
+        for (int i = 0; i < 4; ++i) my_hist[i * kRows] = 0;
       const int vote = epi_vote_any(sh, 4 * pass, !done, a.status);
       // from the third pass on, if every unresolved row's threshold bucket is small, this pass is
       // the last: it also collects those buckets' keys, which are then resolved exactly
@@ -476,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!done) {
           int above = 0;
           for (int bin = 255; bin >= 0; --bin) {
-            const int h = (int)my_hist[bin];
+            const int h = (int)my_hist[bin * kRows];
             if (above + h >= rem) {
               prefix |= (uint32_t)bin << shift;
               mask |= 255u << shift;
@@ -522,8 +525,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // identical in the two warps of a row pair (same rows, same state)
       const bool any_bucket = __any_sync(0xFFFFFFFFu, collect || ties);
       const bool any_ties = __any_sync(0xFFFFFFFFu, ties);
-      uint32_t* cand = my_hist + 128 * half;  // collected (key, j) pairs of this half
-      volatile uint32_t* slot = my_hist;      // tie counts: [half][tile parity]
+      uint32_t* cand = my_hist + 128 * half * kRows;  // collected (key, j) pairs of this half (stride kRows)
+      volatile uint32_t* slot = my_hist;              // tie counts: [half][tile parity] (stride kRows)
       int run = 0;                            // exact ties before this half's columns of the tile
       for (int i = 0; i < n_nt; ++i, ++k) {
         const int buf = (int)(k & 1);
@@ -556,8 +559,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int q = __ffs(bits) - 1;
                 bits &= bits - 1u;
                 if (eqn < kCap) {
-                  cand[2 * eqn] = score_key(__uint_as_float(pick64(v, 32 * w + q)));
-                  cand[2 * eqn + 1] = (uint32_t)(j0 + 32 * w + q);
+                  cand[(2 * eqn) * kRows] = score_key(__uint_as_float(pick64(v, 32 * w + q)));
+                  cand[(2 * eqn + 1) * kRows] = (uint32_t)(j0 + 32 * w + q);
                 }
                 ++eqn;
               }
@@ -572,15 +575,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int cnt = ties ? __popc(bb[0]) + __popc(bb[1]) : 0;
           int got = 0;
           if (half == 0) {
-            if (ties) slot[i & 1] = ((uint32_t)(i + 1) << 8) | (uint32_t)cnt;
+            if (ties) slot[(i & 1) * kRows] = ((uint32_t)(i + 1) << 8) | (uint32_t)cnt;
             if (ties && i > 0) {
-              got = wait_tie_count(slot + 2 + ((i - 1) & 1), (uint32_t)i, sh, a.status);
+              got = wait_tie_count(slot + (2 + ((i - 1) & 1)) * kRows, (uint32_t)i, sh, a.status);
               run += got;
             }
           } else if (ties) {
-            got = wait_tie_count(slot + (i & 1), (uint32_t)(i + 1), sh, a.status);
+            got = wait_tie_count(slot + (i & 1) * kRows, (uint32_t)(i + 1), sh, a.status);
             run += got;
-            slot[2 + (i & 1)] = ((uint32_t)(i + 1) << 8) | (uint32_t)cnt;
+            slot[(2 + (i & 1)) * kRows] = ((uint32_t)(i + 1) << 8) | (uint32_t)cnt;
           }
           if (__any_sync(0xFFFFFFFFu, got < 0)) {
             if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
@@ -600,8 +603,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         taken += __popc(tb[0]) + __popc(tb[1]);
       }
       if (!aborted && half == 1 && act) {
-        my_hist[kCnt1] = (uint32_t)eqn;
-        my_hist[kCnt1 + 1] = (uint32_t)taken;
+        my_hist[kCnt1 * kRows] = (uint32_t)eqn;
+        my_hist[(kCnt1 + 1) * kRows] = (uint32_t)taken;
       }
       emitted = !aborted;
       break;
@@ -610,20 +613,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     // collected keys of both halves are complete
     asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
     if (emitted && half == 0 && act_row(valid, m) && !sh->abort_flag) {
-      int total = taken + (int)my_hist[kCnt1 + 1];
+      int total = taken + (int)my_hist[(kCnt1 + 1) * kRows];
       if (collect) {
         // the collected bucket keys of both halves: key x ranks behind every larger key and every
         // equal key of lower j, and is taken when fewer than rem rank ahead of it
-        const int e1 = (int)my_hist[kCnt1];
+        const int e1 = (int)my_hist[kCnt1 * kRows];
         if (eqn > kCap || e1 > kCap) report(a.status, SGQA_ERR_DEVICE_CHECK);
         const int n0 = min(eqn, kCap), n1 = min(e1, kCap);
         for (int x = 0; x < n0 + n1; ++x) {
-          const uint32_t* px = x < n0 ? my_hist + 2 * x : my_hist + 128 + 2 * (x - n0);
-          const uint32_t kx = px[0], jx = px[1];
+          const uint32_t* px = my_hist + (x < n0 ? 2 * x : 128 + 2 * (x - n0)) * kRows;
+          const uint32_t kx = px[0], jx = px[kRows];
           int ahead = 0;
           for (int y = 0; y < n0 + n1; ++y) {
-            const uint32_t* py = y < n0 ? my_hist + 2 * y : my_hist + 128 + 2 * (y - n0);
-            ahead += (py[0] > kx || (py[0] == kx && py[1] < jx)) ? 1 : 0;
+            const uint32_t* py = my_hist + (y < n0 ? 2 * y : 128 + 2 * (y - n0)) * kRows;
+            ahead += (py[0] > kx || (py[0] == kx && py[kRows] < jx)) ? 1 : 0;
           }
           if (ahead < rem && SGQA_CHECK(jx < (uint32_t)c && (int)(jx >> 5) < a.bstride, a.status)) {
             atomicOr(brow + (jx >> 5), 1u << (jx & 31u));
