@@ -45,8 +45,8 @@ CLOCK_FIELDS = ["pci.bus_id", "clocks.sm", "clocks.max.sm", "power.draw", "clock
 # that produced them are under profiles/.
 NCU_TRAFFIC: dict = {
     # profiles/traffic_prefill128k_decode1m.md, the bench's own 128K / 1M workloads
-    ("attend", "128k"): (6479270656 + 1068269312, "90290afbbced3240"),   # one attend_tc launch
-    ("select", "128k"): (443320832 + 1218017024, "5fefe859bf2faa3c"),    # 4 select_tc + 4 sel_from_bits
+    ("attend", "128k"): (6524326400 + 1068357120, "90290afbbced3240"),   # one attend_tc launch
+    ("select", "128k"): (89709568 + 343720192 + 311718656 + 823901952, "dee08ffbc95d9e6e"),  # 4 select_tc + 4 sel_from_bits
     ("decode_scores", "decode_1m"): (1074968832 + 252713216, "0669c7900a2898e8"),
     ("decode_select", "decode_1m"): (509710080 + 136960, "6b1e39bfc032a2cd"),
     ("decode_attend", "decode_1m"): (1073845760 + 239104, "0b27aa0c5434674b"),

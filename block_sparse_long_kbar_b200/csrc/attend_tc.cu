@@ -243,8 +243,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       if (t < 0) continue;
       const int32_t* row = a.sel + (((long)b * a.sel_T + (t - a.sel_t0)) * G + g) * (long)a.Kb;
       for_each_selected(row, a.Kb, t / B, 0x7FFFFFFF, true, a.status, [&](int j) {
+        // most entries fall in a window already marked: read first (lanes reading one word are
+        // served at once), so that only the first entries of a window pay for an atomic
         const int w = j / kWin;
-        atomicOr(&sh->wbits[w >> 5], 1u << (w & 31));
+        const uint32_t bit = 1u << (w & 31);
+        if (!(*reinterpret_cast<volatile uint32_t*>(&sh->wbits[w >> 5]) & bit)) atomicOr(&sh->wbits[w >> 5], bit);
       });
     }
   }
