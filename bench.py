@@ -358,7 +358,7 @@ def run_ours(args, world, rank):
     dev_all = dict(dev, out=out)
 
     def e2e_step():
-        sg.sgqa_forward_from_host(dims, host, dev_all, out_h, ws, chunks=8, streams=streams)
+        sg.sgqa_forward_from_host(dims, host, dev_all, out_h, ws, chunks=32, streams=streams)
 
     e2e_step()
     torch.cuda.synchronize()

@@ -208,7 +208,7 @@ def sgqa_attend_backward(dims, q, k, v, gate, sel, dout, dq, dk, dv, dgate, ws, 
 INPUTS = ("q", "k", "v", "q_idx", "k_idx", "gate")
 
 
-def sgqa_forward_from_host(dims, host, dev, out_host, ws, chunks=8, streams=None):
+def sgqa_forward_from_host(dims, host, dev, out_host, ws, chunks=32, streams=None):
     """The whole layer (sgqa_forward's result) from pinned host buffers, with the host<->device
     copies overlapped with the computation.
 
