@@ -119,6 +119,23 @@ SELECT_INSTR_PER_KEY = {"hist": 8 + 2, "emit": 8 + 2}
 SELECT_PASSES = {"hist": 2, "emit": 1}
 
 
+def select_ranges(cfg, nq: int) -> int:
+    """Query ranges K2 runs in for nq query rows: bitmap rows of 4 words per 128 blocks, ranges of
+    whole 128-query multiples within a 256 MiB bitmap budget (api.cu, select_bits_dims)."""
+    nblk = cfg.T // cfg.B
+    per_q = cfg.batch * cfg.G * 4 * ((nblk + 127) // 128) * 4
+    q = max(128, (256 << 20) // per_q // 128 * 128) if per_q else nq
+    q = min(q, cfg.T)
+    return (nq + q - 1) // q
+
+
+def forward_launches(cfg, nq: int) -> int:
+    """Library kernel launches of one sgqa_forward(_rows) call over nq query rows: the block means,
+    K2 and its list expansion per query range, the row plan (signature + 3 radix passes of 3
+    kernels) and the attention."""
+    return 1 + 2 * select_ranges(cfg, nq) + 10 + 1
+
+
 def select_alu_model(wc, sm_mhz):
     """Time the select's per-key epilogue work needs at full issue rate (148 SMs x 4 schedulers x
     32 lanes x clock): a kernel-specific ceiling, reported beside the tensor roofline."""
@@ -381,7 +398,7 @@ def run_ours(args, world, rank):
                    "global_batch": world * cfg.batch, "seq_len": cfg.T, "parallelism": f"dp{world} (one sequence per GPU)",
                    "l2": "inputs larger than L2 (q+gate+out 3.2 GB per step), no flush"},
         # per step: compress, select, the plan (signature + 3 radix passes of 3 kernels), attend
-        "gpu_launches": 13 * args.steps,
+        "gpu_launches": forward_launches(cfg, cfg.T) * args.steps,
         "e2e": {"value": tokens_step / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "roofline": roof,
@@ -511,7 +528,7 @@ def run_sharded(args, world, rank):
                    "global_batch": cfg.batch, "seq_len": cfg.T,
                    "parallelism": f"query-sharded x{world} (zig-zag ranges; all-gather of K, V, k_idx over NCCL)",
                    "l2": "inputs larger than L2, no flush"},
-        "gpu_launches": 13 * 2 * args.steps,
+        "gpu_launches": sum(forward_launches(cfg, t1 - t0) for t0, t1 in ranges) * args.steps,
         "e2e": {"value": cfg.batch * cfg.T / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "roofline": {"bound": "tensor", "achieved": per_gpu_flops / (ms / 1e3) / 1e12, "peak": peaks["bf16_tflops"],
