@@ -12,7 +12,9 @@
 // Deterministic, no floating-point atomics:
 //   BQ  (row-centric, one CTA per (b, t, g); a warp per head, four dims per lane): an online-softmax
 //       pass for the row's max and sum (stored as lse) and o, then dgate and D, then a second pass
-//       for dq.
+//       for dq. Tokens are taken NT at a time (a selected block, or half of a 16-token one): their
+//       dot products and warp reductions are independent of one another, and the running maximum
+//       is updated once per group.
 //   reverse index (per (b, g)): for every block j, the rows that selected it, in increasing t
 //       (per-chunk counts, scans over the chunks and the blocks, then every chunk of rows fills
 //       its entries walking its rows in order).
@@ -38,8 +40,9 @@ __device__ __forceinline__ float warp_sum(float x) {
 
 __device__ __forceinline__ float sigmoidf_acc(float x) { return 1.f / (1.f + expf(-x)); }
 
-// BQ: R heads of one (b, t, g) unit; warp w takes heads w, w + 4, ... (up to 4 per warp).
-template <int D>
+// BQ: R heads of one (b, t, g) unit; warp w takes heads w, w + 4, ... (up to 4 per warp); NT
+// tokens of a selected block per step.
+template <int D, int NT>
 __global__ void __launch_bounds__(128) backward_q_kernel(BackwardArgs a) {
   constexpr int DPL = D / 32;  // dims per lane
   constexpr int HPW = 4;       // at most 4 heads per warp (R <= 16)
@@ -78,26 +81,48 @@ __global__ void __launch_bounds__(128) backward_q_kernel(BackwardArgs a) {
       if (lane == 0 && warp == 0) report(a.status, SGQA_ERR_DEVICE_CHECK);
       continue;
     }
-    const int u1 = min(j * a.B + a.B - 1, t);
-    for (int u = j * a.B; u <= u1; ++u) {
-      float kv[DPL], vv[DPL];
+    const int u_hi = min(j * a.B + a.B - 1, t);
+    for (int u0 = j * a.B; u0 <= u_hi; u0 += NT) {
+      float kv[NT][DPL], vv[NT][DPL];
 #pragma unroll
-      for (int e = 0; e < DPL; ++e) {
-        kv[e] = bf16_to_f32(__ldg(kseq + u * kv_stride + lane * DPL + e));
-        vv[e] = bf16_to_f32(__ldg(vseq + u * kv_stride + lane * DPL + e));
+      for (int s2 = 0; s2 < NT; ++s2) {
+        const bool ok = u0 + s2 <= u_hi;
+        const int u = ok ? u0 + s2 : u0;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) {
+          kv[s2][e] = bf16_to_f32(__ldg(kseq + u * kv_stride + lane * DPL + e));
+          vv[s2][e] = bf16_to_f32(__ldg(vseq + u * kv_stride + lane * DPL + e));
+        }
       }
 #pragma unroll
       for (int hh = 0; hh < HPW; ++hh) {
         if (hh >= nh) break;
-        float z = 0.f;
+        float z[NT];
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) z = fmaf(q[hh][e], kv[e], z);
-        z = warp_sum(z) * sc;
-        const float mn = fmaxf(m[hh], z);
-        const float corr = expf(m[hh] - mn), pz = expf(z - mn);
-        l[hh] = l[hh] * corr + pz;
+        for (int s2 = 0; s2 < NT; ++s2) {
+          float acc = 0.f;
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) o[hh][e] = fmaf(o[hh][e], corr, pz * vv[e]);
+          for (int e = 0; e < DPL; ++e) acc = fmaf(q[hh][e], kv[s2][e], acc);
+          z[s2] = acc;
+        }
+#pragma unroll
+        for (int s2 = 0; s2 < NT; ++s2) z[s2] = warp_sum(z[s2]) * sc;
+        float mn = m[hh];
+#pragma unroll
+        for (int s2 = 0; s2 < NT; ++s2)
+          if (u0 + s2 <= u_hi) mn = fmaxf(mn, z[s2]);
+        const float corr = expf(m[hh] - mn);
+        float ps = 0.f;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) o[hh][e] *= corr;
+#pragma unroll
+        for (int s2 = 0; s2 < NT; ++s2) {
+          const float pz = u0 + s2 <= u_hi ? expf(z[s2] - mn) : 0.f;
+          ps += pz;
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) o[hh][e] = fmaf(pz, vv[s2][e], o[hh][e]);
+        }
+        l[hh] = l[hh] * corr + ps;
         m[hh] = mn;
       }
     }
@@ -142,29 +167,47 @@ __global__ void __launch_bounds__(128) backward_q_kernel(BackwardArgs a) {
     const int j = __ldg(srow + i);
     if (j < 0) break;
     if (j > t / a.B) continue;
-    const int u1 = min(j * a.B + a.B - 1, t);
-    for (int u = j * a.B; u <= u1; ++u) {
-      float kv[DPL], vv[DPL];
+    const int u_hi = min(j * a.B + a.B - 1, t);
+    for (int u0 = j * a.B; u0 <= u_hi; u0 += NT) {
+      float kv[NT][DPL], vv[NT][DPL];
 #pragma unroll
-      for (int e = 0; e < DPL; ++e) {
-        kv[e] = bf16_to_f32(__ldg(kseq + u * kv_stride + lane * DPL + e));
-        vv[e] = bf16_to_f32(__ldg(vseq + u * kv_stride + lane * DPL + e));
+      for (int s2 = 0; s2 < NT; ++s2) {
+        const bool ok = u0 + s2 <= u_hi;
+        const int u = ok ? u0 + s2 : u0;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) {
+          kv[s2][e] = bf16_to_f32(__ldg(kseq + u * kv_stride + lane * DPL + e));
+          vv[s2][e] = bf16_to_f32(__ldg(vseq + u * kv_stride + lane * DPL + e));
+        }
       }
 #pragma unroll
       for (int hh = 0; hh < HPW; ++hh) {
         if (hh >= nh) break;
-        float z = 0.f, dp = 0.f;
+        float z[NT], dp[NT];
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) {
-          z = fmaf(q[hh][e], kv[e], z);
-          dp = fmaf(dov[hh][e], vv[e], dp);
+        for (int s2 = 0; s2 < NT; ++s2) {
+          float az = 0.f, ap = 0.f;
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) {
+            az = fmaf(q[hh][e], kv[s2][e], az);
+            ap = fmaf(dov[hh][e], vv[s2][e], ap);
+          }
+          z[s2] = az;
+          dp[s2] = ap;
         }
-        z = warp_sum(z) * sc;
-        dp = warp_sum(dp);
-        const float p = expf(z - lse[hh]);
-        const float dz = p * (dp - Dsum[hh]) * sc;
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) dq[hh][e] = fmaf(dz, kv[e], dq[hh][e]);
+        for (int s2 = 0; s2 < NT; ++s2) {
+          z[s2] = warp_sum(z[s2]) * sc;
+          dp[s2] = warp_sum(dp[s2]);
+        }
+#pragma unroll
+        for (int s2 = 0; s2 < NT; ++s2) {
+          if (u0 + s2 > u_hi) continue;
+          const float p = expf(z[s2] - lse[hh]);
+          const float dz = p * (dp[s2] - Dsum[hh]) * sc;
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) dq[hh][e] = fmaf(dz, kv[s2][e], dq[hh][e]);
+        }
       }
     }
   }
@@ -389,8 +432,14 @@ cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t s) {
   cudaError_t e;
   if ((e = cudaMemsetAsync(a.ccount, 0, (size_t)segs * a.nchunk * a.nblkc * sizeof(int), s)) != cudaSuccess)
     return e;
-  if (a.d == 128) backward_q_kernel<128><<<(unsigned)units, 128, 0, s>>>(a);
-  else backward_q_kernel<64><<<(unsigned)units, 128, 0, s>>>(a);
+  // NT: a whole block of 4 or 8 tokens, or half of a 16-token block, per step
+  if (a.d == 128) {
+    if (a.B == 4) backward_q_kernel<128, 4><<<(unsigned)units, 128, 0, s>>>(a);
+    else backward_q_kernel<128, 8><<<(unsigned)units, 128, 0, s>>>(a);
+  } else {
+    if (a.B == 4) backward_q_kernel<64, 4><<<(unsigned)units, 128, 0, s>>>(a);
+    else backward_q_kernel<64, 8><<<(unsigned)units, 128, 0, s>>>(a);
+  }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   rev_count_kernel<<<(unsigned)((units * 32 + 255) / 256), 256, 0, s>>>(a);
   rev_chunk_scan_kernel<<<(unsigned)((segs * a.nblkc + 255) / 256), 256, 0, s>>>(a);
