@@ -299,22 +299,38 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_bound_kernel(const 
     const uint32_t* tm = tmax + ((long)b * rows + r) * tstride;
     L = kth_largest(n32, m, [&](int i) { return __ldg(tm + i); }, [](int) { return true; }, &rem_dummy);
   }
+  // Both passes below read only the 32-candidate groups whose maximum reaches L (a group below
+  // it holds no key >= L): a warp takes whole groups, four at a time, lane = candidate.
+  const uint32_t* tm = tmax + ((long)b * rows + r) * tstride;
+  const int warp = tid >> 5;
+  constexpr int kWarps = kSelThreads / 32;
+  auto load_groups = [&](int g0, float (&v)[4], bool (&ok)[4]) {
+    uint32_t gm[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int gi = g0 + u * kWarps;
+      gm[u] = gi < n32 ? __ldg(tm + gi) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int gi = g0 + u * kWarps;
+      const int j = gi * 32 + lane;
+      ok[u] = gi < n32 && gm[u] >= L && j < c;
+      v[u] = ok[u] ? __ldg(row + j) : 0.f;
+    }
+  };
   // 2. histogram of the top 12 key bits of the keys >= L
   for (int i = tid; i < kHBins; i += kSelThreads) hist[i] = 0;
   if (tid == 0) { s_cnt = 0; s_pick = 0; }
   __syncthreads();
-  for (int base = 0; base < c; base += 4 * kSelThreads) {
+  for (int g0 = warp; g0 < n32; g0 += 4 * kWarps) {
     float v[4];
+    bool ok[4];
+    load_groups(g0, v, ok);
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int j = base + u * kSelThreads + tid;
-      v[u] = j < c ? __ldg(row + j) : 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int j = base + u * kSelThreads + tid;
       const uint32_t key = score_key(v[u]);
-      hist_add(hist, key >> (32 - kHBits), j < c && key >= L);
+      hist_add(hist, key >> (32 - kHBits), ok[u] && key >= L);
     }
   }
   __syncthreads();
@@ -349,18 +365,15 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_bound_kernel(const 
   const uint32_t lo = (uint32_t)s_bin << (32 - kHBits);
   __syncthreads();  // the histogram area is reused for the survivors below
   // 3. the survivors (keys at or above the threshold bin), any order
-  for (int base = 0; base < c; base += 4 * kSelThreads) {
+  for (int g0 = warp; g0 < n32; g0 += 4 * kWarps) {
     float v[4];
+    bool ok[4];
+    load_groups(g0, v, ok);
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int j = base + u * kSelThreads + tid;
-      v[u] = j < c ? __ldg(row + j) : 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int j = base + u * kSelThreads + tid;
+      const int j = (g0 + u * kWarps) * 32 + lane;
       const uint32_t key = score_key(v[u]);
-      const bool keep = j < c && key >= lo && key >= L;
+      const bool keep = ok[u] && key >= lo && key >= L;
       const unsigned bal = __ballot_sync(0xFFFFFFFFu, keep);
       if (bal == 0u) continue;
       int pos = 0;
