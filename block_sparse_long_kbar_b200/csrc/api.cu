@@ -122,7 +122,7 @@ DecodeWs decode_layout(const sgqa_dims* d, int n_new, void* ws) {
     off += align256((size_t)ug * ucap * 4);
     w.ucount = reinterpret_cast<int*>(base + off);
     off += align256((size_t)ug * 4);
-    w.splits = decode_attend_splits(ug, n_new, Kb, d->B);
+    w.splits = decode_attend_splits(ug, n_new, Kb, d->B, false);  // the larger of the two variants
     w.part = reinterpret_cast<float*>(base + off);
     off += align256(decode_part_bytes(ug, w.splits));
   } else {
@@ -459,7 +459,8 @@ int decode_impl(const sgqa_dims* dims, int cache_len, int n_new, const KvCaches&
     da.k8 = kv.k8; da.v8 = kv.v8; da.k_scale = kv.k_scale; da.v_scale = kv.v_scale;
     da.ublk = w.ublk; da.umask = w.umask; da.ucount = w.ucount; da.ucap = n_new * Kb; da.part = w.part;
     da.batch = dims->batch; da.n_new = n_new; da.t0 = cache_len; da.T_kv = T; da.Hq = dims->Hq; da.G = G; da.d = d;
-    da.B = B; da.splits = w.splits; da.status = w.status; da.stall_cta = g_test_stall_cta;
+    da.B = B; da.status = w.status; da.stall_cta = g_test_stall_cta;
+    da.splits = decode_attend_splits(dims->batch * G, n_new, Kb, B, kv.k8 != nullptr);  // <= w.splits
     if (launch_decode_attend_tc(da, s) != cudaSuccess) return SGQA_ERR_CUDA;
     return SGQA_OK;
   }

@@ -23,8 +23,8 @@
 // output directly when splits == 1).
 //
 // Data movement: K and V tiles of 128 token slots (128/B whole blocks of the union) arrive by 3-D
-// TMA boxes (64 dims x 1 group x B tokens, 128B swizzle) into a two-stage ring; slots past the
-// union are loaded from out of bounds (zero fill) and masked. Warp roles: warp 0 issues TMA, warp
+// TMA boxes (64 dims x 1 group x B tokens, 128B swizzle) into one K and one V stage per CTA, two
+// CTAs per SM; slots past the union are loaded from out of bounds (zero fill) and masked. Warp roles: warp 0 issues TMA, warp
 // 1 allocates TMEM and issues MMAs, warps 2-5 (one per TMEM lane quadrant: a token slot per lane,
 // later a head dimension per lane) compute P and the epilogue. Every wait is bounded by
 // %globaltimer: on expiry the kernel records SGQA_ERR_TIMEOUT, drains its copies and MMAs, frees
@@ -44,8 +44,8 @@ namespace {
 constexpr int kTok = 128;                 // token slots per tile
 constexpr int kNQ = 64;                   // query-head columns
 constexpr int kD = 128;                   // head dim of this kernel
-constexpr int kNK = 3;                    // bf16 caches: K tile stages (free once S^T is issued)
-constexpr int kNV = 2;                    // bf16 caches: V tile stages (free once P V is issued)
+constexpr int kNK = 1;                    // bf16 caches: K tile stages (free once S^T is issued)
+constexpr int kNV = 1;                    // bf16 caches: V tile stages (free once P V is issued)
 constexpr int kSmWarps = 4;
 constexpr int kThreads = (2 + kSmWarps) * 32;
 constexpr int kHalf = kTok * 128;         // one 64-dim half of a K or V tile: [128 tokens][128 B]
@@ -76,13 +76,21 @@ struct DecShared {
 };
 // operand tiles (bf16: the K ring, then the V ring; fp8: one K and one V tile) then, for fp8
 // caches, the staging ring
+// bf16 caches: two CTAs per SM, each with one K stage, one V stage and one P buffer (about 102 KB
+// of shared memory), so that one CTA's hand-offs overlap the other's work; fp8 caches: one CTA
+// per SM with the staging ring and two P buffers.
 template <bool F8>
 struct DaCfg {
-  static constexpr int kOps = F8 ? kStage : (kNK + kNV) * kKV;
+  static constexpr int kRingK = kNK;           // K stages (bf16 caches only)
+  static constexpr int kRingV = kNV;           // V stages (bf16 caches only)
+  static constexpr int kPB = F8 ? 2 : 1;       // P buffers
+  static constexpr int kCtas = F8 ? 1 : 2;     // CTAs per SM
+  static constexpr int kOps = F8 ? kStage : (kRingK + kRingV) * kKV;
   static constexpr int kStaging = F8 ? kS8 * 2 * kRow8 : 0;
-  static constexpr int kSmem = 1024 + kQ + kOps + kStaging + 2 * kP + kOnes + (int)sizeof(DecShared) + 64;
+  static constexpr int kSmem = 1024 + kQ + kOps + kStaging + kPB * kP + kOnes + (int)sizeof(DecShared) + 64;
   static constexpr int kThr = F8 ? kThreads8 : kThreads;
-  static_assert(kSmem <= 232448, "shared memory of one CTA");
+  static_assert(kCtas * (kSmem + 1024) <= 233472, "shared memory of the resident CTAs");
+  static_assert(kCtas * kTmemCols <= 512, "TMEM of the resident CTAs");
 };
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, const int* gstatus) {
@@ -112,7 +120,7 @@ __device__ __forceinline__ uint2 e4m3x4_to_bf16(uint32_t w, float scale) {
 }
 
 template <int B, bool F8>
-__global__ void __launch_bounds__(DaCfg<F8>::kThr, 1)
+__global__ void __launch_bounds__(DaCfg<F8>::kThr, DaCfg<F8>::kCtas)
     decode_attend_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
                             DecodeAttendArgs a) {
   using C = DaCfg<F8>;
@@ -123,7 +131,7 @@ __global__ void __launch_bounds__(DaCfg<F8>::kThr, 1)
   uint8_t* sKV = sQ + kQ;  // [stage][K|V][half][128 tokens][128 B] (one stage for fp8 caches)
   uint8_t* s8 = sKV + C::kOps;  // fp8: [stage][K|V][128 tokens][128 B], 128B swizzle
   uint8_t* sP = s8 + C::kStaging;
-  uint8_t* sOnes = sP + 2 * kP;
+  uint8_t* sOnes = sP + C::kPB * kP;
   DecShared* sh = reinterpret_cast<DecShared*>(sOnes + kOnes);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -143,11 +151,11 @@ __global__ void __launch_bounds__(DaCfg<F8>::kThr, 1)
   // do nothing (the decision is the CTA's, before any barrier or TMEM is set up)
   if (__syncthreads_or(tid == 0 && tc::grid_timed_out(a.status))) return;
   if (tid == 0) {
-    for (int i = 0; i < kNK; ++i) {
+    for (int i = 0; i < C::kRingK; ++i) {
       tc::mbar_init(&sh->kf[i], 1);
       tc::mbar_init(&sh->ke[i], 1);
     }
-    for (int i = 0; i < kNV; ++i) {
+    for (int i = 0; i < C::kRingV; ++i) {
       tc::mbar_init(&sh->vf[i], 1);
       tc::mbar_init(&sh->ve[i], 1);
     }
@@ -162,6 +170,8 @@ __global__ void __launch_bounds__(DaCfg<F8>::kThr, 1)
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&sh->s_full[i], 1);
       tc::mbar_init(&sh->s_empty[i], kSmWarps);
+    }
+    for (int i = 0; i < C::kPB; ++i) {
       tc::mbar_init(&sh->p_full[i], kSmWarps);
       tc::mbar_init(&sh->p_empty[i], 1);
     }
@@ -170,7 +180,7 @@ __global__ void __launch_bounds__(DaCfg<F8>::kThr, 1)
     tc::fence_mbar_init();
   }
   // P buffers start at zero (columns >= NQ are never written), the ones tile is constant
-  for (int i = tid; i < 2 * kP / 16; i += C::kThr) reinterpret_cast<uint4*>(sP)[i] = make_uint4(0, 0, 0, 0);
+  for (int i = tid; i < C::kPB * kP / 16; i += C::kThr) reinterpret_cast<uint4*>(sP)[i] = make_uint4(0, 0, 0, 0);
   for (int i = tid; i < kOnes / 4; i += C::kThr) reinterpret_cast<uint32_t*>(sOnes)[i] = 0x3F803F80u;
   if (tid < kNQ) sh->maxkey[tid] = 0u;
   // Q columns: n = query * R + head (zero beyond NQ); 16-byte chunk c of half h of column n at
@@ -317,8 +327,8 @@ __global__ void __launch_bounds__(DaCfg<F8>::kThr, 1)
           int zk[NB], zv[NB];
           for (int i = tile0; i <= tile1 && !sh->abort_flag; ++i) {
             if (i < tile1) {
-              const int st = (int)(kc % kNK);
-              if (kc >= kNK && !tc::mbar_wait(&sh->ke[st], (uint32_t)(((kc / kNK) - 1) & 1), &sh->abort_flag, a.status)) {
+              const int st = (int)(kc % C::kRingK);
+              if (kc >= C::kRingK && !tc::mbar_wait(&sh->ke[st], (uint32_t)(((kc / C::kRingK) - 1) & 1), &sh->abort_flag, a.status)) {
                 fail();
                 break;
               }
@@ -332,12 +342,12 @@ __global__ void __launch_bounds__(DaCfg<F8>::kThr, 1)
               ++kc;
             }
             if (main_pass && i > tile0) {
-              const int st = (int)(vc % kNV);
-              if (vc >= kNV && !tc::mbar_wait(&sh->ve[st], (uint32_t)(((vc / kNV) - 1) & 1), &sh->abort_flag, a.status)) {
+              const int st = (int)(vc % C::kRingV);
+              if (vc >= C::kRingV && !tc::mbar_wait(&sh->ve[st], (uint32_t)(((vc / C::kRingV) - 1) & 1), &sh->abort_flag, a.status)) {
                 fail();
                 break;
               }
-              uint8_t* dst = sKV + kNK * kKV + st * kKV;
+              uint8_t* dst = sKV + C::kRingK * kKV + st * kKV;
               tc::mbar_arrive_expect_tx(&sh->vf[st], kKV);
 #pragma unroll
               for (int e = 0; e < NB; ++e)
@@ -356,13 +366,13 @@ __global__ void __launch_bounds__(DaCfg<F8>::kThr, 1)
         long pend = -1;
         bool first = true;
         auto issue_pv = [&](long) -> bool {
-          const int pb = (int)(pcnt & 1);
-          if (!tc::mbar_wait(&sh->p_full[pb], (uint32_t)((pcnt >> 1) & 1), &sh->abort_flag, a.status)) return false;
+          const int pb = (int)(pcnt % C::kPB);
+          if (!tc::mbar_wait(&sh->p_full[pb], (uint32_t)((pcnt / C::kPB) & 1), &sh->abort_flag, a.status)) return false;
           if (F8 ? !tc::mbar_wait(&sh->v_full, (uint32_t)(vc & 1), &sh->abort_flag, a.status)
-                 : !tc::mbar_wait(&sh->vf[vc % kNV], (uint32_t)((vc / kNV) & 1), &sh->abort_flag, a.status))
+                 : !tc::mbar_wait(&sh->vf[vc % C::kRingV], (uint32_t)((vc / C::kRingV) & 1), &sh->abort_flag, a.status))
             return false;
           tc::fence_after_sync();
-          const uint8_t* vbase = F8 ? sKV + kKV : sKV + kNK * kKV + (vc % kNV) * kKV;
+          const uint8_t* vbase = F8 ? sKV + kKV : sKV + C::kRingK * kKV + (vc % C::kRingV) * kKV;
           const uint8_t* pbase = sP + pb * kP;
 #pragma unroll
           for (int kk = 0; kk < kTok / 16; ++kk) {
@@ -373,7 +383,7 @@ __global__ void __launch_bounds__(DaCfg<F8>::kThr, 1)
             tc::mma_bf16_ss(tmem_l, d_ones, db, idesc_l, acc);
             first = false;
           }
-          tc::mma_commit(F8 ? &sh->v_empty : &sh->ve[vc % kNV]);
+          tc::mma_commit(F8 ? &sh->v_empty : &sh->ve[vc % C::kRingV]);
           ++vc;
           tc::mma_commit(&sh->p_empty[pb]);
           ++pcnt;
@@ -381,10 +391,10 @@ __global__ void __launch_bounds__(DaCfg<F8>::kThr, 1)
         };
         bool ok = true;
         for (int i = tile0; i < tile1 && ok && !sh->abort_flag; ++i, ++kc, ++scnt) {
-          const int st = F8 ? 0 : (int)(kc % kNK);
+          const int st = F8 ? 0 : (int)(kc % C::kRingK);
           const int sb = (int)(scnt & 1);
           uint64_t* kfull = F8 ? &sh->k_full : &sh->kf[st];
-          const uint32_t kpar = F8 ? (uint32_t)(kc & 1) : (uint32_t)((kc / kNK) & 1);
+          const uint32_t kpar = F8 ? (uint32_t)(kc & 1) : (uint32_t)((kc / C::kRingK) & 1);
           if (!tc::mbar_wait(kfull, kpar, &sh->abort_flag, a.status) ||
               (scnt >= 2 && !tc::mbar_wait(&sh->s_empty[sb], (uint32_t)(((scnt >> 1) - 1) & 1), &sh->abort_flag, a.status))) {
             ok = false;
@@ -524,8 +534,8 @@ __global__ void __launch_bounds__(DaCfg<F8>::kThr, 1)
             if ((cm >> n) & 1ull) atomicMax(&sh->maxkey[n], score_key(__uint_as_float(v[n])));
           continue;
         }
-        const int pb = (int)(pcnt & 1);
-        if (pcnt >= 2 && !warp_wait(&sh->p_empty[pb], (uint32_t)(((pcnt >> 1) - 1) & 1), &sh->abort_flag, a.status)) {
+        const int pb = (int)(pcnt % C::kPB);
+        if (pcnt >= C::kPB && !warp_wait(&sh->p_empty[pb], (uint32_t)(((pcnt / C::kPB) - 1) & 1), &sh->abort_flag, a.status)) {
           if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
           sh->abort_flag = 1;
           break;
@@ -622,10 +632,10 @@ __global__ void __launch_bounds__(DaCfg<F8>::kThr, 1)
       for (long k2 = kc - kS8; k2 < kc; ++k2)
         if (k2 >= 0) tc::mbar_wait(&sh->st8_full[k2 % kS8], (uint32_t)((k2 / kS8) & 1), &no_abort);
     } else {
-      for (long k2 = kc - kNK; k2 < kc; ++k2)
-        if (k2 >= 0) tc::mbar_wait(&sh->kf[k2 % kNK], (uint32_t)((k2 / kNK) & 1), &no_abort);
-      for (long v2 = vc - kNV; v2 < vc; ++v2)
-        if (v2 >= 0) tc::mbar_wait(&sh->vf[v2 % kNV], (uint32_t)((v2 / kNV) & 1), &no_abort);
+      for (long k2 = kc - C::kRingK; k2 < kc; ++k2)
+        if (k2 >= 0) tc::mbar_wait(&sh->kf[k2 % C::kRingK], (uint32_t)((k2 / C::kRingK) & 1), &no_abort);
+      for (long v2 = vc - C::kRingV; v2 < vc; ++v2)
+        if (v2 >= 0) tc::mbar_wait(&sh->vf[v2 % C::kRingV], (uint32_t)((v2 / C::kRingV) & 1), &no_abort);
     }
   }
   if (warp == 1 && lane == 0 && o_commits > 0) {
@@ -822,9 +832,11 @@ bool decode_attend_tc_supported(int Hq, int G, int d, int B, int n_new, int Kb) 
          n_new * Kb <= kUnionMax;
 }
 
-int decode_attend_splits(int units, int n_new, int Kb, int B) {
+int decode_attend_splits(int units, int n_new, int Kb, int B, bool f8) {
   const int max_tiles = (n_new * Kb + kTok / B - 1) / (kTok / B);
-  int s = 148 / (units > 0 ? units : 1);
+  // one wave: 148 SMs x the resident CTAs of the variant
+  const int slots = 148 * (f8 ? DaCfg<true>::kCtas : DaCfg<false>::kCtas);
+  int s = slots / (units > 0 ? units : 1);
   if (s < 1) s = 1;
   if (s > max_tiles) s = max_tiles;
   return s;

@@ -132,7 +132,9 @@ struct DecodeAttendArgs {
   int stall_cta;         // failure-detection test hook: this CTA issues no loads (-1: none)
 };
 bool decode_attend_tc_supported(int Hq, int G, int d, int B, int n_new, int Kb);
-int decode_attend_splits(int units, int n_new, int Kb, int B);
+// splits per (sequence, group) unit: one wave of the variant's resident CTAs (f8: FP8 caches);
+// the bf16 variant's count is the larger and sizes the workspace
+int decode_attend_splits(int units, int n_new, int Kb, int B, bool f8);
 size_t decode_part_bytes(int units, int splits);
 cudaError_t launch_decode_union(const int32_t* sel, int batch, int n_new, int G, int Kb, int32_t* ublk,
                                 uint32_t* umask, int* ucount, int ucap, int* status, cudaStream_t s);
