@@ -188,9 +188,10 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const float*
 // over their keys for the threshold key K*, and among the candidates equal to K* the lowest block
 // ids (radix passes over ~j); the chosen ids are sorted (bitonic) and written ascending. A row
 // whose threshold bin alone holds more than kCap candidates takes the full radix path instead.
-constexpr int kCap = 8192;
+constexpr int kCap = 7168;
 constexpr int kHBits = 12;
 constexpr int kHBins = 1 << kHBits;
+constexpr int kGl = 4096;  // groups listed at a time
 
 // Warp-aggregated histogram increment of bin `bin` (lanes with want == false add nothing).
 __device__ __forceinline__ void hist_add(int* hist, uint32_t bin, bool want) {
@@ -264,7 +265,7 @@ __device__ uint32_t kth_largest(int n, int m, Get get, Valid valid, int* rem_out
   return res;
 }
 
-__global__ void __launch_bounds__(kSelThreads) decode_select_bound_kernel(const float* __restrict__ scores,
+__global__ void __launch_bounds__(kSelThreads, 3) decode_select_bound_kernel(const float* __restrict__ scores,
                                                                           const uint32_t* __restrict__ tmax,
                                                                           int32_t* __restrict__ sel, int n_new, int G,
                                                                           int B, int Kb, int nblk, int tstride, int t0,
@@ -273,8 +274,10 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_bound_kernel(const 
   uint32_t* skey = sm;               // [kCap]
   uint32_t* sj = sm + kCap;          // [kCap]
   uint32_t* sorted = sm + 2 * kCap;  // [sort_n]
+  uint16_t* glist = reinterpret_cast<uint16_t*>(sorted + sort_n);  // [kGl] groups that reach L
   int* hist = reinterpret_cast<int*>(sm);  // [kHBins], before the survivors are collected
-  __shared__ int s_cnt, s_pick, s_bin, s_total;
+  uint32_t* stm = sj;                      // [n32] the row's group maxima while L is found
+  __shared__ int s_cnt, s_pick, s_bin, s_total, s_ng;
   __shared__ int scratch[64];
   const int rows = n_new * G;
   const int b = blockIdx.x / rows, r = blockIdx.x % rows;
@@ -291,49 +294,69 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_bound_kernel(const 
     for (int i = tid; i < Kb; i += kSelThreads) out[i] = i == 0 ? c : -1;
     return;
   }
-  // 1. the bound L from the maxima of 32 candidates
+  // 1. the bound L from the maxima of 32 candidates (staged in shared memory when they fit)
   const int n32 = (c + 31) / 32;
+  const uint32_t* tm = tmax + ((long)b * rows + r) * tstride;
   uint32_t L = 0;
   int rem_dummy;
   if (n32 >= m) {
-    const uint32_t* tm = tmax + ((long)b * rows + r) * tstride;
-    L = kth_largest(n32, m, [&](int i) { return __ldg(tm + i); }, [](int) { return true; }, &rem_dummy);
+    if (n32 <= kCap) {
+      for (int i = tid; i < n32; i += kSelThreads) stm[i] = __ldg(tm + i);
+      __syncthreads();
+      L = kth_largest(n32, m, [&](int i) { return stm[i]; }, [](int) { return true; }, &rem_dummy);
+    } else {
+      L = kth_largest(n32, m, [&](int i) { return __ldg(tm + i); }, [](int) { return true; }, &rem_dummy);
+    }
   }
   // Both passes below read only the 32-candidate groups whose maximum reaches L (a group below
-  // it holds no key >= L): a warp takes whole groups, four at a time, lane = candidate.
-  const uint32_t* tm = tmax + ((long)b * rows + r) * tstride;
+  // it holds no key >= L). Those groups are first listed in shared memory, kGl at a time, so that
+  // a warp then loads 8 listed groups at once (lane = candidate) with no dependent load in front.
   const int warp = tid >> 5;
   constexpr int kWarps = kSelThreads / 32;
-  auto load_groups = [&](int g0, float (&v)[4], bool (&ok)[4]) {
-    uint32_t gm[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int gi = g0 + u * kWarps;
-      gm[u] = gi < n32 ? __ldg(tm + gi) : 0u;
+  auto list_groups = [&](int g_begin) {  // all threads; returns the number listed
+    if (tid == 0) s_ng = 0;
+    __syncthreads();
+    const int g_end = min(n32, g_begin + kGl);
+    for (int g0 = g_begin; g0 < g_end; g0 += kSelThreads) {
+      const int gi = g0 + tid;
+      const bool keep = gi < g_end && __ldg(tm + gi) >= L;
+      const unsigned bal = __ballot_sync(0xFFFFFFFFu, keep);
+      int pos = 0;
+      if (lane == 0 && bal) pos = atomicAdd(&s_ng, __popc(bal));
+      pos = __shfl_sync(0xFFFFFFFFu, pos, 0) + __popc(bal & ((1u << lane) - 1u));
+      if (keep) glist[pos] = (uint16_t)(gi - g_begin);
     }
+    __syncthreads();
+    return s_ng;
+  };
+  // f(j, key, ok) for every candidate of the listed groups (ok: j < c and key >= L); all threads
+  auto for_listed = [&](int g_begin, int ng, auto&& f) {
+    for (int e0 = warp * 8; e0 < ng; e0 += 8 * kWarps) {
+      float v[8];
+      int j[8];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int gi = g0 + u * kWarps;
-      const int j = gi * 32 + lane;
-      ok[u] = gi < n32 && gm[u] >= L && j < c;
-      v[u] = ok[u] ? __ldg(row + j) : 0.f;
+      for (int u = 0; u < 8; ++u) {
+        j[u] = e0 + u < ng ? (g_begin + (int)glist[e0 + u]) * 32 + lane : c;
+        v[u] = j[u] < c ? __ldg(row + j[u]) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t key = score_key(v[u]);
+        f(j[u], key, j[u] < c && key >= L);
+      }
     }
   };
   // 2. histogram of the top 12 key bits of the keys >= L
   for (int i = tid; i < kHBins; i += kSelThreads) hist[i] = 0;
   if (tid == 0) { s_cnt = 0; s_pick = 0; }
   __syncthreads();
-  for (int g0 = warp; g0 < n32; g0 += 4 * kWarps) {
-    float v[4];
-    bool ok[4];
-    load_groups(g0, v, ok);
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const uint32_t key = score_key(v[u]);
-      hist_add(hist, key >> (32 - kHBits), ok[u] && key >= L);
-    }
+  int ng_first = 0;
+  for (int gb = 0; gb < n32; gb += kGl) {
+    const int ng = list_groups(gb);
+    if (gb == 0) ng_first = ng;
+    for_listed(gb, ng, [&](int, uint32_t key, bool ok) { hist_add(hist, key >> (32 - kHBits), ok); });
+    __syncthreads();  // the list is rebuilt for the next chunk
   }
-  __syncthreads();
   // the bin of the m-th largest key: suffix sums over 8 bins per thread, scanned from the top
   {
     constexpr int kPer = kHBins / kSelThreads;
@@ -364,25 +387,27 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_bound_kernel(const 
   }
   const uint32_t lo = (uint32_t)s_bin << (32 - kHBits);
   __syncthreads();  // the histogram area is reused for the survivors below
-  // 3. the survivors (keys at or above the threshold bin), any order
-  for (int g0 = warp; g0 < n32; g0 += 4 * kWarps) {
-    float v[4];
-    bool ok[4];
-    load_groups(g0, v, ok);
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int j = (g0 + u * kWarps) * 32 + lane;
-      const uint32_t key = score_key(v[u]);
-      const bool keep = ok[u] && key >= lo && key >= L;
-      const unsigned bal = __ballot_sync(0xFFFFFFFFu, keep);
-      if (bal == 0u) continue;
-      int pos = 0;
-      if (lane == __ffs(bal) - 1) pos = atomicAdd(&s_cnt, __popc(bal));
-      pos = __shfl_sync(0xFFFFFFFFu, pos, __ffs(bal) - 1) + __popc(bal & ((1u << lane) - 1u));
-      if (keep && pos < kCap) {
-        skey[pos] = key;
-        sj[pos] = (uint32_t)j;
-      }
+  // 3. the survivors (keys at or above the threshold bin), any order; the list of the first
+  // chunk is still in place when it was the only one
+  auto keep_survivor = [&](int j, uint32_t key, bool ok) {
+    const bool keep = ok && key >= lo;
+    const unsigned bal = __ballot_sync(0xFFFFFFFFu, keep);
+    if (bal == 0u) return;
+    int pos = 0;
+    if (lane == __ffs(bal) - 1) pos = atomicAdd(&s_cnt, __popc(bal));
+    pos = __shfl_sync(0xFFFFFFFFu, pos, __ffs(bal) - 1) + __popc(bal & ((1u << lane) - 1u));
+    if (keep && pos < kCap) {
+      skey[pos] = key;
+      sj[pos] = (uint32_t)j;
+    }
+  };
+  if (n32 <= kGl) {
+    for_listed(0, ng_first, keep_survivor);
+  } else {
+    for (int gb = 0; gb < n32; gb += kGl) {
+      const int ng = list_groups(gb);
+      for_listed(gb, ng, keep_survivor);
+      __syncthreads();
     }
   }
   __syncthreads();
@@ -470,7 +495,7 @@ cudaError_t launch_decode_select_bound(const float* scores, const uint32_t* tmax
                                        cudaStream_t s) {
   int sort_n = 1;
   while (sort_n < Kb) sort_n <<= 1;
-  const size_t shmem = (size_t)(2 * kCap + sort_n) * 4;
+  const size_t shmem = (size_t)(2 * kCap + sort_n) * 4 + kGl * sizeof(uint16_t);
   cudaError_t e = cudaFuncSetAttribute(decode_select_bound_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)shmem);
   if (e != cudaSuccess) return e;

@@ -742,28 +742,28 @@ __global__ void __launch_bounds__(256) decode_union_kernel(const int32_t* __rest
   }
 }
 
-// Fixed-order merge of the splits' partial records, then the gate: thread = head dimension.
+// Fixed-order merge of the splits' partial records, then the gate: block = (unit, column),
+// thread = head dimension.
 __global__ void __launch_bounds__(kD) decode_merge_kernel(DecodeAttendArgs a) {
   if (tc::grid_timed_out(a.status)) return;  // the partial records of a stopped launch are incomplete
-  const int unit = blockIdx.x, b = unit / a.G, g = unit % a.G;
-  const int R = a.Hq / a.G, NQ = a.n_new * R;
+  const int unit = blockIdx.x, n = blockIdx.y, b = unit / a.G, g = unit % a.G;
+  const int R = a.Hq / a.G;
   const int r = threadIdx.x;
-  const float* base = a.part + (long)unit * a.splits * (2 * kNQ + kNQ * kD);
-  for (int n = 0; n < NQ; ++n) {
-    float mstar = -INFINITY;
-    for (int s = 0; s < a.splits; ++s) mstar = fmaxf(mstar, base[(long)s * (2 * kNQ + kNQ * kD) + n]);
-    float den = 0.f, num = 0.f;
-    for (int s = 0; s < a.splits; ++s) {
-      const float* rec = base + (long)s * (2 * kNQ + kNQ * kD);
-      const float ms = rec[n];
-      const float w = ms == -INFINITY ? 0.f : exp2f(ms - mstar);
-      den += w * rec[kNQ + n];
-      num += w * rec[2 * kNQ + n * kD + r];
-    }
-    const long off = (((long)b * a.n_new + n / R) * a.Hq + (long)g * R + (n % R)) * kD + r;
-    const float y = den > 0.f ? num / den : 0.f;
-    a.out[off] = f32_to_bf16_rne(y * sigmoid_fast(bf16_to_f32(__ldg(a.gate + off))));
+  constexpr long kRec = 2 * kNQ + kNQ * kD;
+  const float* base = a.part + (long)unit * a.splits * kRec;
+  float mstar = -INFINITY;
+  for (int s = 0; s < a.splits; ++s) mstar = fmaxf(mstar, __ldg(base + s * kRec + n));
+  float den = 0.f, num = 0.f;
+  for (int s = 0; s < a.splits; ++s) {
+    const float* rec = base + s * kRec;
+    const float ms = __ldg(rec + n);
+    const float w = ms == -INFINITY ? 0.f : exp2f(ms - mstar);
+    den += w * __ldg(rec + kNQ + n);
+    num += w * __ldg(rec + 2 * kNQ + n * kD + r);
   }
+  const long off = (((long)b * a.n_new + n / R) * a.Hq + (long)g * R + (n % R)) * kD + r;
+  const float y = den > 0.f ? num / den : 0.f;
+  a.out[off] = f32_to_bf16_rne(y * sigmoid_fast(bf16_to_f32(__ldg(a.gate + off))));
 }
 
 using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -861,7 +861,7 @@ cudaError_t launch_decode_attend_tc(const DecodeAttendArgs& a, cudaStream_t s) {
                   : a.B == 16 ? (f8 ? launch_b<16, true>(a, s) : launch_b<16, false>(a, s))
                               : cudaErrorInvalidValue;
   if (e != cudaSuccess || a.splits == 1) return e;
-  decode_merge_kernel<<<(unsigned)(a.batch * a.G), kD, 0, s>>>(a);
+  decode_merge_kernel<<<dim3((unsigned)(a.batch * a.G), (unsigned)(a.n_new * (a.Hq / a.G))), kD, 0, s>>>(a);
   return cudaGetLastError();
 }
 
