@@ -132,19 +132,34 @@ __device__ __forceinline__ void red_shared_inc(uint32_t addr) {
   asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(addr) : "memory");
 }
 
-// Histogram pass: count, in the row's 256 bins, the next 8 key bits (at `shift`) of the keys
-// whose resolved bits (mask) equal prefix; every other key increments the row's spare slot, so
-// every lane stays active. kFull: all 64 candidates exist (else only q < lim).
+// Histogram pass over the raw float bits (the order-preserving key is applied to the bins, once
+// per row, when the histogram is read): count, in the row's 256 bins, the 8 raw bits at `shift`
+// of the scores whose resolved raw bits (mask) equal prefix; every other score increments the
+// row's spare slot, so every lane stays active. Adding +0.0 first makes -0.0 the same score as
+// +0.0. kFull: all 64 candidates exist (else only q < lim).
 template <bool kFull, bool kFirst>
 __device__ __forceinline__ void hist_chunk(const uint32_t (&v)[64], int lim, uint32_t mask, uint32_t prefix, int shift,
                                            uint32_t hbase) {
 #pragma unroll
   for (int q = 0; q < 64; ++q) {
-    const uint32_t key = score_key(__uint_as_float(v[q]));
-    const uint32_t addr = hbase + (((key >> shift) & 255u) * (kRows * 4u));
+    const uint32_t raw = __float_as_uint(__uint_as_float(v[q]) + 0.0f);
+    const uint32_t addr = hbase + (((raw >> shift) & 255u) * (kRows * 4u));
     if (kFull && kFirst) red_shared_inc(addr);
-    else red_shared_inc(((kFull || q < lim) && (kFirst || (key & mask) == prefix)) ? addr : hbase + kTrash * (kRows * 4u));
+    else red_shared_inc(((kFull || q < lim) && (kFirst || (raw & mask) == prefix)) ? addr : hbase + kTrash * (kRows * 4u));
   }
+}
+
+// Raw-bits view of a key prefix: the resolved raw bits, and whether the digits run in reverse
+// (negative scores: raw = ~key). The sign is the key's top bit, resolved with the first digit.
+__device__ __forceinline__ uint32_t raw_prefix(uint32_t prefix, uint32_t mask) {
+  return (prefix & 0x80000000u) ? (prefix ^ 0x80000000u) : (~prefix & mask);
+}
+
+// The raw bin holding key bin kb of the digit at this level: the first digit maps key top bytes
+// 128..255 (non-negative scores) to raw 0..127 and 0..127 (negative) to raw 255..128; later
+// digits of a negative prefix run in reverse.
+__device__ __forceinline__ int raw_bin(int kb, bool first, bool neg) {
+  return first ? (kb >= 128 ? kb - 128 : 255 - kb) : (neg ? 255 - kb : kb);
 }
 
 // v[q] for a run-time q, keeping the array in registers (used only for the rare bucket keys)
@@ -444,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int shift = 24 - 8 * pass;
         // a resolved row matches nothing (its histogram is not read; in the first pass it may
         // count, harmlessly)
-        const uint32_t mk = done ? 0u : mask, pf = done ? 1u : prefix;
+        const uint32_t mk = done ? 0u : mask, pf = done ? 1u : raw_prefix(prefix, mask);
         for (int i = 0; i < n_nt; ++i, ++k) {
           const int buf = (int)(k & 1);
           if (!warp_wait(&sh->acc_full[buf], (uint32_t)((k >> 1) & 1), &sh->abort_flag, a.status)) {
@@ -479,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!done) {
           int above = 0;
           for (int bin = 255; bin >= 0; --bin) {
-            const int h = (int)my_hist[bin * kRows];
+            const int h = (int)my_hist[raw_bin(bin, pass == 0, (prefix & 0x80000000u) == 0u) * kRows];
             if (above + h >= rem) {
               prefix |= (uint32_t)bin << shift;
               mask |= 255u << shift;
