@@ -234,16 +234,26 @@ __device__ __forceinline__ uint32_t pick64(const uint32_t (&v)[64], int q) {
 }
 
 // Emit pass, 64 consecutive candidates of a row: bits of the taken keys (key >= thr) in tb and,
-// with kBucket, of the bucket keys (blo <= key <= blo + bw) in bb. ALU only.
-template <bool kFull, bool kBucket>
+// with kBucket, of the bucket keys (blo <= key <= blo + bw) in bb. ALU only. kPos (thr above the
+// key of +0.0, and blo at or above it): the comparisons run on the raw float bits, which order
+// the non-negative scores as their keys do and put every negative score (and -0.0) below thr and
+// outside the bucket.
+template <bool kFull, bool kBucket, bool kPos>
 __device__ __forceinline__ void emit_bits(const uint32_t (&v)[64], int lim, uint32_t thr, uint32_t blo, uint32_t bw,
                                           uint32_t (&tb)[2], uint32_t (&bb)[2]) {
+  const int thr_raw = (int)(thr ^ 0x80000000u);
+  const uint32_t blo_raw = blo ^ 0x80000000u;
 #pragma unroll
   for (int q = 0; q < 64; ++q) {
-    const uint32_t key = score_key(__uint_as_float(v[q]));
     const bool in = kFull || q < lim;
-    tb[q >> 5] |= (in && key >= thr) ? (1u << (q & 31)) : 0u;
-    if (kBucket) bb[q >> 5] |= (in && key - blo <= bw) ? (1u << (q & 31)) : 0u;
+    if (kPos) {
+      tb[q >> 5] |= (in && (int)v[q] >= thr_raw) ? (1u << (q & 31)) : 0u;
+      if (kBucket) bb[q >> 5] |= (in && v[q] - blo_raw <= bw) ? (1u << (q & 31)) : 0u;
+    } else {
+      const uint32_t key = score_key(__uint_as_float(v[q]));
+      tb[q >> 5] |= (in && key >= thr) ? (1u << (q & 31)) : 0u;
+      if (kBucket) bb[q >> 5] |= (in && key - blo <= bw) ? (1u << (q & 31)) : 0u;
+    }
   }
 }
 
@@ -539,6 +549,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // identical in the two warps of a row pair (same rows, same state)
       const bool any_bucket = __any_sync(0xFFFFFFFFu, collect || ties);
+      // every row of the warp has a positive threshold (and bucket): raw-bit comparisons
+      const bool pos = __all_sync(0xFFFFFFFFu, thr > 0x80000000u && blo >= 0x80000000u);
       const bool any_ties = __any_sync(0xFFFFFFFFu, ties);
       uint32_t* cand = my_hist + 128 * half * kRows;  // collected (key, j) pairs of this half (stride kRows)
       volatile uint32_t* slot = my_hist;              // tie counts: [half][tile parity] (stride kRows)
@@ -560,11 +572,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::tmem_ld64(tmem + lane_base + (uint32_t)(buf * kN + half * 64), v);
           const bool full = __all_sync(0xFFFFFFFFu, lim >= 64);
           if (any_bucket) {
-            if (full) emit_bits<true, true>(v, lim, thr, blo, bw, tb, bb);
-            else emit_bits<false, true>(v, lim, thr, blo, bw, tb, bb);
+            if (full && pos) emit_bits<true, true, true>(v, lim, thr, blo, bw, tb, bb);
+            else if (full) emit_bits<true, true, false>(v, lim, thr, blo, bw, tb, bb);
+            else emit_bits<false, true, false>(v, lim, thr, blo, bw, tb, bb);
           } else {
-            if (full) emit_bits<true, false>(v, lim, thr, blo, bw, tb, bb);
-            else emit_bits<false, false>(v, lim, thr, blo, bw, tb, bb);
+            if (full && pos) emit_bits<true, false, true>(v, lim, thr, blo, bw, tb, bb);
+            else if (full) emit_bits<true, false, false>(v, lim, thr, blo, bw, tb, bb);
+            else emit_bits<false, false, false>(v, lim, thr, blo, bw, tb, bb);
           }
           if (collect) {  // the few bucket keys of an unresolved row, kept as (key, j) pairs
 #pragma unroll
