@@ -134,18 +134,19 @@ __device__ __forceinline__ void red_shared_inc(uint32_t addr) {
 
 // Histogram pass over the raw float bits (the order-preserving key is applied to the bins, once
 // per row, when the histogram is read): count, in the row's 256 bins, the 8 raw bits at `shift`
-// of the scores whose resolved raw bits (mask) equal prefix; every other score increments the
-// row's spare slot, so every lane stays active. Adding +0.0 first makes -0.0 the same score as
-// +0.0. kFull: all 64 candidates exist (else only q < lim).
+// of the scores whose resolved raw bits equal prefix (whose other bits are zero). With
+// x = (raw ^ prefix) >> shift, a matching score has x = its bin and any other x > 255, so
+// min(x, 256) sends the others to the row's spare slot: every lane stays active. Adding +0.0
+// first makes -0.0 the same score as +0.0. kFull: all 64 candidates exist (else only q < lim).
 template <bool kFull, bool kFirst>
-__device__ __forceinline__ void hist_chunk(const uint32_t (&v)[64], int lim, uint32_t mask, uint32_t prefix, int shift,
+__device__ __forceinline__ void hist_chunk(const uint32_t (&v)[64], int lim, uint32_t prefix, int shift,
                                            uint32_t hbase) {
 #pragma unroll
   for (int q = 0; q < 64; ++q) {
     const uint32_t raw = __float_as_uint(__uint_as_float(v[q]) + 0.0f);
-    const uint32_t addr = hbase + (((raw >> shift) & 255u) * (kRows * 4u));
-    if (kFull && kFirst) red_shared_inc(addr);
-    else red_shared_inc(((kFull || q < lim) && (kFirst || (raw & mask) == prefix)) ? addr : hbase + kTrash * (kRows * 4u));
+    uint32_t x = kFirst ? raw >> 24 : min((raw ^ prefix) >> shift, (uint32_t)kTrash);
+    if (!kFull) x = q < lim ? x : (uint32_t)kTrash;
+    red_shared_inc(hbase + x * (kRows * 4u));
   }
 }
 
@@ -467,9 +468,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!is_emit) {
         const int shift = 24 - 8 * pass;
-        // a resolved row matches nothing (its histogram is not read; in the first pass it may
-        // count, harmlessly)
-        const uint32_t mk = done ? 0u : mask, pf = done ? 1u : raw_prefix(prefix, mask);
+        // a resolved row counts too, harmlessly: its histogram is not read, and its tie-count
+        // slots are zeroed at the start of the emit pass
+        const uint32_t pf = raw_prefix(prefix, mask);
         for (int i = 0; i < n_nt; ++i, ++k) {
           const int buf = (int)(k & 1);
           if (!warp_wait(&sh->acc_full[buf], (uint32_t)((k >> 1) & 1), &sh->abort_flag, a.status)) {
@@ -486,11 +487,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) tc::mbar_arrive(&sh->acc_empty[buf]);
           const int lim = c - (i * kN + half * 64);
           if (__all_sync(0xFFFFFFFFu, lim >= 64)) {
-            if (pass == 0) hist_chunk<true, true>(v, lim, mk, pf, shift, hbase);
-            else hist_chunk<true, false>(v, lim, mk, pf, shift, hbase);
+            if (pass == 0) hist_chunk<true, true>(v, lim, pf, shift, hbase);
+            else hist_chunk<true, false>(v, lim, pf, shift, hbase);
           } else if (lim > 0) {
-            if (pass == 0) hist_chunk<false, true>(v, lim, mk, pf, shift, hbase);
-            else hist_chunk<false, false>(v, lim, mk, pf, shift, hbase);
+            if (pass == 0) hist_chunk<false, true>(v, lim, pf, shift, hbase);
+            else hist_chunk<false, false>(v, lim, pf, shift, hbase);
           }
         }
         if (aborted) break;
