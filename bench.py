@@ -45,11 +45,11 @@ CLOCK_FIELDS = ["pci.bus_id", "clocks.sm", "clocks.max.sm", "power.draw", "clock
 # that produced them are under profiles/.
 NCU_TRAFFIC: dict = {
     # profiles/traffic_prefill128k_decode1m.md, the bench's own 128K / 1M workloads
-    ("attend", "128k"): (6524326400 + 1068357120, "90290afbbced3240"),   # one attend_tc launch
-    ("select", "128k"): (89709568 + 343720192 + 311718656 + 823901952, "dee08ffbc95d9e6e"),  # 4 select_tc + 4 sel_from_bits
-    ("decode_scores", "decode_1m"): (1074968832 + 252713216, "0669c7900a2898e8"),
-    ("decode_select", "decode_1m"): (509710080 + 136960, "6b1e39bfc032a2cd"),
-    ("decode_attend", "decode_1m"): (1073845760 + 239104, "0b27aa0c5434674b"),
+    ("attend", "128k"): (6510472704 + 1068722176, "0ae683a6e388e866"),   # one attend_tc launch
+    ("select", "128k"): (89756416 + 343489280 + 311815424 + 823727616, "474d06fa298073ce"),  # 4 select_tc + 4 sel_from_bits
+    ("decode_scores", "decode_1m"): (1075092224 + 253289728, "0669c7900a2898e8"),
+    ("decode_select", "decode_1m"): (45581568 + 768, "cc7074bb7dae8bdd"),
+    ("decode_attend", "decode_1m"): (1072802816 + 567552, "f1b37928fec6438e"),
 }
 STAGE_SOURCES = {"compress": "compress.cu", "select": "select_tc.cu", "attend": "attend_tc.cu",
                  "decode_scores": "decode_scores_tc.cu", "decode_select": "decode.cu",
@@ -109,14 +109,15 @@ def work_counts(cfg):
 
 
 # Per-key instruction counts of the select kernel's epilogue (select_tc.cu), per pass over the
-# scored candidates: a histogram pass spends about 8 thread-instructions per key (order-preserving
-# key, bin address, prefix test, shared reduction); the emit pass about 8 (key, two compares, two
-# bit updates) plus a bitmap store per 32 keys; the tile's TMEM load adds 2 per key per pass. A
-# typical 128K row (topic-clustered scores) resolves its threshold bucket after 2 histogram passes:
-# the first isolates its topic's blocks, the second leaves a bucket of a few keys, collected in the
-# emit pass.
-SELECT_INSTR_PER_KEY = {"hist": 8 + 2, "emit": 8 + 2}
-SELECT_PASSES = {"hist": 2, "emit": 1}
+# scored candidates. The histogram passes work on the raw float bits: the first spends about 4
+# thread-instructions per key (+0.0 add, top byte, bin address, shared reduction), a later one
+# about 6 (+0.0 add, xor with the prefix, shift, min with the spare slot, address, reduction); the
+# emit pass about 6 (two raw-bit compares, two bit updates, the bucket offset) plus a bitmap store
+# per 32 keys; the tile's TMEM load adds 2 per key per pass. A typical 128K row (topic-clustered
+# scores) resolves its threshold bucket after 2 histogram passes: the first isolates its topic's
+# blocks, the second leaves a bucket of a few keys, collected in the emit pass.
+SELECT_INSTR_PER_KEY = {"hist_first": 4 + 2, "hist_next": 6 + 2, "emit": 6 + 2}
+SELECT_PASSES = {"hist_first": 1, "hist_next": 1, "emit": 1}
 
 
 def select_ranges(cfg, nq: int) -> int:

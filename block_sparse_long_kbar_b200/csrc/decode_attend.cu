@@ -654,7 +654,7 @@ __global__ void __launch_bounds__(DaCfg<F8>::kThr, DaCfg<F8>::kCtas)
 // per block, the mask of the queries that selected it. Each list is ascending; an element is
 // written by the lowest list that holds it, at the rank given by counting, in every list, the
 // elements below it that their lowest lists own (binary searches; no sort).
-__global__ void __launch_bounds__(256) decode_union_kernel(const int32_t* __restrict__ sel, int n_new, int G, int Kb,
+__global__ void __launch_bounds__(1024) decode_union_kernel(const int32_t* __restrict__ sel, int n_new, int G, int Kb,
                                                            int32_t* __restrict__ ublk, uint32_t* __restrict__ umask,
                                                            int* __restrict__ ucount, int ucap, int* status) {
   extern __shared__ int su[];
@@ -851,7 +851,9 @@ cudaError_t launch_decode_union(const int32_t* sel, int batch, int n_new, int G,
   const size_t shmem = (size_t)n_new * Kb * 12;
   cudaError_t e = cudaFuncSetAttribute(decode_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shmem);
   if (e != cudaSuccess) return e;
-  decode_union_kernel<<<(unsigned)(batch * G), 256, shmem, s>>>(sel, n_new, G, Kb, ublk, umask, ucount, ucap, status);
+  // one CTA per (sequence, group): 1024 threads, two or so entries each, so that the binary
+  // searches of many threads overlap
+  decode_union_kernel<<<(unsigned)(batch * G), 1024, shmem, s>>>(sel, n_new, G, Kb, ublk, umask, ucount, ucap, status);
   return cudaGetLastError();
 }
 
