@@ -47,9 +47,9 @@ NCU_TRAFFIC: dict = {
     # profiles/traffic_prefill128k_decode1m.md, the bench's own 128K / 1M workloads
     ("attend", "128k"): (6510472704 + 1068722176, "0ae683a6e388e866"),   # one attend_tc launch
     ("select", "128k"): (89756416 + 343489280 + 311815424 + 823727616, "474d06fa298073ce"),  # 4 select_tc + 4 sel_from_bits
-    ("decode_scores", "decode_1m"): (1075092224 + 253289728, "0669c7900a2898e8"),
-    ("decode_select", "decode_1m"): (45581568 + 768, "cc7074bb7dae8bdd"),
-    ("decode_attend", "decode_1m"): (1072802816 + 567552, "f1b37928fec6438e"),
+    ("decode_scores", "decode_1m"): (1074967296 + 252742400, "0669c7900a2898e8"),
+    ("decode_select", "decode_1m"): (45581824 + 512, "cc7074bb7dae8bdd"),
+    ("decode_attend", "decode_1m"): (1072768256 + 274176, "f4009ea09891d2e4"),
 }
 STAGE_SOURCES = {"compress": "compress.cu", "select": "select_tc.cu", "attend": "attend_tc.cu",
                  "decode_scores": "decode_scores_tc.cu", "decode_select": "decode.cu",
