@@ -15,17 +15,17 @@
 // fp32; splitting it into bf16 hi + lo planes keeps the product exact to ~2^-17 relative, and
 // q_idx is exactly bf16, so the contraction runs at the bf16 tensor rate.
 //
-// Warp roles: warp 8 issues TMA loads, warp 9 allocates TMEM and issues MMAs, warps 0-7 are the
-// epilogue, two per TMEM lane quadrant (TMEM lane = row); each of the two takes half of every
-// tile's columns. The epilogue performs an exact radix select of the m-th largest order-preserving
+// Warp roles: warp 16 issues TMA loads, warp 17 allocates TMEM and issues MMAs, warps 0-15 are
+// the epilogue, four per TMEM lane quadrant (TMEM lane = row); each of the four takes a quarter
+// (32 columns) of every tile, so that every scheduler interleaves four epilogue warps. The epilogue performs an exact radix select of the m-th largest order-preserving
 // 32-bit score key per row: every pass re-streams the same score tiles (recomputed,
 // bit-identical); in a histogram pass each thread adds its keys that still match the resolved
 // prefix to the row's 256-bin shared histogram of the next 8 key bits (keys that do not match go
 // to a spare slot of the row, so the shared-memory reductions stay branch-free and mostly free of
 // bank conflicts). Once every row's threshold bucket is resolved or taken whole, the emit pass
-// marks the taken candidates of each 64-column half-tile in two 32-bit words and stores them to
+// marks the taken candidates of each 32-column quarter-tile in one 32-bit word and stores it to
 // the row's bitmap in global memory: keys above the threshold; bucket keys taken whole; exact ties
-// in j order (the two threads of a row exchange their tie counts through shared memory, so ties
+// in j order (the four threads of a row exchange their tie counts through shared memory, so ties
 // go to the lower block index); or, when every unresolved row's bucket is small (from the third
 // pass on), the bucket keys are collected and resolved exactly afterwards, their bits set with
 // atomics. A separate kernel expands every row's bitmap into the ascending block list, appends
@@ -47,13 +47,19 @@ constexpr int kRows = 128;
 constexpr int kN = 128;          // candidate blocks per MMA tile
 constexpr int kStages = 2;
 constexpr int kHistStride = 257;  // words per row (256 bins + spare slot); stored bin-major, below
-constexpr int kEpiWarps = 8;     // two per TMEM lane quadrant: each histograms half the columns
+constexpr int kParts = 4;        // epilogue warps per TMEM lane quadrant, each takes kCols columns
+constexpr int kCols = kN / kParts;
+constexpr int kEpiWarps = 4 * kParts;
+static_assert(kCols == 32, "one bitmap word per part and tile");
 constexpr int kThreads = (kEpiWarps + 2) * 32;
 constexpr int kProducerWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
 constexpr int kMaxPasses = 5;
-constexpr int kCap = 63;         // bucket keys a row may collect for an early exact finish (per half, 2 words each)
+constexpr int kCap = 31;         // bucket keys a row may collect for an early exact finish (2 words each)
+constexpr int kCandWords = 2 * kCap;  // words of one part's collected keys
 constexpr int kTrash = 256;      // the row's spare histogram slot: target of the keys that do not count
-constexpr int kCnt1 = 254;       // the upper half's collected count and taken count of the row (emit pass)
+constexpr int kCntBase = kParts * kCandWords;  // parts 1..: collected count and taken count (emit pass)
+constexpr int kTieWords = 2 * kParts;          // tie-count slots [part][tile parity]
+static_assert(kCntBase + 2 * (kParts - 1) <= kTrash, "per-row words of the emit pass");
 
 template <int DI>
 struct SelCfg {
@@ -132,17 +138,17 @@ __device__ __forceinline__ void red_shared_inc(uint32_t addr) {
   asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(addr) : "memory");
 }
 
-// Histogram pass over the raw float bits (the order-preserving key is applied to the bins, once
+// Histogram pass over the raw float bits (kCols consecutive candidates of a row per call) (the order-preserving key is applied to the bins, once
 // per row, when the histogram is read): count, in the row's 256 bins, the 8 raw bits at `shift`
 // of the scores whose resolved raw bits equal prefix (whose other bits are zero). With
 // x = (raw ^ prefix) >> shift, a matching score has x = its bin and any other x > 255, so
 // min(x, 256) sends the others to the row's spare slot: every lane stays active. Adding +0.0
 // first makes -0.0 the same score as +0.0. kFull: all 64 candidates exist (else only q < lim).
 template <bool kFull, bool kFirst>
-__device__ __forceinline__ void hist_chunk(const uint32_t (&v)[64], int lim, uint32_t prefix, int shift,
+__device__ __forceinline__ void hist_chunk(const uint32_t (&v)[kCols], int lim, uint32_t prefix, int shift,
                                            uint32_t hbase) {
 #pragma unroll
-  for (int q = 0; q < 64; ++q) {
+  for (int q = 0; q < kCols; ++q) {
     const uint32_t raw = __float_as_uint(__uint_as_float(v[q]) + 0.0f);
     uint32_t x = kFirst ? raw >> 24 : min((raw ^ prefix) >> shift, (uint32_t)kTrash);
     if (!kFull) x = q < lim ? x : (uint32_t)kTrash;
@@ -164,7 +170,7 @@ __device__ __forceinline__ int raw_bin(int kb, bool first, bool neg) {
 }
 
 // v[q] for a run-time q, keeping the array in registers (used only for the rare bucket keys)
-__device__ __forceinline__ uint32_t pick64(const uint32_t (&v)[64], int q) {
+__device__ __forceinline__ uint32_t pick32(const uint32_t (&v)[kCols], int q) {
   switch (q) {
     case 0: return v[0];
     case 1: return v[1];
@@ -198,62 +204,30 @@ __device__ __forceinline__ uint32_t pick64(const uint32_t (&v)[64], int q) {
     case 29: return v[29];
     case 30: return v[30];
     case 31: return v[31];
-    case 32: return v[32];
-    case 33: return v[33];
-    case 34: return v[34];
-    case 35: return v[35];
-    case 36: return v[36];
-    case 37: return v[37];
-    case 38: return v[38];
-    case 39: return v[39];
-    case 40: return v[40];
-    case 41: return v[41];
-    case 42: return v[42];
-    case 43: return v[43];
-    case 44: return v[44];
-    case 45: return v[45];
-    case 46: return v[46];
-    case 47: return v[47];
-    case 48: return v[48];
-    case 49: return v[49];
-    case 50: return v[50];
-    case 51: return v[51];
-    case 52: return v[52];
-    case 53: return v[53];
-    case 54: return v[54];
-    case 55: return v[55];
-    case 56: return v[56];
-    case 57: return v[57];
-    case 58: return v[58];
-    case 59: return v[59];
-    case 60: return v[60];
-    case 61: return v[61];
-    case 62: return v[62];
-    case 63: return v[63];
     default: return 0u;
   }
 }
 
-// Emit pass, 64 consecutive candidates of a row: bits of the taken keys (key >= thr) in tb and,
+// Emit pass, kCols consecutive candidates of a row: bits of the taken keys (key >= thr) in tb and,
 // with kBucket, of the bucket keys (blo <= key <= blo + bw) in bb. ALU only. kPos (thr above the
 // key of +0.0, and blo at or above it): the comparisons run on the raw float bits, which order
 // the non-negative scores as their keys do and put every negative score (and -0.0) below thr and
 // outside the bucket.
 template <bool kFull, bool kBucket, bool kPos>
-__device__ __forceinline__ void emit_bits(const uint32_t (&v)[64], int lim, uint32_t thr, uint32_t blo, uint32_t bw,
-                                          uint32_t (&tb)[2], uint32_t (&bb)[2]) {
+__device__ __forceinline__ void emit_bits(const uint32_t (&v)[kCols], int lim, uint32_t thr, uint32_t blo, uint32_t bw,
+                                          uint32_t& tb, uint32_t& bb) {
   const int thr_raw = (int)(thr ^ 0x80000000u);
   const uint32_t blo_raw = blo ^ 0x80000000u;
 #pragma unroll
-  for (int q = 0; q < 64; ++q) {
+  for (int q = 0; q < kCols; ++q) {
     const bool in = kFull || q < lim;
     if (kPos) {
-      tb[q >> 5] |= (in && (int)v[q] >= thr_raw) ? (1u << (q & 31)) : 0u;
-      if (kBucket) bb[q >> 5] |= (in && v[q] - blo_raw <= bw) ? (1u << (q & 31)) : 0u;
+      tb |= (in && (int)v[q] >= thr_raw) ? (1u << q) : 0u;
+      if (kBucket) bb |= (in && v[q] - blo_raw <= bw) ? (1u << q) : 0u;
     } else {
       const uint32_t key = score_key(__uint_as_float(v[q]));
-      tb[q >> 5] |= (in && key >= thr) ? (1u << (q & 31)) : 0u;
-      if (kBucket) bb[q >> 5] |= (in && key - blo <= bw) ? (1u << (q & 31)) : 0u;
+      tb |= (in && key >= thr) ? (1u << q) : 0u;
+      if (kBucket) bb |= (in && key - blo <= bw) ? (1u << q) : 0u;
     }
   }
 }
@@ -267,7 +241,7 @@ __device__ __forceinline__ uint32_t first_bits(uint32_t x, int n) {
   return x & ((1u << __fns(x, 0u, n + 1)) - 1u);
 }
 
-// Per-lane bounded wait for the partner half's tie count of a tile: the slot holds
+// Per-lane bounded wait for another part's tie count of a tile: the slot holds
 // (tile + 1) << 8 | count once written. Returns the count, or -1 on giving up.
 __device__ __forceinline__ int wait_tie_count(volatile uint32_t* slot, uint32_t tag, SelShared* sh,
                                               const int* gstatus) {
@@ -419,10 +393,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ---------------- epilogue: one row per thread pair ----------------
-    // Warps w and w + 4 read TMEM lane quadrant w % 4 (row r = 32 * (w % 4) + lane); each takes
-    // half of every tile's columns, in the histogram passes and in the emit pass.
-    const int quad = warp & 3, half = warp >> 2;
+    // ---------------- epilogue: one row per four threads ----------------
+    // Warps w, w + 4, w + 8, w + 12 read TMEM lane quadrant w % 4 (row r = 32 * (w % 4) + lane);
+    // warp w takes columns 32 * (w / 4) .. + 31 of every tile, in the histogram passes and in
+    // the emit pass.
+    const int quad = warp & 3, part = warp >> 2;
     const int r = quad * 32 + lane;
     const int t = tq0 + r / G, g = r % G;
     const bool valid = t <= t_last;
@@ -446,10 +421,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int pass = 0; pass < kMaxPasses; ++pass) {
       // zero the histograms for this pass (a resolved row: its tie-count slots), then a
       // barrier+vote: is any row still unresolved?
-      if (half == 0 && !done && pass < kMaxPasses - 1)
+      if (part == 0 && !done && pass < kMaxPasses - 1)
         for (int i = 0; i < 256; ++i) my_hist[i * kRows] = 0;
-      if (half == 0 && done)
-        for (int i = 0; i < 4; ++i) my_hist[i * kRows] = 0;
+      if (part == 0 && done)
+        for (int i = 0; i < kTieWords; ++i) my_hist[i * kRows] = 0;
       const int vote = epi_vote_any(sh, 4 * pass, !done, a.status);
       // from the third pass on, if every unresolved row's threshold bucket is small, this pass is
       // the last: it also collects those buckets' keys, which are then resolved exactly
@@ -480,13 +455,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc::fence_after_sync();
-          uint32_t v[64];
-          tc::tmem_ld64(tmem + lane_base + (uint32_t)(buf * kN + half * 64), v);
+          uint32_t v[kCols];
+          tc::tmem_ld32(tmem + lane_base + (uint32_t)(buf * kN + part * kCols), v);
           tc::fence_before_sync();
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(&sh->acc_empty[buf]);
-          const int lim = c - (i * kN + half * 64);
-          if (__all_sync(0xFFFFFFFFu, lim >= 64)) {
+          const int lim = c - (i * kN + part * kCols);
+          if (__all_sync(0xFFFFFFFFu, lim >= kCols)) {
             if (pass == 0) hist_chunk<true, true>(v, lim, pf, shift, hbase);
             else hist_chunk<true, false>(v, lim, pf, shift, hbase);
           } else if (lim > 0) {
@@ -495,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (aborted) break;
-        // both halves' histogram updates are complete before either reads the histogram
+        // every part's histogram updates are complete before any reads the histogram
         if (epi_vote_any(sh, 4 * pass + 1, false, a.status) < 0) {
           if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
           sh->abort_flag = 1;
@@ -517,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           done = (rem == nb) || (mask == 0xFFFFFFFFu);
         }
-        // both halves have read the histogram before the next pass zeroes it
+        // every part has read the histogram before the next pass zeroes it
         if (epi_vote_any(sh, 4 * pass + 2, false, a.status) < 0) {
           if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
           sh->abort_flag = 1;
@@ -527,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
 
-      // ---- emit pass: this half's 64 columns of every tile become two bitmap words ----
+      // ---- emit pass: this part's kCols columns of every tile become one bitmap word ----
       // rule of this row: take keys >= thr; the bucket [blo, blo + bw] is collected (unresolved
       // row), taken whole (thr = prefix), or holds exact ties taken in j order up to rem
       const bool act = valid && m > 0;
@@ -548,14 +523,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           ties = true;
         }
       }
-      // identical in the two warps of a row pair (same rows, same state)
+      // identical in the kParts warps of a row group (same rows, same state)
       const bool any_bucket = __any_sync(0xFFFFFFFFu, collect || ties);
       // every row of the warp has a positive threshold (and bucket): raw-bit comparisons
       const bool pos = __all_sync(0xFFFFFFFFu, thr > 0x80000000u && blo >= 0x80000000u);
       const bool any_ties = __any_sync(0xFFFFFFFFu, ties);
-      uint32_t* cand = my_hist + 128 * half * kRows;  // collected (key, j) pairs of this half (stride kRows)
-      volatile uint32_t* slot = my_hist;              // tie counts: [half][tile parity] (stride kRows)
-      int run = 0;                            // exact ties before this half's columns of the tile
+      uint32_t* cand = my_hist + part * kCandWords * kRows;  // this part's collected (key, j) pairs (stride kRows)
+      volatile uint32_t* slot = my_hist;                     // tie counts: [part][tile parity] (stride kRows)
+      int run = 0;  // exact ties before this part's columns of the tile
       for (int i = 0; i < n_nt; ++i, ++k) {
         const int buf = (int)(k & 1);
         if (!warp_wait(&sh->acc_full[buf], (uint32_t)((k >> 1) & 1), &sh->abort_flag, a.status)) {
@@ -565,13 +540,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc::fence_after_sync();
-        const int j0 = i * kN + half * 64;
+        const int j0 = i * kN + part * kCols;
         const int lim = act ? c - j0 : 0;
-        uint32_t tb[2] = {0u, 0u}, bb[2] = {0u, 0u};
+        uint32_t tb = 0u, bb = 0u;
         if (__any_sync(0xFFFFFFFFu, lim > 0)) {
-          uint32_t v[64];
-          tc::tmem_ld64(tmem + lane_base + (uint32_t)(buf * kN + half * 64), v);
-          const bool full = __all_sync(0xFFFFFFFFu, lim >= 64);
+          uint32_t v[kCols];
+          tc::tmem_ld32(tmem + lane_base + (uint32_t)(buf * kN + part * kCols), v);
+          const bool full = __all_sync(0xFFFFFFFFu, lim >= kCols);
           if (any_bucket) {
             if (full && pos) emit_bits<true, true, true>(v, lim, thr, blo, bw, tb, bb);
             else if (full) emit_bits<true, true, false>(v, lim, thr, blo, bw, tb, bb);
@@ -582,18 +557,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             else emit_bits<false, false, false>(v, lim, thr, blo, bw, tb, bb);
           }
           if (collect) {  // the few bucket keys of an unresolved row, kept as (key, j) pairs
-#pragma unroll
-            for (int w = 0; w < 2; ++w) {
-              uint32_t bits = bb[w];
-              while (bits) {
-                const int q = __ffs(bits) - 1;
-                bits &= bits - 1u;
-                if (eqn < kCap) {
-                  cand[(2 * eqn) * kRows] = score_key(__uint_as_float(pick64(v, 32 * w + q)));
-                  cand[(2 * eqn + 1) * kRows] = (uint32_t)(j0 + 32 * w + q);
-                }
-                ++eqn;
+            uint32_t bits = bb;
+            while (bits) {
+              const int q = __ffs(bits) - 1;
+              bits &= bits - 1u;
+              if (eqn < kCap) {
+                cand[(2 * eqn) * kRows] = score_key(__uint_as_float(pick32(v, q)));
+                cand[(2 * eqn + 1) * kRows] = (uint32_t)(j0 + q);
               }
+              ++eqn;
             }
           }
         }
@@ -601,19 +573,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&sh->acc_empty[buf]);
         if (any_ties) {
-          // exact ties in j order: the lower half's columns of tile i precede the upper half's
-          const int cnt = ties ? __popc(bb[0]) + __popc(bb[1]) : 0;
+          // exact ties in j order: in tile i the parts' columns run part 0, 1, ..., so a part
+          // counts the ties of the lower parts in tile i and of the higher parts in tile i - 1
+          // (its own and all earlier tiles are already in run). Each part publishes its count
+          // for tile i before it waits, so the waits only reach back to earlier publications.
+          const int cnt = ties ? __popc(bb) : 0;
           int got = 0;
-          if (half == 0) {
-            if (ties) slot[(i & 1) * kRows] = ((uint32_t)(i + 1) << 8) | (uint32_t)cnt;
-            if (ties && i > 0) {
-              got = wait_tie_count(slot + (2 + ((i - 1) & 1)) * kRows, (uint32_t)i, sh, a.status);
-              run += got;
+          if (ties) {
+            slot[(2 * part + (i & 1)) * kRows] = ((uint32_t)(i + 1) << 8) | (uint32_t)cnt;
+            for (int q = 0; q < kParts && got >= 0; ++q) {
+              if (q == part || (q > part && i == 0)) continue;
+              const int ti = q < part ? i : i - 1;
+              const int x = wait_tie_count(slot + (2 * q + (ti & 1)) * kRows, (uint32_t)(ti + 1), sh, a.status);
+              if (x < 0) got = -1;
+              else run += x;
             }
-          } else if (ties) {
-            got = wait_tie_count(slot + (i & 1) * kRows, (uint32_t)(i + 1), sh, a.status);
-            run += got;
-            slot[(2 + (i & 1)) * kRows] = ((uint32_t)(i + 1) << 8) | (uint32_t)cnt;
           }
           if (__any_sync(0xFFFFFFFFu, got < 0)) {
             if (lane == 0 && !sh->abort_flag) report(a.status, SGQA_ERR_TIMEOUT);
@@ -622,45 +596,55 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           if (ties) {
-            const int n = rem - run;
-            tb[0] |= first_bits(bb[0], n);
-            tb[1] |= first_bits(bb[1], n - __popc(bb[0]));
+            tb |= first_bits(bb, rem - run);
             run += cnt;
           }
         }
-        if (lim > 0 && SGQA_CHECK((j0 >> 5) + 1 < a.bstride && t < a.t_end, a.status))
-          *reinterpret_cast<uint2*>(brow + (j0 >> 5)) = make_uint2(tb[0], tb[1]);
-        taken += __popc(tb[0]) + __popc(tb[1]);
+        if (lim > 0 && SGQA_CHECK((j0 >> 5) < a.bstride && t < a.t_end, a.status)) brow[j0 >> 5] = tb;
+        taken += __popc(tb);
       }
-      if (!aborted && half == 1 && act) {
-        my_hist[kCnt1 * kRows] = (uint32_t)eqn;
-        my_hist[(kCnt1 + 1) * kRows] = (uint32_t)taken;
+      if (!aborted && part > 0 && act) {
+        my_hist[(kCntBase + 2 * (part - 1)) * kRows] = (uint32_t)eqn;
+        my_hist[(kCntBase + 2 * (part - 1) + 1) * kRows] = (uint32_t)taken;
       }
       emitted = !aborted;
       break;
     }
     // every epilogue warp gets here (all waits above are bounded): the bitmap words and the
-    // collected keys of both halves are complete
+    // collected keys of all parts are complete
     asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
-    if (emitted && half == 0 && act_row(valid, m) && !sh->abort_flag) {
-      int total = taken + (int)my_hist[(kCnt1 + 1) * kRows];
+    if (emitted && part == 0 && act_row(valid, m) && !sh->abort_flag) {
+      int total = taken;
+      int ncol[kParts];
+      ncol[0] = eqn;
+#pragma unroll
+      for (int p = 1; p < kParts; ++p) {
+        total += (int)my_hist[(kCntBase + 2 * (p - 1) + 1) * kRows];
+        ncol[p] = (int)my_hist[(kCntBase + 2 * (p - 1)) * kRows];
+      }
       if (collect) {
-        // the collected bucket keys of both halves: key x ranks behind every larger key and every
+        // the collected bucket keys of all parts: key x ranks behind every larger key and every
         // equal key of lower j, and is taken when fewer than rem rank ahead of it
-        const int e1 = (int)my_hist[kCnt1 * kRows];
-        if (eqn > kCap || e1 > kCap) report(a.status, SGQA_ERR_DEVICE_CHECK);
-        const int n0 = min(eqn, kCap), n1 = min(e1, kCap);
-        for (int x = 0; x < n0 + n1; ++x) {
-          const uint32_t* px = my_hist + (x < n0 ? 2 * x : 128 + 2 * (x - n0)) * kRows;
-          const uint32_t kx = px[0], jx = px[kRows];
-          int ahead = 0;
-          for (int y = 0; y < n0 + n1; ++y) {
-            const uint32_t* py = my_hist + (y < n0 ? 2 * y : 128 + 2 * (y - n0)) * kRows;
-            ahead += (py[0] > kx || (py[0] == kx && py[kRows] < jx)) ? 1 : 0;
-          }
-          if (ahead < rem && SGQA_CHECK(jx < (uint32_t)c && (int)(jx >> 5) < a.bstride, a.status)) {
-            atomicOr(brow + (jx >> 5), 1u << (jx & 31u));
-            ++total;
+#pragma unroll
+        for (int p = 0; p < kParts; ++p) {
+          if (ncol[p] > kCap) report(a.status, SGQA_ERR_DEVICE_CHECK);
+          ncol[p] = min(ncol[p], kCap);
+        }
+        for (int px = 0; px < kParts; ++px) {
+          for (int x = 0; x < ncol[px]; ++x) {
+            const uint32_t* cx = my_hist + (px * kCandWords + 2 * x) * kRows;
+            const uint32_t kx = cx[0], jx = cx[kRows];
+            int ahead = 0;
+            for (int py = 0; py < kParts; ++py) {
+              for (int y = 0; y < ncol[py]; ++y) {
+                const uint32_t* cy = my_hist + (py * kCandWords + 2 * y) * kRows;
+                ahead += (cy[0] > kx || (cy[0] == kx && cy[kRows] < jx)) ? 1 : 0;
+              }
+            }
+            if (ahead < rem && SGQA_CHECK(jx < (uint32_t)c && (int)(jx >> 5) < a.bstride, a.status)) {
+              atomicOr(brow + (jx >> 5), 1u << (jx & 31u));
+              ++total;
+            }
           }
         }
       }
@@ -785,7 +769,7 @@ cudaError_t launch_di(const SelectArgs& a, cudaStream_t s) {
 
 void select_bits_dims(int batch, int T, int G, int B, size_t budget, int* bstride, int* bits_q) {
   const long nblk = T / B;
-  *bstride = (int)(4 * ((nblk + kN - 1) / kN));  // whole tiles: a tile's two words per half stay in the row
+  *bstride = (int)(4 * ((nblk + kN - 1) / kN));  // whole tiles: a tile's word per part stays in the row
   const size_t per_q = (size_t)batch * G * (size_t)*bstride * 4;
   long q = per_q ? (long)(budget / per_q) : (long)T;
   q = q / 128 * 128;  // whole K2 tiles (128 / G tokens) per range
