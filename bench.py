@@ -46,7 +46,7 @@ CLOCK_FIELDS = ["pci.bus_id", "clocks.sm", "clocks.max.sm", "power.draw", "clock
 NCU_TRAFFIC: dict = {
     # profiles/traffic_prefill128k_decode1m.md, the bench's own 128K / 1M workloads
     ("attend", "128k"): (6508516608 + 1068875008, "0ae683a6e388e866"),   # one attend_tc launch
-    ("select", "128k"): (96827136 + 350853632 + 311874560 + 824761856, "4eb4b3b9e3b6ade2"),  # 4 select_tc + 4 sel_from_bits
+    ("select", "128k"): (96827136 + 350853632 + 311874560 + 824761856, "4c4c0517e456e378"),  # 4 select_tc + 4 sel_from_bits
     ("decode_scores", "decode_1m"): (1074967296 + 252742400, "0669c7900a2898e8"),
     ("decode_select", "decode_1m"): (45581824 + 512, "cc7074bb7dae8bdd"),
     ("decode_attend", "decode_1m"): (1072768256 + 274176, "f4009ea09891d2e4"),

@@ -17,12 +17,13 @@
 //
 // Warp roles: warp 16 issues TMA loads, warp 17 allocates TMEM and issues MMAs, warps 0-15 are
 // the epilogue, four per TMEM lane quadrant (TMEM lane = row); each of the four takes a quarter
-// (32 columns) of every tile, so that every scheduler interleaves four epilogue warps. The epilogue performs an exact radix select of the m-th largest order-preserving
-// 32-bit score key per row: every pass re-streams the same score tiles (recomputed,
-// bit-identical); in a histogram pass each thread adds its keys that still match the resolved
-// prefix to the row's 256-bin shared histogram of the next 8 key bits (keys that do not match go
-// to a spare slot of the row, so the shared-memory reductions stay branch-free and mostly free of
-// bank conflicts). Once every row's threshold bucket is resolved or taken whole, the emit pass
+// (32 columns) of every tile, so that every scheduler interleaves four epilogue warps. The
+// epilogue performs an exact radix select of the m-th largest order-preserving 32-bit score key
+// per row: every pass re-streams the same score tiles (recomputed, bit-identical); in a histogram
+// pass each thread adds its scores that still match the resolved prefix to the row's 256-bin
+// shared histogram of the next 8 bits, counted on the raw float bits and read back in key order
+// (scores that do not match go to a spare slot of the row, so the shared-memory reductions stay
+// branch-free and free of bank conflicts). Once every row's threshold bucket is resolved or taken whole, the emit pass
 // marks the taken candidates of each 32-column quarter-tile in one 32-bit word and stores it to
 // the row's bitmap in global memory: keys above the threshold; bucket keys taken whole; exact ties
 // in j order (the four threads of a row exchange their tie counts through shared memory, so ties
