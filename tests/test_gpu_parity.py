@@ -559,3 +559,13 @@ def test_full_size_decode_1m_sampled():
     cfg = CONFIGS["decode_1m"]
     errs = _decode_case(cfg, cfg.T, DECODE_NEW, [0, 5, 9, 14, 18, 23, 27, 31])
     print(f"decode 1M: {errs}")
+
+
+def test_decode_cache_beyond_4096_candidate_groups():
+    """A cache of 1.2M tokens (B = 8): rows of more than 4096 groups of 32 candidates, which the
+    decode select lists in several chunks."""
+    cfg = CONFIGS["decode_1m"].replace(batch=2)
+    cache_len = 1258288
+    assert (cache_len // cfg.B + 31) // 32 > 4096
+    errs = _decode_case(cfg, cache_len, DECODE_NEW, [0, 1])
+    print(f"decode 1.2M: {errs}")
