@@ -223,6 +223,32 @@ def test_exact_ties_go_to_lower_blocks():
             np.testing.assert_array_equal(got[b, :, g], want)
 
 
+def test_zero_scores_tie_to_lower_blocks():
+    """Nine blocks in ten have all-zero index keys, so most scores are exactly zero (the tensor
+    cores may give +0.0 or -0.0, depending on the signs of the products) and many rows' m-th best
+    score is 0: the zeros are one score, tied, and go to the lower block indices. The selections
+    must equal the oracle's exactly (at s_m = 0 the near-tie rule would excuse any order)."""
+    cfg = Config("zeros", 1, 2048, 8, 2, 64, 32, 8, 512, 256, 25)
+    dims = sg.sgqa_dims.of(cfg)
+    k_idx = gen_full(cfg, "k_idx").reshape(shape_of(cfg, "k_idx")).copy()
+    blocks = np.arange(cfg.T) // cfg.B
+    k_idx[:, blocks % 10 != 0] = 0  # bf16 +0.0
+    q_h = gen_full(cfg, "q_idx").reshape(shape_of(cfg, "q_idx"))
+    kbar = torch.empty((cfg.batch, cfg.T // cfg.B, cfg.d_idx), device="cuda")
+    sg.sgqa_compress_keys(dims, to_dev(k_idx, shape_of(cfg, "k_idx")), kbar, None)
+    ws = _ws(dims)
+    sel = torch.full((cfg.batch, cfg.T, cfg.G, cfg.Kb), -7, dtype=torch.int32, device="cuda")
+    sg.sgqa_select(dims, to_dev(q_h, shape_of(cfg, "q_idx")), kbar, sel, ws)
+    _status_ok(ws)
+    dm = oracle.dims_of(cfg)
+    kbar64 = oracle.compress(dm, k_idx)
+    rows = all_rows(cfg)
+    sel_o, s_m, _ = oracle.select(dm, kbar64, rows, q_h.reshape(len(rows), -1))
+    chosen = np.asarray(rows)[:, 1] // cfg.B > cfg.Kb - 1  # rows that choose among their candidates
+    assert np.sum(s_m[chosen] == 0) > 500  # the case is exercised
+    np.testing.assert_array_equal(sel.cpu().numpy().reshape(sel_o.shape), sel_o)
+
+
 def test_causality_on_gpu():
     cfg = Config("causal", 1, 2500, 8, 2, 64, 32, 8, 256, 300, 15)
     dims = sg.sgqa_dims.of(cfg)
