@@ -137,6 +137,20 @@ def forward_launches(cfg, nq: int) -> int:
     return 1 + 2 * select_ranges(cfg, nq) + 10 + 1
 
 
+def decode_launches(cfg, n_new: int, cache_len: int, fp8: bool) -> int:
+    """Library kernel launches of one decode step (api.cu, sgqa_decode): the appends (K and V
+    quantized for FP8 caches, k_idx), the block means when the new rows complete a block, K4, K5,
+    the union, K6 and, when K6 splits a (sequence, group), the merge. K6 takes one wave of
+    148 x (1 CTA per SM for FP8 caches, 2 for bf16) CTAs, split over the (sequence, group) units
+    up to the union's 128-token tiles (decode_attend.cu, decode_attend_splits)."""
+    appends = 3
+    compress = 1 if (cache_len + n_new) // cfg.B > cache_len // cfg.B else 0
+    units = cfg.batch * cfg.G
+    max_tiles = -(-(n_new * cfg.Kb) // (128 // cfg.B))
+    splits = min(max(1, 148 * (1 if fp8 else 2) // units), max_tiles)
+    return appends + compress + 4 + (1 if splits > 1 else 0)
+
+
 def select_alu_model(wc, sm_mhz):
     """Time the select's per-key epilogue work needs at full issue rate (148 SMs x 4 schedulers x
     32 lanes x clock): a kernel-specific ceiling, reported beside the tensor roofline."""
@@ -602,7 +616,7 @@ def run_decode(args, world, s):
            "hbm_frac": (kbar_bytes + gather) / (ms / 1e3) / 1e9 / load_peaks()["hbm_gbs"],
            "kernel_traffic_bytes": {k: measured_traffic(k, "decode_1m")
                                     for k in ("decode_scores", "decode_select", "decode_attend")},
-           "gpu_launches_per_step": 7}  # append x3, scores, select, union, attend
+           "gpu_launches_per_step": decode_launches(cfg, n_new, cache_len, False)}
     del caches, kbar, new, out, ws
     torch.cuda.empty_cache()
     return res
@@ -676,7 +690,7 @@ def run_decode_fp8(args, world, s):
                        f"seed {cfg.seed}",
            "algorithmic_bytes": kbar_bytes + gather,
            "hbm_frac": (kbar_bytes + gather) / (ms / 1e3) / 1e9 / load_peaks()["hbm_gbs"],
-           "gpu_launches_per_step": 8}
+           "gpu_launches_per_step": decode_launches(cfg, n_new, cache_len, True)}
     del c8, csc, kidx, kbar, new, out, ws
     torch.cuda.empty_cache()
     return res

@@ -40,3 +40,17 @@ def test_counts_at_128k():
     assert wc["gather_bytes"] == pytest.approx(1.08e12, rel=3e-3)
     # compulsory DRAM bytes of the attention: q, gate, out; the selection; K and V once
     assert wc["qgo_bytes"] + wc["sel_bytes"] + wc["kv_bytes"] == 4563402752
+
+
+def test_decode_launch_counts():
+    """Decode steps at the 1M workload: bf16 caches split each (sequence, group) over two CTAs
+    and merge (8 launches: 3 appends, K4, K5, union, K6, merge); FP8 caches run one CTA per unit
+    with no merge (7: 2 quantizing appends, the k_idx append, K4, K5, union, K6). The ncu launch
+    list of the bench shows the merge kernel once per bf16 step only. A step whose new rows
+    complete a block adds the block means."""
+    cfg = CONFIGS["decode_1m"]
+    assert bench.decode_launches(cfg, 4, cfg.T, fp8=False) == 8
+    assert bench.decode_launches(cfg, 4, cfg.T, fp8=True) == 7
+    assert bench.decode_launches(cfg, 4, cfg.T + 4, fp8=True) == 8  # completes block (T + 8) / 8 - 1
+    one = cfg.replace(batch=1)
+    assert bench.decode_launches(one, 4, cfg.T, fp8=True) == 8      # 4 units: K6 splits, merge
